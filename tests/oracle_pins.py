@@ -1,0 +1,297 @@
+"""Checks that pin the fp64 oracle to facts fixed outside itself.
+
+Each ``pin_*`` function takes an oracle front end (``oracle.Oracle``) and
+raises AssertionError when it disagrees with a closed form, an invariant the
+lecture page states, finite differences, a library special case or a worked
+fixture.  ``tests/test_oracle.py`` runs them against the real oracle;
+``tests/test_oracle_mutants.py`` compiles deliberately broken copies of the
+oracle and checks that every planted mistake trips at least one pin.
+
+Page cited throughout: "Let's build GPT: from scratch, in code, spelled out"
+(the lecture page with the chapter list and corrections).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _split(qkv, n_head):
+    """View qkv[B,T,3C] as q, k, v of shape [B, n_head, T, hs] (heads as a batch dim)."""
+    B, T, C3 = qkv.shape
+    C = C3 // 3
+    hs = C // n_head
+    x = qkv.reshape(B, T, 3, n_head, hs)
+    return [np.ascontiguousarray(x[:, :, i].transpose(0, 2, 1, 3)) for i in range(3)]
+
+
+def pin_single_token(orc):
+    """T=1: a token sees only itself, so its weight is exactly 1 and y = v;
+    lse is the one visible score q.k / sqrt(hs) (chapter 'version 4')."""
+    B, n_head, hs = 3, 2, 8
+    C = n_head * hs
+    qkv = _rng(1).standard_normal((B, 1, 3 * C))
+    y, lse = orc.forward(qkv, n_head)
+    assert np.array_equal(y, qkv[:, :, 2 * C:]), "T=1 must return V exactly"
+    q, k, _ = _split(qkv, n_head)
+    score = (q * k).sum(-1) / math.sqrt(hs)          # [B, nh, 1]
+    assert np.allclose(lse, score, rtol=0, atol=1e-14)
+
+
+def pin_uniform_scores_prefix_mean(orc):
+    """Zero queries make every score equal: the weights become the lecture's
+    version-1 average of the past context, y[t] = mean(v_0..v_t), and the
+    normaliser is t+1 (lse = ln(t+1))."""
+    B, T, n_head, hs = 2, 19, 3, 5
+    C = n_head * hs
+    qkv = _rng(2).standard_normal((B, T, 3 * C))
+    qkv[:, :, :C] = 0.0
+    y, lse = orc.forward(qkv, n_head)
+    v = qkv[:, :, 2 * C:]
+    for b in range(B):
+        for t in range(T):
+            acc = np.zeros(C)
+            for s in range(t + 1):       # version 1: a for loop over the past
+                acc += v[b, s]
+            assert np.allclose(y[b, t], acc / (t + 1), rtol=0, atol=1e-13)
+    expect = np.log(np.arange(1, T + 1, dtype=np.float64))
+    assert np.allclose(lse, np.broadcast_to(expect, lse.shape), rtol=0, atol=1e-14)
+
+
+def pin_tril_average_fixture(orc):
+    """Golden fixture: with equal affinities the weights are the
+    lower-triangular averaging matrix of chapters 'version 2'/'version 3'.
+    One-hot values (v_s = e_s) expose the weights in y."""
+    fx = json.load(open(os.path.join(GOLDEN, "tril_average_T5.json")))
+    T = fx["T"]
+    W = np.array([[float(eval(x)) for x in row] for row in fx["weights_exact"]])  # fractions like "1/3"
+    n_head, hs = 1, T
+    C = hs
+    qkv = np.zeros((1, T, 3 * C))
+    qkv[0, :, 2 * C:] = np.eye(T)
+    qkv[0, :, C:2 * C] = _rng(3).standard_normal((T, C))   # keys are irrelevant when q = 0
+    y, _ = orc.forward(qkv, n_head)
+    assert np.allclose(y[0], W, rtol=0, atol=1e-15)
+    P = orc.probs(qkv, n_head, 0, 0)
+    assert np.allclose(P, W, rtol=0, atol=1e-15)
+
+
+def pin_rows_are_distributions(orc):
+    """Softmax rows sum to one, the future (s > t) has weight exactly zero and
+    the diagonal is visible (correction to 00:57:00: the future cannot
+    communicate; a token is not in its own future)."""
+    B, T, n_head, hs = 2, 23, 2, 6
+    C = n_head * hs
+    qkv = 2.0 * _rng(4).standard_normal((B, T, 3 * C))
+    for b in range(B):
+        for h in range(n_head):
+            P = orc.probs(qkv, n_head, b, h)
+            assert np.allclose(P.sum(1), 1.0, rtol=0, atol=1e-14)
+            assert np.all(P[np.triu_indices(T, 1)] == 0.0)
+            assert np.all(np.diag(P) > 0.0)
+            assert np.all(P >= 0.0)
+
+
+def pin_weights_from_softmax_of_scaled_scores(orc):
+    """Brute force on a tiny case: each weight is exp(score)/sum over the
+    visible row, with score = q.k/sqrt(head_size) (note 6, correction to
+    01:20:05), evaluated one element at a time with Python floats."""
+    T, n_head, hs = 4, 2, 3
+    C = n_head * hs
+    qkv = _rng(5).standard_normal((1, T, 3 * C))
+    for h in range(n_head):
+        P = orc.probs(qkv, n_head, 0, h)
+        for t in range(T):
+            sc = []
+            for s in range(t + 1):
+                dot = sum(qkv[0, t, h * hs + d] * qkv[0, s, C + h * hs + d] for d in range(hs))
+                sc.append(dot / math.sqrt(hs))
+            den = sum(math.exp(x) for x in sc)
+            for s in range(t + 1):
+                assert abs(P[t, s] - math.exp(sc[s]) / den) < 1e-14
+
+
+def pin_worked_two_heads(orc):
+    """Golden fixture: a T=2, two-head case worked by hand (scale sqrt(hs) = 2,
+    not sqrt(C)); also recomputed here from its closed form."""
+    fx = json.load(open(os.path.join(GOLDEN, "worked_T2_two_heads.json")))
+    qkv = np.array(fx["qkv"])
+    y, lse = orc.forward(qkv, fx["n_head"])
+    assert np.allclose(y, np.array(fx["y"]), rtol=0, atol=1e-13)
+    assert np.allclose(lse, np.array(fx["lse"]), rtol=0, atol=1e-13)
+    # closed form of head 0 at t=1: weights (1, 3)/(1+3)
+    v0, v1 = qkv[0, 0, 16:20], qkv[0, 1, 16:20]
+    assert np.allclose(y[0, 1, 0:4], 0.25 * v0 + 0.75 * v1, rtol=0, atol=1e-13)
+
+
+def pin_causality(orc):
+    """Perturbing tokens after position t leaves everything at positions <= t
+    unchanged: y, lse and dq (the future cannot communicate)."""
+    B, T, n_head, hs = 2, 17, 2, 4
+    C = n_head * hs
+    r = _rng(6)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    y0, l0 = orc.forward(qkv, n_head)
+    g0 = orc.backward(qkv, dy, n_head)
+    for t in (0, 5, 11):
+        q2 = qkv.copy()
+        d2 = dy.copy()
+        q2[:, t + 1:] += r.standard_normal(q2[:, t + 1:].shape)
+        d2[:, t + 1:] += r.standard_normal(d2[:, t + 1:].shape)
+        y1, l1 = orc.forward(q2, n_head)
+        g1 = orc.backward(q2, d2, n_head)
+        assert np.array_equal(y1[:, :t + 1], y0[:, :t + 1])
+        assert np.array_equal(l1[:, :, :t + 1], l0[:, :, :t + 1])
+        assert np.array_equal(g1[:, :t + 1, :C], g0[:, :t + 1, :C])
+        assert not np.allclose(y1[:, t + 1:], y0[:, t + 1:])
+
+
+def pin_batch_independence(orc):
+    """No communication across the batch dimension (note 3)."""
+    B, T, n_head, hs = 3, 9, 2, 4
+    C = n_head * hs
+    r = _rng(7)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    y0, l0 = orc.forward(qkv, n_head)
+    g0 = orc.backward(qkv, dy, n_head)
+    q2, d2 = qkv.copy(), dy.copy()
+    q2[1] = r.standard_normal(q2[1].shape)
+    d2[1] = r.standard_normal(d2[1].shape)
+    y1, l1 = orc.forward(q2, n_head)
+    g1 = orc.backward(q2, d2, n_head)
+    for b in (0, 2):
+        assert np.array_equal(y1[b], y0[b]) and np.array_equal(l1[b], l0[b])
+        assert np.array_equal(g1[b], g0[b])
+
+
+def pin_head_permutation(orc):
+    """Heads are a batch dimension (exercise EX1): permuting the heads of q, k
+    and v together permutes the heads of y, lse and dqkv the same way."""
+    B, T, n_head, hs = 2, 11, 4, 3
+    C = n_head * hs
+    r = _rng(8)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    perm = np.array([2, 0, 3, 1])
+
+    def permute_cols(x, parts):
+        x = x.reshape(B, T, parts, n_head, hs)[:, :, :, perm]
+        return x.reshape(B, T, parts * C)
+
+    y0, l0 = orc.forward(qkv, n_head)
+    g0 = orc.backward(qkv, dy, n_head)
+    y1, l1 = orc.forward(permute_cols(qkv, 3), n_head)
+    g1 = orc.backward(permute_cols(qkv, 3), permute_cols(dy, 1), n_head)
+    assert np.array_equal(y1, permute_cols(y0, 1))
+    assert np.array_equal(l1, l0[:, perm])
+    assert np.array_equal(g1, permute_cols(g0, 3))
+
+
+def pin_set_semantics(orc):
+    """Attention has no notion of space (note 2): shuffling the tokens before
+    position t leaves y[t] and lse[t] unchanged."""
+    B, T, n_head, hs = 1, 12, 2, 5
+    C = n_head * hs
+    r = _rng(9)
+    qkv = r.standard_normal((B, T, 3 * C))
+    y0, l0 = orc.forward(qkv, n_head)
+    t = 9
+    perm = r.permutation(t)
+    q2 = qkv.copy()
+    q2[:, :t] = qkv[:, perm]
+    y1, l1 = orc.forward(q2, n_head)
+    assert np.allclose(y1[:, t], y0[:, t], rtol=0, atol=1e-13)
+    assert np.allclose(l1[:, :, t], l0[:, :, t], rtol=0, atol=1e-13)
+
+
+def pin_finite_differences(orc):
+    """The backward is the gradient of L = sum(y * dy): central differences in
+    fp64 (h = 1e-6) agree with it for every input element."""
+    for (B, T, n_head, hs, seed) in ((1, 5, 2, 4, 10), (1, 8, 1, 3, 11)):
+        C = n_head * hs
+        r = _rng(seed)
+        qkv = r.standard_normal((B, T, 3 * C))
+        G = r.standard_normal((B, T, C))
+        grad = orc.backward(qkv, G, n_head)
+        h = 1e-6
+        fd = np.zeros_like(qkv)
+        flat = qkv.reshape(-1)
+        for i in range(flat.size):
+            xp = flat.copy()
+            xm = flat.copy()
+            xp[i] += h
+            xm[i] -= h
+            yp, _ = orc.forward(xp.reshape(qkv.shape), n_head)
+            ym, _ = orc.forward(xm.reshape(qkv.shape), n_head)
+            fd.reshape(-1)[i] = ((yp * G).sum() - (ym * G).sum()) / (2 * h)
+        err = np.abs(fd - grad).max() / np.abs(grad).max()
+        assert err < 1e-6, f"finite-difference mismatch {err:.3e}"
+
+
+def pin_library_special_case(orc):
+    """A different implementation of the same function: PyTorch's
+    scaled_dot_product_attention(is_causal=True) and autograd, in fp64 on
+    the CPU (its default scale is 1/sqrt(head_size))."""
+    B, T, n_head, hs = 2, 37, 3, 8
+    C = n_head * hs
+    r = _rng(12)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    x = torch.tensor(qkv, dtype=torch.float64, requires_grad=True)
+    q, k, v = x.split(C, dim=2)
+    heads = lambda a: a.view(B, T, n_head, hs).transpose(1, 2)
+    out = torch.nn.functional.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=True)
+    y_ref = out.transpose(1, 2).reshape(B, T, C)
+    (y_ref * torch.tensor(dy)).sum().backward()
+    y, lse = orc.forward(qkv, n_head)
+    g = orc.backward(qkv, dy, n_head)
+    assert np.abs(y - y_ref.detach().numpy()).max() < 1e-12
+    assert np.abs(g - x.grad.numpy()).max() < 1e-12
+    # lse against torch.logsumexp of the masked scaled scores
+    qh, kh = heads(q).detach(), heads(k).detach()
+    s = qh @ kh.transpose(-1, -2) / math.sqrt(hs)
+    s = s.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), float("-inf"))
+    assert np.abs(lse - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+def pin_regression_fixture(orc):
+    """Regression fixture written by tests/golden/make_golden.py from this
+    oracle: catches any later change to the oracle's arithmetic."""
+    fx = json.load(open(os.path.join(GOLDEN, "oracle_small_seeded.json")))
+    qkv, dy = np.array(fx["qkv"]), np.array(fx["dy"])
+    y, lse = orc.forward(qkv, fx["n_head"])
+    g = orc.backward(qkv, dy, fx["n_head"])
+    assert np.allclose(y, fx["y"], rtol=0, atol=1e-13)
+    assert np.allclose(lse, fx["lse"], rtol=0, atol=1e-13)
+    assert np.allclose(g, fx["dqkv"], rtol=0, atol=1e-13)
+
+
+def pin_empty(orc):
+    """Empty batch or sequence: nothing to compute, shapes preserved."""
+    y, lse = orc.forward(np.zeros((0, 4, 12)), 2)
+    assert y.shape == (0, 4, 4) and lse.shape == (0, 2, 4)
+    y, lse = orc.forward(np.zeros((2, 0, 12)), 2)
+    assert y.shape == (2, 0, 4) and lse.shape == (2, 2, 0)
+    g = orc.backward(np.zeros((2, 0, 12)), np.zeros((2, 0, 4)), 2)
+    assert g.shape == (2, 0, 12)
+
+
+ALL_PINS = [
+    pin_single_token, pin_uniform_scores_prefix_mean, pin_tril_average_fixture,
+    pin_rows_are_distributions, pin_weights_from_softmax_of_scaled_scores,
+    pin_worked_two_heads, pin_causality, pin_batch_independence, pin_head_permutation,
+    pin_set_semantics, pin_finite_differences, pin_library_special_case,
+    pin_regression_fixture, pin_empty,
+]

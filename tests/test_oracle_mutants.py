@@ -1,0 +1,57 @@
+"""Plant plausible mistakes in copies of the oracle (on the CPU) and check that
+each one trips at least one pin -- evidence that the pins constrain every
+step: the scale, the mask, the softmax shift, operand order and the backward
+terms."""
+import os
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = open(oracle.SOURCE).read()
+
+# (name, original text, mutated text) -- each original occurs exactly once
+MUTANTS = [
+    ("scale_by_sqrt_C", "Pt[s] = acc * scale;", "Pt[s] = acc * (1.0 / sqrt((double)C));"),
+    ("scale_dropped", "Pt[s] = acc * scale;", "Pt[s] = acc;"),
+    ("lse_missing_max", "lse_row[t] = m + log(l);", "lse_row[t] = log(l);"),
+    ("scores_transposed",
+     "acc += qkv_at(qkv, T, C, hs, b, t, 0, h, d) * qkv_at(qkv, T, C, hs, b, s, 1, h, d);",
+     "acc += qkv_at(qkv, T, C, hs, b, s, 0, h, d) * qkv_at(qkv, T, C, hs, b, t, 1, h, d);"),
+    ("output_sums_keys", "acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);",
+     "acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);"),
+    ("future_leaks", "for (int s = t + 1; s < T; ++s) Pt[s] = 0.0;",
+     "for (int s = t + 1; s < T; ++s) Pt[s] = (s == t + 1) ? 1e-3 : 0.0;"),
+    ("softmax_jacobian_sign", "dSt[s] = Pt[s] * (dSt[s] - rowdot);", "dSt[s] = Pt[s] * (dSt[s] + rowdot);"),
+    ("softmax_jacobian_dropped", "dSt[s] = Pt[s] * (dSt[s] - rowdot);", "dSt[s] = Pt[s] * dSt[s];"),
+    ("dP_uses_keys",
+     "acc += dyb[(size_t)t * ld_dy + d] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);",
+     "acc += dyb[(size_t)t * ld_dy + d] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);"),
+    ("dV_transposed_P", "acc += P[(size_t)t * (size_t)T + s] * dyb[(size_t)t * ld_dy + d];",
+     "acc += P[(size_t)s * (size_t)T + t] * dyb[(size_t)t * ld_dy + d];"),
+    ("dQ_uses_queries",
+     "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);",
+     "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 0, h, d);"),
+    ("dK_missing_scale", "dk[(size_t)s * ld_dqkv + d] = acc * scale;", "dk[(size_t)s * ld_dqkv + d] = acc;"),
+    ("dK_transposed_dS",
+     "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);",
+     "acc += dS[(size_t)s * (size_t)T + t] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    assert SRC.count(old) == 1, f"mutation anchor for {name} not unique"
+    src = tmp_path / f"{name}.c"
+    src.write_text(SRC.replace(old, new))
+    so = oracle.compile_source(str(src), str(tmp_path / f"{name}.so"))
+    mutant = oracle.Oracle(so)
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(mutant)
+        except (AssertionError, RuntimeError, ValueError, FloatingPointError):
+            failed.append(pin.__name__)
+            break
+    assert failed, f"mutant {name} passed every pin"
