@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark: causal self-attention forward + backward TFLOP/s on B200.
+
+One step = gptattn_fwd + gptattn_bwd (all kernels of the path) over one batch of
+the workload, through the C ABI.  Default workload: the GPT-2 124M attention
+shape (B=16, T=1024, 12 heads of 64, bf16), seeded synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gpt2_124m]
+
+FLOPs are counted causally (half of dense): fwd 2*B*nh*T^2*hs, bwd 2.5x that.
+The L2 is flushed (256 MiB write) before every timed step, outside the step's
+CUDA events.  Under torchrun every rank runs its own batch (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+
+Prints one JSON line (rank 0).  --impl reference times the fp64 CPU oracle on
+a bounded sample of the same workload instead (test infrastructure, the only
+place besides the cpu_baseline leg where bench.py runs it).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="gpt2_124m")
+    p.add_argument("--cpu-sample-seconds", type=float, default=12.0)
+    p.add_argument("--skip-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while work runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.gpu_index)],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(w, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle on whole (batch, head) pairs of the workload until
+    about budget_s seconds have elapsed.  Returns (TFLOP/s, cores, sample text)."""
+    import numpy as np
+
+    import oracle
+    from causal_self_attention_gptattn_b200.workloads import workload_inputs
+
+    qkv, dy = workload_inputs(w, B=1)
+    q = qkv.double().numpy()
+    g = dy.double().numpy()
+    C, hs, nh = w.C, w.hs, w.n_head
+    heads_done = 0
+    elapsed = 0.0
+    while elapsed < budget_s and heads_done < w.B * nh:
+        h = heads_done % nh
+        cols = np.r_[h * hs:(h + 1) * hs, C + h * hs:C + (h + 1) * hs, 2 * C + h * hs:2 * C + (h + 1) * hs]
+        qh = np.ascontiguousarray(q[:, :, cols])
+        gh = np.ascontiguousarray(g[:, :, h * hs:(h + 1) * hs])
+        t0 = time.perf_counter()
+        oracle.forward(qh, 1)
+        oracle.backward(qh, gh, 1)
+        elapsed += time.perf_counter() - t0
+        heads_done += 1
+    flops = 3.5 * 2.0 * heads_done * w.T * w.T * w.hs
+    sample = (f"{heads_done} (batch, head) pairs of {w.name} (T={w.T}, hs={w.hs}), fwd+bwd each, "
+              f"fp64 oracle; {elapsed:.1f} s")
+    return flops / elapsed / 1e12, oracle.num_threads(), sample, elapsed
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    import oracle
+    cores = oracle.num_threads()
+    # size each step so the whole run stays within a few minutes
+    per_pair = None
+    steps_run = 0
+    total_s = 0.0
+    total_flops = 0.0
+    budget_total = 150.0
+    start = time.perf_counter()
+    for k in range(args.warmup + args.steps):
+        if time.perf_counter() - start > budget_total and k > args.warmup:
+            break
+        per_step_budget = budget_total / (args.warmup + args.steps)
+        v, _, sample, el = time_oracle(w, per_step_budget)
+        if k >= args.warmup:
+            steps_run += 1
+            total_s += el
+            total_flops += v * 1e12 * el
+    value = total_flops / total_s / 1e12 if total_s > 0 else 0.0
+    line = {
+        "impl": "reference", "metric": "causal attention fwd+bwd TFLOP/s (bf16, 1 B200)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": steps_run, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / max(steps_run, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {**w.describe(), "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {sample}"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+
+    from causal_self_attention_gptattn_b200 import gptattn as ga
+    from causal_self_attention_gptattn_b200.workloads import make_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    dt = ga.GPTATTN_BF16 if w.dtype == "bf16" else ga.GPTATTN_F32
+    B, T, C, nh = w.B, w.T, w.C, w.n_head
+    qkv_c, dy_c = make_inputs(B, T, nh, w.hs, dtype=w.torch_dtype, seed=1000 + w.index + 7919 * rank,
+                              recipe=w.recipe, qkv_scale=w.qkv_scale)
+    qkv = qkv_c.to(dev)
+    dy = dy_c.to(dev)
+    y = torch.empty(B, T, C, dtype=w.torch_dtype, device=dev)
+    lse = torch.empty(B, nh, T, dtype=torch.float32, device=dev)
+    dqkv = torch.empty_like(qkv)
+    nbytes = ga.gptattn_bwd_workspace_bytes(B, T, C, nh, dt)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
+    s = torch.cuda.current_stream(dev)
+
+    def step(q=qkv, g=dy):
+        ga.check(ga.gptattn_fwd(q, y, lse, B, T, C, nh, dt, s), "gptattn_fwd")
+        ga.check(ga.gptattn_bwd(q, y, lse, g, dqkv, ws, nbytes, B, T, C, nh, dt, s), "gptattn_bwd")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ga.check(ga.gptattn_get_device_status(s), "device status after warm-up")
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.25)
+    ga.gptattn_profile_enable(4 * K + 64)
+    launches0 = ga.gptattn_launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(K):
+        flush.zero_()
+        starts[k].record(s)
+        step()
+        ends[k].record(s)
+    torch.cuda.synchronize()
+    barrier()
+    wall1 = time.perf_counter()
+    launches = ga.gptattn_launch_count() - launches0
+    prof = ga.gptattn_profile_read(4 * K + 64)
+    ga.gptattn_profile_enable(0)
+    # keep the same loop running (untimed) so the clock sampler sees >= ~1.5 s of load
+    extra_until = wall0 + 1.5
+    while time.perf_counter() < extra_until:
+        for _ in range(50):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ga.check(ga.gptattn_get_device_status(s), "device status after timing")
+
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms))
+    flops = w.flops_fwd_bwd()
+    value = world * K * flops / (total_ms / 1e3) / 1e12
+
+    # per-kernel durations recorded by the library inside the timed loop
+    per_kernel = {}
+    for name, ms in prof:
+        per_kernel.setdefault(name, []).append(ms)
+    kern_avg = {k: statistics.mean(v) for k, v in per_kernel.items()}
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region)
+    qkv_h = qkv_c.pin_memory()
+    dy_h = dy_c.pin_memory()
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    dqkv_h = torch.empty(dqkv.shape, dtype=dqkv.dtype).pin_memory()
+    qkv_d = torch.empty_like(qkv)
+    dy_d = torch.empty_like(dy)
+    Ke = max(1, min(K, 200))
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+    for _ in range(3):
+        qkv_d.copy_(qkv_h, non_blocking=True)
+        dy_d.copy_(dy_h, non_blocking=True)
+        step(qkv_d, dy_d)
+    torch.cuda.synchronize()
+    barrier()
+    for k in range(Ke):
+        flush.zero_()
+        e_starts[k].record(s)
+        qkv_d.copy_(qkv_h, non_blocking=True)
+        dy_d.copy_(dy_h, non_blocking=True)
+        step(qkv_d, dy_d)
+        y_h.copy_(y, non_blocking=True)
+        dqkv_h.copy_(dqkv, non_blocking=True)
+        e_ends[k].record(s)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_starts, e_ends)))
+    e2e_value = world * Ke * flops / (e2e_ms / 1e3) / 1e12
+    h2d = qkv_h.numel() * qkv_h.element_size() + dy_h.numel() * dy_h.element_size()
+    d2h = y_h.numel() * y_h.element_size() + dqkv_h.numel() * dqkv_h.element_size()
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    dominant = "bwd_bf16_sm100" if dt == ga.GPTATTN_BF16 else "bwd_dkv_f32"
+    dom_ms = kern_avg.get(dominant)
+    dom_flops = w.flops_bwd()  # the main backward kernel does all 5 backward matmuls
+    roofline = None
+    if dom_ms:
+        achieved = dom_flops / (dom_ms / 1e3) / 1e12
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "peak_source": f"{peak_src} bf16 burst",
+                    "traffic": None, "avg_ms": dom_ms}
+
+    cpu = None
+    if world == 1 and not args.skip_cpu_baseline:
+        v, cores, sample, _ = time_oracle(w, args.cpu_sample_seconds)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    line = {
+        "metric": "causal attention fwd+bwd TFLOP/s (bf16, 1 B200)",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {**w.describe(), "parallelism": f"dp{world} (independent batches per GPU)",
+                   "flops_per_step_per_gpu": flops,
+                   "l2": "flushed before every timed step (256 MiB write, outside the step events)"},
+        "pct_of_peak": {"measured_bf16_burst": value / world / float(peaks.get("bf16_tflops", 1590.0)),
+                        "datasheet_2250": value / world / 2250.0},
+        "kernels_ms": kern_avg,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": Ke},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "wall_s_timed": wall1 - wall0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from causal_self_attention_gptattn_b200.workloads import by_name
+    w = by_name(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    run_ours(args, w, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

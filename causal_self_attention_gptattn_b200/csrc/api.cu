@@ -1,0 +1,405 @@
+// api.cu -- the C ABI of libgptattn (declared in include/gptattn.h).
+//
+// Host-side responsibilities: validate every argument before anything is
+// enqueued, build the TMA tensor maps that let the kernels address q, k, v of
+// one head directly inside the packed qkv tensor (heads as a batch dimension,
+// exercise EX1 of the lecture page "Let's build GPT: from scratch, in code,
+// spelled out"), carve the caller's workspace, launch, and map CUDA errors to
+// status codes.  Also owns the device status word that kernels use to report
+// a bounded wait that ran out.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "gptattn.h"
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace gptattn {
+
+// Device status word: 0, or the status code of the first kernel that gave up
+// on a wait since it was last read.  One per device that loads the library.
+__device__ int g_device_status;
+
+namespace {
+
+constexpr unsigned long long kDefaultBudgetNs = 1000000000ull;  // 1 s per wait
+constexpr int kMaxDevices = 64;
+
+std::mutex g_mutex;
+int *g_status_ptr[kMaxDevices] = {};
+std::atomic<unsigned long long> g_launches{0};
+
+gptattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GPTATTN_OK : GPTATTN_ERR_CUDA; }
+
+// Device address of g_device_status for the current device (looked up once
+// per device, with that device current).
+cudaError_t status_ptr(int **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_status);
+        if (e != cudaSuccess) return e;
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    *out = g_status_ptr[dev];
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps (driver entry point fetched through the runtime, so the library
+// needs no link-time dependency on libcuda).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor [B][T][W] viewed as 3-D (W, T, B); box (64, 128, 1); 128-byte
+// swizzle; rows past T read as zero and are not written.
+bool map_bf16_rows(CUtensorMap *m, const void *ptr, int W, int T, int B) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)W * 2u, (cuuint64_t)W * 2u * (cuuint64_t)T};
+    cuuint32_t box[3] = {64, (cuuint32_t)kTile, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 matrix [rows][hs] viewed as 2-D (hs, rows); box (32, 128); 128-byte swizzle.
+bool map_f32_acc(CUtensorMap *m, const void *ptr, int hs, long long rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)hs, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)hs * 4u};
+    cuuint32_t box[2] = {32, (cuuint32_t)kTile};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// Validation (pure host; nothing is enqueued on failure)
+// ---------------------------------------------------------------------------
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gptattn_status check_shape(int B, int T, int C, int n_head, gptattn_dtype dt, int *hs_out) {
+    if (B < 0 || T < 0 || C <= 0 || n_head <= 0) return GPTATTN_ERR_INVALID_ARG;
+    if (C % n_head != 0) return GPTATTN_ERR_INVALID_ARG;
+    const int hs = C / n_head;
+    if (dt == GPTATTN_BF16) {
+        if (hs != 64 && hs != 128) return GPTATTN_ERR_UNSUPPORTED;
+    } else if (dt == GPTATTN_F32) {
+        if (hs != 16 && hs != 32 && hs != 64 && hs != 128) return GPTATTN_ERR_UNSUPPORTED;
+    } else {
+        return GPTATTN_ERR_UNSUPPORTED;
+    }
+    // Size limits: 3C fits a TMA dimension and an int index; grid fits in x.
+    if ((long long)C * 3 > (1LL << 30)) return GPTATTN_ERR_UNSUPPORTED;
+    const long long tiles = (long long)((T + kTile - 1) / kTile) * B * n_head;
+    if (tiles > 0x7fffffffLL) return GPTATTN_ERR_UNSUPPORTED;
+    if ((long long)B * n_head > 65535LL && dt == GPTATTN_F32) return GPTATTN_ERR_UNSUPPORTED;  // grid.y
+    *hs_out = hs;
+    return GPTATTN_OK;
+}
+
+int padded_T(int T) { return ((T + kTile - 1) / kTile) * kTile; }
+
+size_t align256(size_t x) { return (x + 255u) & ~(size_t)255u; }
+
+struct BwdWorkspace {
+    size_t D, lse2, dqacc, total;
+};
+
+BwdWorkspace workspace_layout(int B, int T, int n_head, int hs, gptattn_dtype dt) {
+    BwdWorkspace w{};
+    if (dt == GPTATTN_F32) {
+        w.D = 0;
+        w.total = align256((size_t)B * n_head * T * sizeof(float));
+        return w;
+    }
+    const size_t rows = (size_t)B * n_head * padded_T(T);
+    w.D = 0;
+    w.lse2 = align256(rows * sizeof(float));
+    w.dqacc = w.lse2 + align256(rows * sizeof(float));
+    w.total = w.dqacc + align256(rows * (size_t)hs * sizeof(float));
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// Instrumentation: optional CUDA events around each kernel launch.
+// ---------------------------------------------------------------------------
+struct ProfRecord {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+struct Profiler {
+    int capacity = 0;
+    std::vector<ProfRecord> records;   // filled in order
+    std::vector<cudaEvent_t> pool;     // reusable events
+} g_prof;
+
+cudaEvent_t prof_event() {
+    if (!g_prof.pool.empty()) {
+        cudaEvent_t e = g_prof.pool.back();
+        g_prof.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+template <class F>
+cudaError_t run_kernel(int kernel_id, cudaStream_t s, F &&launch) {
+    ProfRecord rec{kernel_id, nullptr, nullptr};
+    bool recording = false;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_prof.capacity > 0 && (int)g_prof.records.size() < g_prof.capacity) {
+            rec.start = prof_event();
+            rec.stop = prof_event();
+            recording = rec.start && rec.stop;
+        }
+    }
+    if (recording) cudaEventRecord(rec.start, s);
+    cudaError_t e = launch();
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (recording) {
+        cudaEventRecord(rec.stop, s);
+        std::lock_guard<std::mutex> lock(g_mutex);
+        g_prof.records.push_back(rec);
+    }
+    return e;
+}
+
+// ---------------------------------------------------------------------------
+// Bounded-wait self-test kernel: waits on a barrier nobody arrives at.
+// ---------------------------------------------------------------------------
+__global__ void selftest_timeout_kernel(int *status, unsigned long long budget_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const WaitGuard g{&abort_flag, status, budget_ns};
+        (void)mbar_wait(smem_u32(&bar), 0, g);  // nothing ever completes phase 0
+    }
+    __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s) {
+    selftest_timeout_kernel<<<1, 32, 0, s>>>(ctx.status, ctx.budget_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace gptattn
+
+using namespace gptattn;
+
+extern "C" {
+
+const char *gptattn_status_string(gptattn_status s) {
+    switch (s) {
+        case GPTATTN_OK: return "ok";
+        case GPTATTN_ERR_INVALID_ARG: return "invalid argument";
+        case GPTATTN_ERR_UNSUPPORTED: return "unsupported head size, dtype or size";
+        case GPTATTN_ERR_CUDA: return "CUDA error";
+        case GPTATTN_ERR_TIMEOUT: return "a kernel wait timed out";
+        case GPTATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    }
+    return "unknown status";
+}
+
+int gptattn_version(void) { return 100; }
+
+gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, gptattn_dtype dt,
+                           gptattn_stream_t stream) {
+    int hs = 0;
+    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
+    if (st != GPTATTN_OK) return st;
+    if (B == 0 || T == 0) return GPTATTN_OK;
+    if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    if (dt == GPTATTN_F32) {
+        return from_cuda(run_kernel(kKFwdF32, s, [&] {
+            return launch_fwd_f32(hs, static_cast<const float *>(qkv), static_cast<float *>(y), lse, B, T, C, n_head, s);
+        }));
+    }
+    int *status = nullptr;
+    cudaError_t e = status_ptr(&status);
+    if (e != cudaSuccess) return GPTATTN_ERR_CUDA;
+    CUtensorMap mq, my;
+    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&my, y, C, T, B)) return GPTATTN_ERR_CUDA;
+    const DevCtx ctx{status, kDefaultBudgetNs};
+    return from_cuda(run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, ctx, s); }));
+}
+
+size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt) {
+    int hs = 0;
+    if (check_shape(B, T, C, n_head, dt, &hs) != GPTATTN_OK) return (size_t)-1;
+    if (B == 0 || T == 0) return 0;
+    return workspace_layout(B, T, n_head, hs, dt).total;
+}
+
+gptattn_status gptattn_bwd(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
+                           void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, gptattn_dtype dt,
+                           gptattn_stream_t stream) {
+    int hs = 0;
+    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
+    if (st != GPTATTN_OK) return st;
+    if (B == 0 || T == 0) return GPTATTN_OK;
+    if (!qkv || !y || !lse || !dy || !dqkv) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse) || !aligned16(dy) || !aligned16(dqkv))
+        return GPTATTN_ERR_INVALID_ARG;
+    const BwdWorkspace w = workspace_layout(B, T, n_head, hs, dt);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < w.total)
+        return GPTATTN_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+
+    if (dt == GPTATTN_F32) {
+        const float *fq = static_cast<const float *>(qkv);
+        const float *fy = static_cast<const float *>(y);
+        const float *fg = static_cast<const float *>(dy);
+        float *fo = static_cast<float *>(dqkv);
+        float *D = reinterpret_cast<float *>(ws + w.D);
+        cudaError_t e = run_kernel(kKBwdPreF32, s, [&] { return launch_bwd_f32_pre(hs, fy, fg, D, B, T, C, n_head, s); });
+        if (e == cudaSuccess)
+            e = run_kernel(kKBwdDqF32, s, [&] { return launch_bwd_f32_dq(hs, fq, fg, lse, D, fo, B, T, C, n_head, s); });
+        if (e == cudaSuccess)
+            e = run_kernel(kKBwdDkvF32, s, [&] { return launch_bwd_f32_dkv(hs, fq, fg, lse, D, fo, B, T, C, n_head, s); });
+        return from_cuda(e);
+    }
+
+    int *status = nullptr;
+    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    const int T_pad = padded_T(T);
+    float *D = reinterpret_cast<float *>(ws + w.D);
+    float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
+    float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
+    CUtensorMap mq, mdy, mdqkv, mdq;
+    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&mdy, dy, C, T, B) ||
+        !map_bf16_rows(&mdqkv, dqkv, 3 * C, T, B) || !map_f32_acc(&mdq, dqacc, hs, (long long)B * n_head * T_pad))
+        return GPTATTN_ERR_CUDA;
+    const DevCtx ctx{status, kDefaultBudgetNs};
+    cudaError_t e = run_kernel(kKBwdPreBf16, s, [&] {
+        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, s);
+    });
+    if (e == cudaSuccess)
+        e = run_kernel(kKBwdMainBf16, s, [&] {
+            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
+        });
+    if (e == cudaSuccess)
+        e = run_kernel(kKBwdPostBf16, s, [&] { return launch_bwd_post_bf16(hs, dqacc, dqkv, B, T, C, n_head, T_pad, s); });
+    return from_cuda(e);
+}
+
+gptattn_status gptattn_get_device_status(gptattn_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    int *p = nullptr;
+    if (status_ptr(&p) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    return v == 0 ? GPTATTN_OK : static_cast<gptattn_status>(v);
+}
+
+gptattn_status gptattn_profile_enable(int max_records) {
+    if (max_records < 0) return GPTATTN_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_prof.capacity = max_records;
+    // create the events now, so recording inside a timed region allocates nothing
+    const size_t want = 2u * (size_t)max_records;
+    while (g_prof.pool.size() + 2u * g_prof.records.size() < want) {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) return GPTATTN_ERR_CUDA;
+        g_prof.pool.push_back(e);
+    }
+    if (max_records == 0) {
+        for (auto &r : g_prof.records) {
+            g_prof.pool.push_back(r.start);
+            g_prof.pool.push_back(r.stop);
+        }
+        g_prof.records.clear();
+        for (cudaEvent_t e : g_prof.pool) cudaEventDestroy(e);
+        g_prof.pool.clear();
+    }
+    return GPTATTN_OK;
+}
+
+int gptattn_profile_read(int *kernel_ids, float *ms, int capacity) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int n = 0;
+    for (auto &r : g_prof.records) {
+        if (n < capacity && kernel_ids && ms) {
+            float t = -1.f;
+            if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+                t = -1.f;
+            kernel_ids[n] = r.kernel;
+            ms[n] = t;
+            ++n;
+        }
+        g_prof.pool.push_back(r.start);
+        g_prof.pool.push_back(r.stop);
+    }
+    g_prof.records.clear();
+    return n;
+}
+
+const char *gptattn_kernel_name(int kernel_id) {
+    static const char *names[kKNumKernels] = {
+        "fwd_bf16_sm100", "bwd_pre_bf16", "bwd_bf16_sm100", "bwd_post_bf16", "fwd_f32_simt",
+        "bwd_pre_f32",    "bwd_dq_f32",   "bwd_dkv_f32",    "selftest_timeout"};
+    if (kernel_id < 0 || kernel_id >= kKNumKernels) return "unknown";
+    return names[kernel_id];
+}
+
+unsigned long long gptattn_launch_count(void) { return g_launches.load(); }
+
+gptattn_status gptattn_selftest_wait_timeout(unsigned long long budget_ns, gptattn_stream_t stream) {
+    if (budget_ns < 1000ull || budget_ns > 2000000000ull) return GPTATTN_ERR_INVALID_ARG;
+    int *status = nullptr;
+    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const DevCtx ctx{status, budget_ns};
+    return from_cuda(run_kernel(kKSelftest, s, [&] { return launch_selftest_timeout(ctx, s); }));
+}
+
+}  // extern "C"

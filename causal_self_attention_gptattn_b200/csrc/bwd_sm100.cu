@@ -1,0 +1,555 @@
+// bwd_sm100.cu -- bf16 causal self-attention backward for sm_100a.
+//
+// Chain rule through the forward (lecture page "Let's build GPT: from scratch,
+// in code, spelled out", chapters "version 3: adding softmax" and "version 4:
+// self-attention"), with P recomputed from the saved logsumexp instead of
+// stored:
+//     P   = exp(S * scale - lse)           S = Q K^T, masked causally
+//     dV  = P^T dY,  dP = dY V^T
+//     dS  = P o (dP - D),  D = rowsum(dY o y)   (= rowsum(P o dP))
+//     dQ  = dS K * scale,  dK = dS^T Q * scale
+//
+// Three kernels:
+//   pre   D and lse*log2(e) per query row into the workspace; zero dQ accumulator
+//   main  one CTA per (key tile j, b, h); loops over query tiles i >= j:
+//           S^T = K Q_i^T, dP^T = V dO_i^T          (tcgen05, TMEM)
+//           P^T (bf16) back into TMEM; dS^T (bf16) into shared memory
+//           dV += P^T dO_i (P from TMEM), dK += dS^T Q_i   (TMEM accumulators)
+//           dQ_i = dS K -> TMEM -> smem -> TMA reduce-add into the fp32 accumulator
+//         epilogue: dK * scale and dV -> bf16 -> TMA store into dqkv
+//   post  dQ accumulator * scale -> bf16 into dqkv[..., 0:C]
+//
+// Main-kernel roles (10 warps):
+//   warp 0      TMA producer (K, V once; Q_i, dO_i, lse_i, D_i per iteration)
+//   warp 1      TMEM owner + MMA issuer
+//   warps 2..5  "softmax" warps, one key row each: P, dS, final dK/dV epilogue
+//   warps 6..9  dQ drain warps, one query row each: TMEM -> smem -> TMA reduce
+// TMEM columns: S^T [0,128) (P^T packed into [0,64)), dP^T [128,256),
+// dV [256,256+hs), dK [256+hs, 256+2hs).  dQ: hs=64 at [384,448); hs=128 in
+// two 64-column halves at [64,128) and [192,256), the parts of S^T / dP^T that
+// are free once P^T and dS^T have been produced.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace gptattn {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlabBytes = 128 * 128;
+
+template <int HS>
+struct BwdCfg {
+    static constexpr int kSlabs = HS / 64;
+    static constexpr uint32_t kTileBytes = 128u * HS * 2u;
+    static constexpr int kStages = (HS == 64) ? 2 : 1;
+    static constexpr uint32_t kOffK = 0;
+    static constexpr uint32_t kOffV = kOffK + kTileBytes;
+    static constexpr uint32_t kOffQ = kOffV + kTileBytes;
+    static constexpr uint32_t kOffdO = kOffQ + kStages * kTileBytes;
+    static constexpr uint32_t kOffdS = kOffdO + kStages * kTileBytes;  // 128 x 128 bf16, two slabs
+    static constexpr uint32_t kOffdQ = kOffdS + 2 * kSlabBytes;          // 128 x 64 fp32 staging, two slabs
+    static constexpr uint32_t kOffLse = kOffdQ + 2 * kSlabBytes;         // kStages x 128 fp32
+    static constexpr uint32_t kOffD = kOffLse + kStages * 512;
+    static constexpr uint32_t kOffBar = kOffD + kStages * 512;
+    static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+    static constexpr uint32_t kColS = 0, kColdP = 128, kColdV = 256, kColdK = 256 + HS;
+    static constexpr uint32_t kColdQ0 = (HS == 64) ? 384 : 64;
+    static constexpr uint32_t kColdQ1 = 192;  // second half, hs = 128 only
+    static constexpr bool kDqAliases = (HS == 128);
+    // barriers
+    static constexpr int kBarKV = 0;
+    static constexpr int kBarFull = 1;                 // kStages
+    static constexpr int kBarEmpty = kBarFull + kStages;  // kStages
+    static constexpr int kBarS = kBarEmpty + kStages;
+    static constexpr int kBardP = kBarS + 1;
+    static constexpr int kBarP = kBardP + 1;
+    static constexpr int kBardS = kBarP + 1;
+    static constexpr int kBardQFull = kBardS + 1;
+    static constexpr int kBardQEmpty = kBardQFull + 1;
+    static constexpr int kBarKdV = kBardQEmpty + 1;
+    static constexpr int kBarDone = kBarKdV + 1;
+    static constexpr int kNumBars = kBarDone + 1;
+    static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitGuard &g) {
+    bool ok = mbar_wait(bar, parity, g);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > budget_ns) break;
+    }
+}
+
+template <int HS>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_bf16_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
+                    const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
+                    const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C, int n_head,
+                    int T_pad, int n_t, int *status, unsigned long long budget_ns) {
+    using K = BwdCfg<HS>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int BH = B * n_head;
+    const int bh = blockIdx.x % BH;
+    const int kt = blockIdx.x / BH;   // key tile; small kt = most query tiles = scheduled first
+    const int b = bh / n_head;
+    const int h = bh % n_head;
+    const int niter = n_t - kt;       // query tiles kt..n_t-1
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K::kOffBar);
+    auto bar = [&](int idx) -> uint32_t { return smem_u32(&bars[idx]); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + K::kOffBar + K::kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K::kOffBar + K::kNumBars * 8 + 4);
+    const WaitGuard g{abort_flag, status, budget_ns};
+
+    const uint32_t sK = sbase + K::kOffK, sV = sbase + K::kOffV;
+    auto sQ = [&](int st) -> uint32_t { return sbase + K::kOffQ + st * K::kTileBytes; };
+    auto sdO = [&](int st) -> uint32_t { return sbase + K::kOffdO + st * K::kTileBytes; };
+    const uint32_t sdS = sbase + K::kOffdS, sdQ = sbase + K::kOffdQ;
+    const float *sLse = reinterpret_cast<const float *>(smem + K::kOffLse);
+    const float *sD = reinterpret_cast<const float *>(smem + K::kOffD);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(K::kBarKV), 1);
+        for (int s = 0; s < K::kStages; ++s) {
+            mbar_init(bar(K::kBarFull + s), 1);
+            mbar_init(bar(K::kBarEmpty + s), 1);
+        }
+        mbar_init(bar(K::kBarS), 1);
+        mbar_init(bar(K::kBardP), 1);
+        mbar_init(bar(K::kBarP), 128);
+        mbar_init(bar(K::kBardS), 128);
+        mbar_init(bar(K::kBardQFull), 1);
+        mbar_init(bar(K::kBardQEmpty), 128);
+        mbar_init(bar(K::kBarKdV), 1);
+        mbar_init(bar(K::kBarDone), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_map(&map_qkv);
+            tma_prefetch_map(&map_dy);
+            const int col_q = h * HS, col_k = C + h * HS, col_v = 2 * C + h * HS;
+            mbar_arrive_expect_tx(bar(K::kBarKV), 2 * K::kTileBytes);
+            for (int s = 0; s < K::kSlabs; ++s) {
+                tma_load_3d(sK + s * kSlabBytes, &map_qkv, bar(K::kBarKV), col_k + 64 * s, kt * kTile, b);
+                tma_load_3d(sV + s * kSlabBytes, &map_qkv, bar(K::kBarKV), col_v + 64 * s, kt * kTile, b);
+            }
+            int issued = 0;
+            bool ok = true;
+            for (int it = 0; it < niter; ++it) {
+                const int qt = kt + it;
+                const int st = it % K::kStages;
+                const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
+                if (it >= K::kStages && !mbar_wait(bar(K::kBarEmpty + st), ph ^ 1u, g)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = bar(K::kBarFull + st);
+                mbar_arrive_expect_tx(fb, 2 * K::kTileBytes + 1024);
+                for (int s = 0; s < K::kSlabs; ++s) {
+                    tma_load_3d(sQ(st) + s * kSlabBytes, &map_qkv, fb, col_q + 64 * s, qt * kTile, b);
+                    tma_load_3d(sdO(st) + s * kSlabBytes, &map_dy, fb, h * HS + 64 * s, qt * kTile, b);
+                }
+                const size_t rowoff = (size_t)bh * (size_t)T_pad + (size_t)qt * kTile;
+                bulk_load(sbase + K::kOffLse + st * 512, lse2 + rowoff, 512, fb);
+                bulk_load(sbase + K::kOffD + st * 512, Dvec + rowoff, 512, fb);
+                issued = it + 1;
+            }
+            if (!ok || *abort_flag) {
+                drain_wait(bar(K::kBarKV), 0, budget_ns);
+                for (int it = (issued > K::kStages ? issued - K::kStages : 0); it < issued; ++it)
+                    drain_wait(bar(K::kBarFull + it % K::kStages), (uint32_t)(it / K::kStages) & 1u, budget_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idSS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+            constexpr uint32_t idAcc = idesc_bf16_f32(128, HS, false, true);   // dV, dK (B = dO / Q, N-major)
+            constexpr uint32_t idQ = idesc_bf16_f32(128, 64, true, true);      // dQ half (A = dS, M-major)
+            bool ok = mbar_wait(bar(K::kBarKV), 0, g);
+            bool any = false;
+            for (int it = 0; it < niter && ok; ++it) {
+                const int st = it % K::kStages;
+                const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
+                if (!(ok = mbar_wait(bar(K::kBarFull + st), ph, g))) break;
+                if (K::kDqAliases && it > 0 && !(ok = mbar_wait(bar(K::kBardQEmpty), (uint32_t)(it - 1) & 1u, g)))
+                    break;
+                tc_fence_after();
+                // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+#pragma unroll
+                for (int kk = 0; kk < HS / 16; ++kk) {
+                    const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
+                    umma_ss(tmem + K::kColS, sdesc_sw128(sK + koff, 16, 1024), sdesc_sw128(sQ(st) + koff, 16, 1024),
+                            idSS, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar(K::kBarS));
+#pragma unroll
+                for (int kk = 0; kk < HS / 16; ++kk) {
+                    const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
+                    umma_ss(tmem + K::kColdP, sdesc_sw128(sV + koff, 16, 1024), sdesc_sw128(sdO(st) + koff, 16, 1024),
+                            idSS, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar(K::kBardP));
+                any = true;
+                // dV += P^T dO   (A = P^T in TMEM, K = query rows)
+                if (!(ok = mbar_wait(bar(K::kBarP), (uint32_t)it & 1u, g))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + K::kColdV, tmem + K::kColS + 8u * kk,
+                            sdesc_sw128(sdO(st) + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                // dK += dS^T Q   (A = dS^T in smem, key rows x query cols, K-major)
+                if (!(ok = mbar_wait(bar(K::kBardS), (uint32_t)it & 1u, g))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
+                    umma_ss(tmem + K::kColdK, sdesc_sw128(sdS + koff, 16, 1024),
+                            sdesc_sw128(sQ(st) + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar(K::kBarEmpty + st));  // Q_i / dO_i / lse_i / D_i no longer needed
+                // dQ_i = dS K   (A = dS, M-major view of the same smem; B = K, N-major)
+                if (!K::kDqAliases && it > 0 &&
+                    !(ok = mbar_wait(bar(K::kBardQEmpty), (uint32_t)(it - 1) & 1u, g)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int half = 0; half < HS / 64; ++half) {
+                    const uint32_t dcol = half == 0 ? K::kColdQ0 : K::kColdQ1;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ss(tmem + dcol, sdesc_sw128(sdS + kk * 2048u, kSlabBytes, 1024),
+                                sdesc_sw128(sK + half * kSlabBytes + kk * 2048u, kSlabBytes, 1024), idQ,
+                                kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar(K::kBardQFull));
+            }
+            if (ok) umma_commit(bar(K::kBarKdV));
+            if (any || ok) {
+                umma_commit(bar(K::kBarDone));
+                drain_wait(bar(K::kBarDone), 0, budget_ns);
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ softmax warps (key rows)
+        const int sp = warp & 3;
+        const int row = sp * 32 + lane;  // key row within the tile
+        const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
+        const float scale_log2 = (HS == 64 ? 0.125f : 0.08838834764831845f) * 1.4426950408889634f;
+        bool ok = true;
+        for (int it = 0; it < niter; ++it) {
+            const int st = it % K::kStages;
+            const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
+            ok = warp_wait(bar(K::kBarFull + st), ph, g) && warp_wait(bar(K::kBarS), (uint32_t)it & 1u, g);
+            if (!ok) break;
+            tc_fence_after();
+            const float *lse_i = sLse + st * 128;
+            const float *D_i = sD + st * 128;
+            uint32_t pk[64];  // P^T row, bf16 pairs
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t sr[32];
+                tmem_ld_x32(trow + K::kColS + 32 * ch, sr);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int c = 32 * ch + e;
+                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, -lse_i[c]));
+                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), scale_log2, -lse_i[c + 1]));
+                    if (it == 0) {  // diagonal tile: query c sees key row only if row <= c
+                        if (c < row) p0 = 0.f;
+                        if (c + 1 < row) p1 = 0.f;
+                    }
+                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                }
+                // columns [16ch, 16ch+16) were read in an earlier (or this) chunk
+                tmem_st_x16(trow + K::kColS + 16 * ch, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * ch]));
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(K::kBarP));
+
+            ok = warp_wait(bar(K::kBardP), (uint32_t)it & 1u, g);
+            if (ok && it > 0) ok = warp_wait(bar(K::kBardQFull), (uint32_t)(it - 1) & 1u, g);  // dS buffer free
+            if (!ok) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t dr[32];
+                tmem_ld_x32(trow + K::kColdP + 32 * ch, dr);
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int c = 32 * ch + e;
+                    const uint32_t pp = pk[c >> 1];
+                    const float ds0 = bf16lo_to_f32(pp) * (__uint_as_float(dr[e]) - D_i[c]);
+                    const float ds1 = bf16hi_to_f32(pp) * (__uint_as_float(dr[e + 1]) - D_i[c + 1]);
+                    w[e >> 1] = pack_bf16x2(ds0, ds1);
+                }
+                // dS^T row `row`, query columns [32ch, 32ch+32): slab ch/2, 16-byte chunks 4*(ch&1)..+3
+                const uint32_t rbase = sdS + (uint32_t)(ch >> 1) * kSlabBytes + (uint32_t)row * 128u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t chunk = (uint32_t)(4 * (ch & 1) + q);
+                    st_shared_v4(rbase + ((chunk ^ (uint32_t)(row & 7)) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2],
+                                 w[4 * q + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(K::kBardS));
+        }
+        // -------------------------------------------------------- dK / dV epilogue
+        if (ok) ok = warp_wait(bar(K::kBarKdV), 0, g);
+        if (ok) {
+            tc_fence_after();
+            const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
+            // staging: dV tile in the Q buffer of stage 0, dK tile in the dO buffer of stage 0
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? K::kColdV : K::kColdK;
+                const float mul = which == 0 ? 1.f : scale;
+                const uint32_t stage_buf = which == 0 ? sQ(0) : sdO(0);
+#pragma unroll
+                for (int c0 = 0; c0 < HS; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld_x32(trow + col + c0, o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
+                    const uint32_t rbase = stage_buf + (uint32_t)(c0 >> 6) * kSlabBytes + (uint32_t)row * 128u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t chunk = (uint32_t)(((c0 & 63) >> 3) + q);
+                        st_shared_v4(rbase + ((chunk ^ (uint32_t)(row & 7)) << 4), w[4 * q], w[4 * q + 1],
+                                     w[4 * q + 2], w[4 * q + 3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0 && !*abort_flag) {
+            for (int s = 0; s < K::kSlabs; ++s) {
+                tma_store_3d(&map_dqkv, sQ(0) + s * kSlabBytes, 2 * C + h * HS + 64 * s, kt * kTile, b);
+                tma_store_3d(&map_dqkv, sdO(0) + s * kSlabBytes, C + h * HS + 64 * s, kt * kTile, b);
+            }
+            bulk_commit_group();
+            bulk_wait_group_0();
+        }
+    } else {
+        // ------------------------------------------------------------ dQ drain warps (query rows)
+        const int sp = warp & 3;
+        const int row = sp * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
+        const bool leader = (warp == 6 && lane == 0);
+        // Every thread of this role executes the same sequence of named
+        // barriers whatever happens; after a failed wait the work is skipped.
+        bool ok = true;
+        for (int it = 0; it < niter; ++it) {
+            const int qt = kt + it;
+            if (ok) ok = warp_wait(bar(K::kBardQFull), (uint32_t)it & 1u, g);
+            if (ok) tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < HS / 64; ++half) {
+                uint32_t v[64];
+                const uint32_t dcol = half == 0 ? K::kColdQ0 : K::kColdQ1;
+                if (ok) {
+                    tmem_ld_x32(trow + dcol, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                    tmem_ld_x32(trow + dcol + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                    if (half == HS / 64 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(K::kBardQEmpty));
+                    }
+                }
+                if (leader) bulk_wait_group_read_0();  // staging free again
+                named_bar_sync(2, 128);
+                if (ok) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const uint32_t rbase = sdQ + (uint32_t)u * kSlabBytes + (uint32_t)row * 128u;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), v[32 * u + 4 * q],
+                                         v[32 * u + 4 * q + 1], v[32 * u + 4 * q + 2], v[32 * u + 4 * q + 3]);
+                    }
+                    fence_proxy_async_smem();
+                }
+                named_bar_sync(2, 128);
+                if (leader && ok && !*abort_flag) {
+                    const int r0 = bh * T_pad + qt * kTile;
+                    tma_reduce_add_2d(&map_dq, sdQ, half * 64, r0);
+                    tma_reduce_add_2d(&map_dq, sdQ + kSlabBytes, half * 64 + 32, r0);
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (leader) bulk_wait_group_0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// preprocess: D = rowsum(dy o y) per (b, h, t); lse2 = lse * log2(e); rows
+// t >= T of each (b, h) get D = 0 and lse2 = +inf (so recomputed P is 0);
+// dQ accumulator zeroed.
+// ---------------------------------------------------------------------------
+template <int HS>
+__global__ void bwd_pre_kernel(const __nv_bfloat16 *__restrict__ y, const __nv_bfloat16 *__restrict__ dy,
+                               const float *__restrict__ lse, float *__restrict__ D, float *__restrict__ lse2,
+                               float4 *__restrict__ dqacc, int B, int T, int C, int n_head, int T_pad) {
+    const long long rows = (long long)B * n_head * T_pad;
+    const long long zero4 = rows * HS / 4;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < rows; idx += stride) {
+        const int t = (int)(idx % T_pad);
+        const long long bh = idx / T_pad;
+        const int h = (int)(bh % n_head);
+        const long long b = bh / n_head;
+        float d = 0.f, l2 = INFINITY;
+        if (t < T) {
+            const size_t off = ((size_t)b * T + t) * (size_t)C + (size_t)h * HS;
+            const uint4 *yv = reinterpret_cast<const uint4 *>(y + off);
+            const uint4 *gv = reinterpret_cast<const uint4 *>(dy + off);
+#pragma unroll
+            for (int k = 0; k < HS / 8; ++k) {
+                const uint4 a = yv[k], c = gv[k];
+                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    d = fmaf(bf16lo_to_f32(av[q]), bf16lo_to_f32(cv[q]), d);
+                    d = fmaf(bf16hi_to_f32(av[q]), bf16hi_to_f32(cv[q]), d);
+                }
+            }
+            l2 = lse[bh * T + t] * 1.4426950408889634f;
+        }
+        D[idx] = d;
+        lse2[idx] = l2;
+    }
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < zero4; idx += stride) dqacc[idx] = z;
+}
+
+// postprocess: dq = bf16(dqacc * scale) into dqkv[..., 0:C]
+template <int HS>
+__global__ void bwd_post_kernel(const float *__restrict__ dqacc, __nv_bfloat16 *__restrict__ dqkv, int B, int T,
+                                int C, int n_head, int T_pad) {
+    const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
+    const long long n8 = (long long)B * T * n_head * (HS / 8);
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < n8; idx += stride) {
+        const int k = (int)(idx % (HS / 8));
+        long long r = idx / (HS / 8);
+        const int h = (int)(r % n_head);
+        r /= n_head;
+        const int t = (int)(r % T);
+        const long long b = r / T;
+        const float4 *src = reinterpret_cast<const float4 *>(
+            dqacc + (((size_t)b * n_head + h) * (size_t)T_pad + (size_t)t) * HS + (size_t)k * 8);
+        const float4 a = src[0], c = src[1];
+        uint4 o;
+        o.x = pack_bf16x2(a.x * scale, a.y * scale);
+        o.y = pack_bf16x2(a.z * scale, a.w * scale);
+        o.z = pack_bf16x2(c.x * scale, c.y * scale);
+        o.w = pack_bf16x2(c.z * scale, c.w * scale);
+        *reinterpret_cast<uint4 *>(dqkv + ((size_t)b * T + t) * (size_t)(3 * C) + (size_t)h * HS + (size_t)k * 8) = o;
+    }
+}
+
+inline unsigned grid_for(long long work, int threads) {
+    long long blocks = (work + threads - 1) / threads;
+    const long long cap = 148LL * 16;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (unsigned)blocks;
+}
+
+template <int HS>
+cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
+                             const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
+                             int n_head, int T_pad, DevCtx ctx, cudaStream_t s) {
+    using K = BwdCfg<HS>;
+    cudaError_t e = cudaFuncSetAttribute(bwd_bf16_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)K::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int n_t = ceil_div(T, kTile);
+    const long long blocks = (long long)n_t * B * n_head;
+    bwd_bf16_kernel<HS><<<dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s>>>(
+        map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
+                                float *dqacc, int B, int T, int C, int n_head, int T_pad, cudaStream_t s) {
+    const long long work = (long long)B * n_head * T_pad * hs / 4;
+    const unsigned grid = grid_for(work, 256);
+    auto yy = static_cast<const __nv_bfloat16 *>(y);
+    auto gg = static_cast<const __nv_bfloat16 *>(dy);
+    auto zz = reinterpret_cast<float4 *>(dqacc);
+    if (hs == 64)
+        bwd_pre_kernel<64><<<grid, 256, 0, s>>>(yy, gg, lse, D, lse2, zz, B, T, C, n_head, T_pad);
+    else if (hs == 128)
+        bwd_pre_kernel<128><<<grid, 256, 0, s>>>(yy, gg, lse, D, lse2, zz, B, T, C, n_head, T_pad);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
+                                 const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
+                                 const float *D, int B, int T, int C, int n_head, int T_pad, DevCtx ctx,
+                                 cudaStream_t s) {
+    if (hs == 64)
+        return launch_main_impl<64>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
+    if (hs == 128)
+        return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head, int T_pad,
+                                 cudaStream_t s) {
+    const long long work = (long long)B * T * n_head * hs / 8;
+    const unsigned grid = grid_for(work, 256);
+    auto out = static_cast<__nv_bfloat16 *>(dqkv);
+    if (hs == 64)
+        bwd_post_kernel<64><<<grid, 256, 0, s>>>(dqacc, out, B, T, C, n_head, T_pad);
+    else if (hs == 128)
+        bwd_post_kernel<128><<<grid, 256, 0, s>>>(dqacc, out, B, T, C, n_head, T_pad);
+    else
+        return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+}  // namespace gptattn

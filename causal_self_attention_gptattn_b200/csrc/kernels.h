@@ -1,0 +1,73 @@
+// kernels.h -- internal launch interface between the C-ABI layer (api.cu) and
+// the kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gptattn {
+
+// Per-launch device context: where a kernel records a timeout, and how long
+// any single wait may last before it gives up.
+struct DevCtx {
+    int *status;
+    unsigned long long budget_ns;
+};
+
+// Rows per tile along T used by the tensor-core kernels (queries and keys).
+constexpr int kTile = 128;
+
+inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ---- bf16 tensor-core path (sm_100a) --------------------------------------
+// map_qkv: 3-D view (3C, T, B) of qkv, box (64, 128, 1), 128-byte swizzle.
+// map_y:   3-D view (C, T, B) of y, same box.
+cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse,
+                            int B, int T, int C, int n_head, DevCtx ctx, cudaStream_t s);
+
+// D[bh][t] = sum_d y*dy, lse2[bh][t] = lse*log2(e) (rows t >= T: 0 and +inf),
+// dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].
+cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
+                                float *dqacc, int B, int T, int C, int n_head, int T_pad, cudaStream_t s);
+
+// map_dy: 3-D view (C, T, B) of dy; map_dqkv: 3-D view (3C, T, B) of dqkv;
+// map_dq: 2-D view (hs, B*n_head*T_pad) of dqacc (fp32), box (32, 128), 128-byte swizzle.
+cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
+                                 const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
+                                 const float *D, int B, int T, int C, int n_head, int T_pad, DevCtx ctx,
+                                 cudaStream_t s);
+
+// dqkv[b][t][h*hs+d] = bf16(dqacc[(b*n_head+h)*T_pad + t][d] / sqrt(hs)).
+cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head,
+                                 int T_pad, cudaStream_t s);
+
+// ---- fp32 CUDA-core path --------------------------------------------------
+cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head,
+                           cudaStream_t s);
+cudaError_t launch_bwd_f32_pre(int hs, const float *y, const float *dy, float *D, int B, int T, int C,
+                               int n_head, cudaStream_t s);
+cudaError_t launch_bwd_f32_dq(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
+                              float *dqkv, int B, int T, int C, int n_head, cudaStream_t s);
+cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
+                               float *dqkv, int B, int T, int C, int n_head, cudaStream_t s);
+
+// ---- bounded-wait self-test -----------------------------------------------
+cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s);
+
+// Kernel identifiers for the instrumentation records.
+enum KernelId {
+    kKFwdBf16 = 0,
+    kKBwdPreBf16 = 1,
+    kKBwdMainBf16 = 2,
+    kKBwdPostBf16 = 3,
+    kKFwdF32 = 4,
+    kKBwdPreF32 = 5,
+    kKBwdDqF32 = 6,
+    kKBwdDkvF32 = 7,
+    kKSelftest = 8,
+    kKNumKernels = 9
+};
+
+}  // namespace gptattn

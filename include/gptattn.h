@@ -1,0 +1,141 @@
+/*
+ * gptattn.h -- C ABI of libgptattn: batched multi-head causal scaled
+ * dot-product self-attention, forward and backward, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (lecture page "Let's build GPT: from scratch, in code, spelled
+ * out", chapters "version 4: self-attention", "multi-headed self-attention",
+ * note 6 and the two corrections; exercise EX1 for heads as a batch dimension):
+ *
+ *     for every batch b and head h, with q, k, v the head's slices of qkv,
+ *     S[t][s] = q_t . k_s / sqrt(hs)      for s <= t   (the future is masked)
+ *     P[t][:] = softmax(S[t][:])          over the visible s <= t
+ *     y_t     = sum_s P[t][s] v_s
+ *     lse[t]  = ln sum_{s<=t} exp(S[t][s])   (natural log)
+ *
+ * Layout (all row-major, contiguous, no padding):
+ *     qkv  [B][T][3C]  q = columns [0,C), k = [C,2C), v = [2C,3C); head h owns
+ *                      columns [h*hs, (h+1)*hs) of each part (hs = C/n_head).
+ *                      This is the output of a GPT-2 block's c_attn projection.
+ *     y    [B][T][C]   heads concatenated back in the same column order.
+ *     lse  [B][n_head][T]  float32 always.
+ *     dy   [B][T][C], dqkv [B][T][3C]: same layouts as y and qkv.
+ *
+ * Element types: GPTATTN_BF16 -> qkv, y, dy, dqkv are bfloat16 (tensor-core
+ * path, fp32 softmax and accumulation); GPTATTN_F32 -> they are float32 (fp32
+ * CUDA-core path).  lse and the workspace are float32 in both cases.
+ *
+ * Supported head sizes: bf16 hs in {64, 128}; f32 hs in {16, 32, 64, 128}.
+ * Scale is fixed at 1/sqrt(hs); masking is always causal; no dropout.
+ *
+ * Ownership and synchronisation: every pointer is a caller-owned DEVICE
+ * pointer on the current CUDA device, 16-byte aligned.  The library never
+ * allocates device memory per call; the backward's scratch is the caller's
+ * `workspace`.  Calls enqueue kernels on `stream` and return without
+ * synchronising (stream may be NULL for the legacy default stream).  Output
+ * buffers must not overlap inputs.
+ *
+ * Errors: arguments are validated on the host before anything is enqueued;
+ * an invalid call returns a non-zero status and enqueues nothing.  A launch
+ * failure returns GPTATTN_ERR_CUDA.  Kernels never trap: every internal wait
+ * is bounded, and a wait that runs out makes the kernel record
+ * GPTATTN_ERR_TIMEOUT in a device status word and return early (outputs are
+ * then undefined); gptattn_get_device_status() reads and clears that word.
+ * B == 0 or T == 0 is a valid empty call: it returns GPTATTN_OK and touches
+ * nothing (pointers may then be NULL).
+ */
+#ifndef GPTATTN_H
+#define GPTATTN_H
+
+#include <stddef.h>
+
+/* Only the entry points below are exported from libgptattn.so. */
+#if defined(__GNUC__)
+#define GPTATTN_API __attribute__((visibility("default")))
+#else
+#define GPTATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *gptattn_stream_t;
+
+typedef enum gptattn_status {
+    GPTATTN_OK = 0,
+    GPTATTN_ERR_INVALID_ARG = 1,  /* negative size, NULL or misaligned pointer, C % n_head != 0 */
+    GPTATTN_ERR_UNSUPPORTED = 2,  /* head size or dtype outside the supported set */
+    GPTATTN_ERR_CUDA = 3,         /* a CUDA runtime/driver call or a launch failed (no device included) */
+    GPTATTN_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out (reported by get_device_status) */
+    GPTATTN_ERR_WORKSPACE = 5     /* workspace NULL/misaligned or smaller than gptattn_bwd_workspace_bytes */
+} gptattn_status;
+
+typedef enum gptattn_dtype {
+    GPTATTN_F32 = 0,
+    GPTATTN_BF16 = 1
+} gptattn_dtype;
+
+/* Forward.  Reads qkv; writes y and lse.
+ * Causal self-attention forward as defined at the top of this file
+ * ("version 4: self-attention" with the causal mask and 1/sqrt(hs) scale). */
+GPTATTN_API gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse,
+                           int B, int T, int C, int n_head,
+                           gptattn_dtype dt, gptattn_stream_t stream);
+
+/* Bytes of device scratch gptattn_bwd needs for this shape (0 for an empty
+ * shape; (size_t)-1 for an invalid one).  Pure host function. */
+GPTATTN_API size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt);
+
+/* Backward.  Given the forward's qkv, y and lse and the incoming gradient dy,
+ * writes dqkv = d(sum(y o dy))/d(qkv) (chain rule through the weighted sum, the
+ * row softmax and the scaled dot products; same packing as qkv).  `workspace`
+ * is caller-owned device scratch of at least gptattn_bwd_workspace_bytes(...)
+ * bytes, 256-byte aligned; its contents on entry are ignored and on return are
+ * undefined.  Two calls that run concurrently need separate workspaces. */
+GPTATTN_API gptattn_status gptattn_bwd(const void *qkv, const void *y, const float *lse, const void *dy,
+                           void *dqkv, void *workspace, size_t workspace_bytes,
+                           int B, int T, int C, int n_head,
+                           gptattn_dtype dt, gptattn_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: GPTATTN_OK, GPTATTN_ERR_TIMEOUT if a kernel gave up on
+ * a wait since the last call, or GPTATTN_ERR_CUDA if the stream reports an
+ * error. */
+GPTATTN_API gptattn_status gptattn_get_device_status(gptattn_stream_t stream);
+
+/* Static human-readable name of a status code. */
+GPTATTN_API const char *gptattn_status_string(gptattn_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+GPTATTN_API int gptattn_version(void);
+
+/* ---- Instrumentation (no counterpart on the pages; used by the benchmark) --
+ * gptattn_profile_enable(n) with n > 0 makes later calls on the current device
+ * record a pair of CUDA events around each kernel they launch, keeping up to n
+ * records (n = 0 turns recording off and releases the events).  Recording adds
+ * two event records per launch and nothing else.
+ * gptattn_profile_read() synchronises on the recorded events and copies up to
+ * `capacity` (kernel id, milliseconds) pairs, oldest first; it returns the
+ * number copied and clears the record list.  gptattn_kernel_name() maps a
+ * kernel id to a static name.  gptattn_launch_count() is the number of kernels
+ * the library has launched since it was loaded. */
+GPTATTN_API gptattn_status gptattn_profile_enable(int max_records);
+GPTATTN_API int gptattn_profile_read(int *kernel_ids, float *ms, int capacity);
+GPTATTN_API const char *gptattn_kernel_name(int kernel_id);
+GPTATTN_API unsigned long long gptattn_launch_count(void);
+
+/* ---- Bounded-wait self-test (no counterpart on the pages) ------------------
+ * Enqueues one tiny kernel that waits, with the library's bounded-wait
+ * routine, on a barrier that nothing ever completes.  After `budget_ns`
+ * nanoseconds the wait gives up, the kernel records GPTATTN_ERR_TIMEOUT in the
+ * device status word and returns, leaving the context usable.  Used by tests
+ * to show that a lost producer ends in a status code, not a hang or a trap.
+ * budget_ns must be in [1000, 2000000000]. */
+GPTATTN_API gptattn_status gptattn_selftest_wait_timeout(unsigned long long budget_ns, gptattn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTATTN_H */

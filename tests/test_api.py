@@ -1,0 +1,110 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and validates arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from causal_self_attention_gptattn_b200 import gptattn as ga
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptattn.h")
+
+FAKE = 0x7f0000000000  # 16-byte aligned address that is never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptattn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_builds_and_loads():
+    from causal_self_attention_gptattn_b200 import build
+    build.build()
+    assert os.path.exists(ga.LIB_PATH)
+    assert ga.gptattn_version() == 100
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert set(names) == set(ga.EXPORTED), names
+    raw = ctypes.CDLL(ga.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} not exported"
+
+
+def test_only_c_abi_symbols_are_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", ga.LIB_PATH], capture_output=True, text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    ours = {s for s in syms if s.startswith("gptattn_")}
+    assert ours == set(declared_functions())
+
+
+def test_status_strings():
+    for code in range(6):
+        assert ga.gptattn_status_string(code)
+    assert ga.gptattn_kernel_name(2) == "bwd_bf16_sm100"
+    assert ga.gptattn_kernel_name(99) == "unknown"
+
+
+@pytest.mark.parametrize("B,T,C,nh,dt,want", [
+    (-1, 4, 128, 2, ga.GPTATTN_BF16, ga.GPTATTN_ERR_INVALID_ARG),
+    (1, -4, 128, 2, ga.GPTATTN_BF16, ga.GPTATTN_ERR_INVALID_ARG),
+    (1, 4, 0, 2, ga.GPTATTN_BF16, ga.GPTATTN_ERR_INVALID_ARG),
+    (1, 4, 128, 0, ga.GPTATTN_BF16, ga.GPTATTN_ERR_INVALID_ARG),
+    (1, 4, 130, 4, ga.GPTATTN_BF16, ga.GPTATTN_ERR_INVALID_ARG),     # C % n_head != 0
+    (1, 4, 96, 3, ga.GPTATTN_BF16, ga.GPTATTN_ERR_UNSUPPORTED),      # hs = 32 on bf16
+    (1, 4, 96, 4, ga.GPTATTN_F32, ga.GPTATTN_ERR_UNSUPPORTED),       # hs = 24 on fp32
+    (1, 4, 256, 1, ga.GPTATTN_BF16, ga.GPTATTN_ERR_UNSUPPORTED),     # hs = 256
+    (1, 4, 128, 2, 7, ga.GPTATTN_ERR_UNSUPPORTED),                   # bad dtype code
+])
+def test_fwd_shape_validation(B, T, C, nh, dt, want):
+    assert ga.gptattn_fwd(FAKE, FAKE, FAKE, B, T, C, nh, dt, None) == want
+
+
+def test_null_and_misaligned_pointers_rejected():
+    args = (2, 8, 128, 2, ga.GPTATTN_BF16, None)
+    assert ga.gptattn_fwd(None, FAKE, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd(FAKE, None, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd(FAKE, FAKE, None, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd(FAKE + 8, FAKE, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd(FAKE, FAKE + 2, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    ws = ga.gptattn_bwd_workspace_bytes(2, 8, 128, 2, ga.GPTATTN_BF16)
+    assert ga.gptattn_bwd(FAKE, FAKE, FAKE, None, FAKE, FAKE, ws, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, ws, *args) == ga.GPTATTN_ERR_INVALID_ARG
+
+
+def test_workspace_checks():
+    args = (2, 200, 128, 2, ga.GPTATTN_BF16, None)
+    ws = ga.gptattn_bwd_workspace_bytes(2, 200, 128, 2, ga.GPTATTN_BF16)
+    # D + lse*log2e (B*nh*T_pad floats each) + dQ accumulator (B*nh*T_pad*hs floats), 256-byte aligned parts
+    T_pad = 256
+    rows = 2 * 2 * T_pad
+    assert ws == rows * 4 + rows * 4 + rows * 64 * 4
+    assert ga.gptattn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 1, *args) == ga.GPTATTN_ERR_WORKSPACE
+    assert ga.gptattn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, ws, *args) == ga.GPTATTN_ERR_WORKSPACE
+    assert ga.gptattn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 16, ws, *args) == ga.GPTATTN_ERR_WORKSPACE
+    assert ga.gptattn_bwd_workspace_bytes(2, 64, 64, 4, ga.GPTATTN_F32) == 2 * 4 * 64 * 4
+    assert ga.gptattn_bwd_workspace_bytes(2, 64, 65, 4, ga.GPTATTN_F32) == (1 << 64) - 1
+    assert ga.gptattn_bwd_workspace_bytes(0, 64, 64, 4, ga.GPTATTN_F32) == 0
+
+
+def test_empty_calls_are_noops():
+    for dt, C in ((ga.GPTATTN_BF16, 128), (ga.GPTATTN_F32, 64)):
+        assert ga.gptattn_fwd(None, None, None, 0, 16, C, 2, dt, None) == ga.GPTATTN_OK
+        assert ga.gptattn_fwd(None, None, None, 3, 0, C, 2, dt, None) == ga.GPTATTN_OK
+        assert ga.gptattn_bwd(None, None, None, None, None, None, 0, 0, 16, C, 2, dt, None) == ga.GPTATTN_OK
+
+
+def test_selftest_budget_range():
+    assert ga.gptattn_selftest_wait_timeout(10, None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_selftest_wait_timeout(3 * 10**9, None) == ga.GPTATTN_ERR_INVALID_ARG
+
+
+def test_profile_enable_rejects_negative():
+    assert ga.gptattn_profile_enable(-1) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_profile_enable(0) == ga.GPTATTN_OK
+    assert ga.gptattn_profile_read(8) == []

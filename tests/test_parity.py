@@ -1,0 +1,116 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, element by element, at the tolerances in gpu_helpers."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from causal_self_attention_gptattn_b200.workloads import WORKLOADS, make_inputs, workload_inputs
+from gpu_helpers import compare, run_fwd_bwd, select_heads
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_all(qkv, dy, n_head):
+    y, lse = oracle.forward(qkv, n_head)
+    dqkv = oracle.backward(qkv, dy, n_head)
+    return y, lse, dqkv
+
+
+# ---- fp32 CUDA-core path ---------------------------------------------------
+
+def test_fp32_tiny_workload():
+    w = WORKLOADS[1]
+    qkv, dy = workload_inputs(w)
+    got = run_fwd_bwd(qkv, dy, w.n_head)
+    compare(got, oracle_all(qkv, dy, w.n_head), torch.float32, "fp32_tiny")
+
+
+@pytest.mark.parametrize("B,T,n_head,hs", [(1, 77, 2, 32), (2, 130, 2, 64), (1, 65, 1, 128), (3, 1, 2, 16)])
+def test_fp32_shapes(B, T, n_head, hs):
+    qkv, dy = make_inputs(B, T, n_head, hs, dtype=torch.float32, seed=B * 1000 + T + hs)
+    got = run_fwd_bwd(qkv, dy, n_head)
+    compare(got, oracle_all(qkv, dy, n_head), torch.float32, f"fp32 {B},{T},{n_head},{hs}")
+
+
+# ---- bf16 tensor-core path: small cases spanning several tiles + ragged tails -
+
+SMALL = [
+    (1, 1, 1, 64), (2, 17, 2, 64), (1, 127, 2, 64), (2, 128, 2, 64), (1, 129, 2, 64),
+    (2, 200, 3, 64), (1, 384, 2, 64), (1, 300, 1, 64),
+    (1, 1, 1, 128), (2, 17, 2, 128), (1, 129, 2, 128), (2, 200, 2, 128), (1, 384, 1, 128),
+]
+
+
+@pytest.mark.parametrize("B,T,n_head,hs", SMALL)
+def test_bf16_small(B, T, n_head, hs):
+    qkv, dy = make_inputs(B, T, n_head, hs, dtype=torch.bfloat16, seed=7 * B + 11 * T + hs)
+    got = run_fwd_bwd(qkv, dy, n_head)
+    compare(got, oracle_all(qkv, dy, n_head), torch.bfloat16, f"bf16 {B},{T},{n_head},{hs}")
+
+
+def test_bf16_sharp_softmax():
+    """Large-magnitude scores (q and k ~ 4 N(0,1), score std ~ 16, nearly one-hot
+    rows): the online max / rescale path matters.  v stays ~ N(0,1) so that y is
+    representable in bf16 within the y tolerance (|y| ~ 16 would already have a
+    bf16 half-ulp of 0.031)."""
+    qkv, dy = make_inputs(2, 333, 2, 64, dtype=torch.bfloat16, seed=5)
+    C = 2 * 64
+    qkv[:, :, :2 * C] *= 4
+    got = run_fwd_bwd(qkv, dy, 2)
+    compare(got, oracle_all(qkv, dy, 2), torch.bfloat16, "sharp")
+
+
+# ---- full-size workloads, in the configuration the benchmark times ---------
+# The whole tensor is computed on the GPU; the oracle checks a sample of
+# (batch, head) pairs -- batches and heads are independent, so each sampled
+# pair is compared element by element against its exact definition.
+
+SAMPLES = {
+    2: ([0, 37, 63], None),
+    3: ([0, 15], None),
+    4: ([0, 7], [0, 12, 24]),
+    5: ([0], [0, 9, 15]),
+}
+
+
+@pytest.mark.parametrize("idx", [2, 3, 4, 5])
+def test_bf16_full_workload(idx):
+    w = WORKLOADS[idx]
+    qkv, dy = workload_inputs(w)
+    y, lse, dqkv = run_fwd_bwd(qkv, dy, w.n_head)
+    batches, heads = SAMPLES[idx]
+    heads = list(range(w.n_head)) if heads is None else heads
+    q64 = qkv[batches].double().numpy()
+    g64 = dy[batches].double().numpy()
+    q_s = select_heads(q64, w.n_head, 3, heads)
+    g_s = select_heads(g64, w.n_head, 1, heads)
+    ref = oracle_all(q_s, g_s, len(heads))
+    got = (select_heads(y[batches], w.n_head, 1, heads), lse[batches][:, heads],
+           select_heads(dqkv[batches], w.n_head, 3, heads))
+    ey, el, eg, sg = compare(got, ref, torch.bfloat16, w.name)
+    print(f"{w.name}: y {ey:.2e}  lse {el:.2e}  dqkv {eg:.2e} (max|ref| {sg:.2e})")
+
+
+def test_bf16_causality_at_full_size():
+    """Perturbing tokens after position t leaves y and lse at positions <= t
+    bit-identical (no key tile of the future is read for earlier query tiles;
+    inside the diagonal tile the future gets weight exactly zero)."""
+    w = WORKLOADS[3]
+    qkv, dy = workload_inputs(w, B=2)
+    y0, l0, _ = run_fwd_bwd(qkv, dy, w.n_head)
+    t = 700
+    q2 = qkv.clone()
+    q2[:, t + 1:] = torch.randn(q2[:, t + 1:].shape, generator=torch.Generator().manual_seed(3)).to(q2.dtype)
+    y1, l1, _ = run_fwd_bwd(q2, dy, w.n_head)
+    assert np.array_equal(y0[:, :t + 1], y1[:, :t + 1])
+    assert np.array_equal(l0[:, :, :t + 1], l1[:, :, :t + 1])
+
+
+def test_bf16_rows_sum_to_one_at_full_size():
+    """With v = 1 everywhere, every output is the sum of a row of weights: 1."""
+    w = WORKLOADS[5]
+    qkv, dy = workload_inputs(w, B=1)
+    qkv[:, :, 2 * w.C:] = 1.0
+    y, lse, _ = run_fwd_bwd(qkv, dy, w.n_head)
+    assert np.abs(y - 1.0).max() <= 1e-2
