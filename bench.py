@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--workload", default="gpt2_124m")
     p.add_argument("--cpu-sample-seconds", type=float, default=12.0)
     p.add_argument("--skip-cpu-baseline", action="store_true")
+    p.add_argument("--profile-run", action="store_true",
+                   help="warm-up and timed steps only (no clock sampling, e2e or CPU leg): for ncu captures")
     return p.parse_args()
 
 
@@ -227,8 +229,9 @@ def run_ours(args, w, rank, world, local_rank):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     sampler = ClockSampler(local_rank)
-    sampler.start()
-    time.sleep(0.25)
+    if not args.profile_run:
+        sampler.start()
+        time.sleep(0.25)
     ga.gptattn_profile_enable(4 * K + 64)
     launches0 = ga.gptattn_launch_count()
     barrier()
@@ -246,7 +249,7 @@ def run_ours(args, w, rank, world, local_rank):
     prof = ga.gptattn_profile_read(4 * K + 64)
     ga.gptattn_profile_enable(0)
     # keep the same loop running (untimed) so the clock sampler sees >= ~1.5 s of load
-    extra_until = wall0 + 1.5
+    extra_until = wall0 + (0.0 if args.profile_run else 1.5)
     while time.perf_counter() < extra_until:
         for _ in range(50):
             flush.zero_()
@@ -273,7 +276,7 @@ def run_ours(args, w, rank, world, local_rank):
     dqkv_h = torch.empty(dqkv.shape, dtype=dqkv.dtype).pin_memory()
     qkv_d = torch.empty_like(qkv)
     dy_d = torch.empty_like(dy)
-    Ke = max(1, min(K, 200))
+    Ke = 0 if args.profile_run else max(1, min(K, 200))
     e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
     e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
     for _ in range(3):
@@ -294,7 +297,7 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(e_starts, e_ends)))
-    e2e_value = world * Ke * flops / (e2e_ms / 1e3) / 1e12
+    e2e_value = world * Ke * flops / (e2e_ms / 1e3) / 1e12 if Ke else None
     h2d = qkv_h.numel() * qkv_h.element_size() + dy_h.numel() * dy_h.element_size()
     d2h = y_h.numel() * y_h.element_size() + dqkv_h.numel() * dqkv_h.element_size()
 
@@ -317,7 +320,7 @@ def run_ours(args, w, rank, world, local_rank):
                     "traffic": None, "avg_ms": dom_ms}
 
     cpu = None
-    if world == 1 and not args.skip_cpu_baseline:
+    if world == 1 and not (args.skip_cpu_baseline or args.profile_run):
         v, cores, sample, _ = time_oracle(w, args.cpu_sample_seconds)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample}
 
