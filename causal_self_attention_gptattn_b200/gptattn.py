@@ -30,7 +30,7 @@ GPTATTN_BF16 = 1
 EXPORTED = (
     "gptattn_fwd", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
-    "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout",
+    "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
 )
 
 
@@ -85,6 +85,8 @@ def lib():
             L.gptattn_launch_count.restype = ctypes.c_ulonglong
             L.gptattn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, st]
             L.gptattn_selftest_wait_timeout.restype = i
+            L.gptattn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, st]
+            L.gptattn_bwd_noalloc.restype = i
             _lib = L
     return _lib
 
@@ -116,6 +118,17 @@ def gptattn_bwd_workspace_bytes(B, T, C, n_head, dt) -> int:
 def gptattn_bwd(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, dt, stream=None) -> int:
     return lib().gptattn_bwd(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), _ptr(workspace),
                              workspace_bytes, B, T, C, n_head, dt, _stream(stream))
+
+
+def gptattn_bwd_noalloc(qkv, y, lse, dy, dqkv, B, T, C, n_head, dt, stream=None) -> int:
+    """gptattn_bwd without a workspace argument, for callers that cannot allocate:
+    the scratch is a fixed 64 MiB array inside the library (shared by all calls,
+    so calls must not overlap on the GPU)."""
+    return lib().gptattn_bwd_noalloc(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), B, T, C, n_head, dt,
+                                     _stream(stream))
+
+
+GPTATTN_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 
 def gptattn_get_device_status(stream=None) -> int:

@@ -98,6 +98,29 @@ GPTATTN_API gptattn_status gptattn_bwd(const void *qkv, const void *y, const flo
                            int B, int T, int C, int n_head,
                            gptattn_dtype dt, gptattn_stream_t stream);
 
+/* Backward for callers that cannot allocate device memory (no counterpart on
+ * the pages: it is a packaging variant of gptattn_bwd, not part of the
+ * method).  Some callers have no allocator to call -- e.g. a plugin inside
+ * another runtime that owns all device memory -- or must not call cudaMalloc
+ * on their path, since it can synchronise the device.  This entry point takes
+ * the same arguments as gptattn_bwd minus the workspace: the scratch comes
+ * from one array of GPTATTN_NOALLOC_SCRATCH_BYTES (64 MiB) compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  The caller still owns and passes every input and output.
+ * Returns GPTATTN_ERR_WORKSPACE, enqueueing nothing, when the shape needs more
+ * scratch than that (gptattn_bwd_workspace_bytes(...) > 64 MiB).  It allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the previous call's
+ * contents (the backward re-initialises what it needs); calls whose work
+ * overlaps on the GPU -- on two streams or from two host threads -- race on it
+ * and produce wrong results, so serialise them. */
+#define GPTATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+GPTATTN_API gptattn_status gptattn_bwd_noalloc(const void *qkv, const void *y, const float *lse, const void *dy,
+                                               void *dqkv, int B, int T, int C, int n_head,
+                                               gptattn_dtype dt, gptattn_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: GPTATTN_OK, GPTATTN_ERR_TIMEOUT if a kernel gave up on
  * a wait since the last call, or GPTATTN_ERR_CUDA if the stream reports an
