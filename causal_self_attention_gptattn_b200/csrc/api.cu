@@ -36,7 +36,13 @@ std::mutex g_mutex;
 int *g_status_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_launches{0};
 
-gptattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GPTATTN_OK : GPTATTN_ERR_CUDA; }
+thread_local const char *t_last_error = "no error";
+
+gptattn_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return GPTATTN_OK;
+    t_last_error = cudaGetErrorString(e);
+    return GPTATTN_ERR_CUDA;
+}
 
 // Device address of g_device_status for the current device (looked up once
 // per device, with that device current).
@@ -244,6 +250,8 @@ const char *gptattn_status_string(gptattn_status s) {
 }
 
 int gptattn_version(void) { return 100; }
+
+const char *gptattn_last_error_string(void) { return t_last_error; }
 
 gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, gptattn_dtype dt,
                            gptattn_stream_t stream) {

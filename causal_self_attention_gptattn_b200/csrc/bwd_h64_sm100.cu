@@ -1,0 +1,489 @@
+// bwd_h64_sm100.cu -- persistent bf16 causal self-attention backward, head size 64.
+//
+// Same mathematics as bwd_sm100.cu (chain rule through "version 3: adding
+// softmax" and "version 4: self-attention" of the lecture page "Let's build
+// GPT: from scratch, in code, spelled out"; P recomputed from the saved
+// logsumexp):  dV += P^T dY,  dP = dY V^T,  dS = P o (dP - D),
+//              dK += dS^T Q * scale,  dQ += dS K * scale.
+//
+// Schedule: one persistent CTA per SM walks a static list of work items
+// (key tile j, batch b, head h), ordered longest first (small j first), with
+// stride gridDim.x.  Per item the CTA loops over query tiles i >= j.
+//
+// Warp roles (14 warps):
+//   warp 0        TMA producer: K_j, V_j (double-buffered across items), and
+//                 Q_i, dO_i, lse_i, D_i through a 3-stage ring
+//   warp 1        TMEM owner + MMA issuer
+//   warps 2..9    softmax: TMEM sub-partition warp%4 (32 key rows), column
+//                 half (warp-2)/4 (64 query columns): P^T, dS^T, dK/dV epilogue
+//   warps 10..13  dQ drain: TMEM -> smem (fp32, swizzled) -> TMA reduce-add
+// TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T [256,320) (bf16 pairs)
+//                     dV [320,384)  dK [384,448)  dQ [448,512)
+// MMA order per item: S_0 dP_0 | S_1 dV_0 dK_0 dQ_0 dP_1 | S_2 dV_1 ...
+// S^T and dP^T are released as soon as the softmax warps hold them in
+// registers, so the tensor pipe computes tile i+1 while tile i is in softmax.
+// Every wait is bounded; roles never leave their loops early, so all named
+// barriers are reached the same number of times by every thread of a role.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace gptattn {
+namespace {
+
+constexpr int kThreads = 448;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlabBytes = 128 * 128;
+constexpr int HS = 64;
+constexpr uint32_t kTileBytes = 128u * 64u * 2u;  // one 128 x 64 bf16 tile = one slab
+constexpr int kQStages = 3;
+constexpr int kKVStages = 2;
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr uint32_t kOffK = 0;                                   // kKVStages tiles
+constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;       // kKVStages tiles
+constexpr uint32_t kOffQ = kOffV + kKVStages * kTileBytes;       // kQStages tiles
+constexpr uint32_t kOffdO = kOffQ + kQStages * kTileBytes;       // kQStages tiles
+constexpr uint32_t kOffdS = kOffdO + kQStages * kTileBytes;      // 128 x 128 bf16 (2 slabs)
+constexpr uint32_t kOffdQ = kOffdS + 2 * kSlabBytes;             // 128 x 32 fp32 staging (1 slab)
+constexpr uint32_t kOffLse = kOffdQ + kSlabBytes;                // kQStages x 128 fp32
+constexpr uint32_t kOffD = kOffLse + kQStages * 512;             // kQStages x 128 fp32
+constexpr uint32_t kOffBar = kOffD + kQStages * 512;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+// TMEM columns
+constexpr uint32_t kColS = 0, kColdP = 128, kColP = 256, kColdV = 320, kColdK = 384, kColdQ = 448;
+
+// barriers
+constexpr int kBarKVFull = 0;                      // kKVStages
+constexpr int kBarKVEmpty = kBarKVFull + kKVStages;  // kKVStages
+constexpr int kBarQFull = kBarKVEmpty + kKVStages;   // kQStages
+constexpr int kBarQEmpty = kBarQFull + kQStages;     // kQStages
+constexpr int kBarSFull = kBarQEmpty + kQStages;
+constexpr int kBarSEmpty = kBarSFull + 1;
+constexpr int kBardPFull = kBarSEmpty + 1;
+constexpr int kBardPEmpty = kBardPFull + 1;
+constexpr int kBarPFull = kBardPEmpty + 1;
+constexpr int kBarPEmpty = kBarPFull + 1;
+constexpr int kBardSFull = kBarPEmpty + 1;
+constexpr int kBardSEmpty = kBardSFull + 1;
+constexpr int kBardQFull = kBardSEmpty + 1;
+constexpr int kBardQEmpty = kBardQFull + 1;
+constexpr int kBarKdV = kBardQEmpty + 1;
+constexpr int kBarAccFree = kBarKdV + 1;
+constexpr int kBarDone = kBarAccFree + 1;
+constexpr int kNumBars = kBarDone + 1;
+static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
+
+constexpr int kSoftmaxThreads = 256;
+constexpr int kDrainThreads = 128;
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitGuard &g) {
+    bool ok = mbar_wait(bar, parity, g);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > budget_ns) break;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_h64_persistent(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
+                       const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
+                       const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C,
+                       int n_head, int T_pad, int n_t, int *status, unsigned long long budget_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int BH = B * n_head;
+    const int n_items = n_t * BH;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    auto bar = [&](int idx) -> uint32_t { return smem_u32(&bars[idx]); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + kNumBars * 8 + 4);
+    const WaitGuard g{abort_flag, status, budget_ns};
+
+    auto sK = [&](int s) -> uint32_t { return sbase + kOffK + s * kTileBytes; };
+    auto sV = [&](int s) -> uint32_t { return sbase + kOffV + s * kTileBytes; };
+    auto sQ = [&](int s) -> uint32_t { return sbase + kOffQ + s * kTileBytes; };
+    auto sdO = [&](int s) -> uint32_t { return sbase + kOffdO + s * kTileBytes; };
+    const uint32_t sdS = sbase + kOffdS, sdQ = sbase + kOffdQ;
+    const float *sLse = reinterpret_cast<const float *>(smem + kOffLse);
+    const float *sD = reinterpret_cast<const float *>(smem + kOffD);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kKVStages; ++s) {
+            mbar_init(bar(kBarKVFull + s), 1);
+            mbar_init(bar(kBarKVEmpty + s), 1);
+        }
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(bar(kBarQFull + s), 1);
+            mbar_init(bar(kBarQEmpty + s), 1);
+        }
+        mbar_init(bar(kBarSFull), 1);
+        mbar_init(bar(kBarSEmpty), kSoftmaxThreads);
+        mbar_init(bar(kBardPFull), 1);
+        mbar_init(bar(kBardPEmpty), kSoftmaxThreads);
+        mbar_init(bar(kBarPFull), kSoftmaxThreads);
+        mbar_init(bar(kBarPEmpty), 1);
+        mbar_init(bar(kBardSFull), kSoftmaxThreads);
+        mbar_init(bar(kBardSEmpty), 1);
+        mbar_init(bar(kBardQFull), 1);
+        mbar_init(bar(kBardQEmpty), kDrainThreads);
+        mbar_init(bar(kBarKdV), 1);
+        mbar_init(bar(kBarAccFree), kSoftmaxThreads);
+        mbar_init(bar(kBarDone), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================================ producer
+        if (lane == 0) {
+            tma_prefetch_map(&map_qkv);
+            tma_prefetch_map(&map_dy);
+            bool ok = true;
+            int n = 0;   // items started
+            int gq = 0;  // query tiles issued (ring position)
+            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++n) {
+                const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
+                const int kvs = n & 1;
+                if (n >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + kvs), (uint32_t)((n >> 1) & 1) ^ 1u, g)))
+                    break;
+                mbar_arrive_expect_tx(bar(kBarKVFull + kvs), 2 * kTileBytes);
+                tma_load_3d(sK(kvs), &map_qkv, bar(kBarKVFull + kvs), C + h * HS, kt * kTile, b);
+                tma_load_3d(sV(kvs), &map_qkv, bar(kBarKVFull + kvs), 2 * C + h * HS, kt * kTile, b);
+                for (int qt = kt; qt < n_t; ++qt, ++gq) {
+                    const int st = gq % kQStages;
+                    const uint32_t ph = (uint32_t)(gq / kQStages) & 1u;
+                    if (gq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + st), ph ^ 1u, g))) break;
+                    const uint32_t fb = bar(kBarQFull + st);
+                    mbar_arrive_expect_tx(fb, 2 * kTileBytes + 1024);
+                    tma_load_3d(sQ(st), &map_qkv, fb, h * HS, qt * kTile, b);
+                    tma_load_3d(sdO(st), &map_dy, fb, h * HS, qt * kTile, b);
+                    const size_t rowoff = (size_t)bh * (size_t)T_pad + (size_t)qt * kTile;
+                    bulk_load(sbase + kOffLse + st * 512, lse2 + rowoff, 512, fb);
+                    bulk_load(sbase + kOffD + st * 512, Dvec + rowoff, 512, fb);
+                }
+            }
+            if (!ok || *abort_flag) {
+                // let the last copies of each buffer land before shared memory is released
+                for (int k = (n > kKVStages ? n - kKVStages : 0); k < n; ++k)
+                    drain_wait(bar(kBarKVFull + (k & 1)), (uint32_t)(k >> 1) & 1u, budget_ns);
+                for (int k = (gq > kQStages ? gq - kQStages : 0); k < gq; ++k)
+                    drain_wait(bar(kBarQFull + k % kQStages), (uint32_t)(k / kQStages) & 1u, budget_ns);
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idSS = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t idAcc = idesc_bf16_f32(128, HS, false, true);
+            constexpr uint32_t idQ = idesc_bf16_f32(128, HS, true, true);
+            bool ok = true, any = false;
+            int n = 0, gi = 0;
+            auto issue_S = [&](int kvs, int st) {
+#pragma unroll
+                for (int kk = 0; kk < HS / 16; ++kk)
+                    umma_ss(tmem + kColS, sdesc_sw128(sK(kvs) + kk * 32u, 16, 1024),
+                            sdesc_sw128(sQ(st) + kk * 32u, 16, 1024), idSS, kk > 0 ? 1u : 0u);
+                umma_commit(bar(kBarSFull));
+            };
+            auto issue_dP = [&](int kvs, int st) {
+#pragma unroll
+                for (int kk = 0; kk < HS / 16; ++kk)
+                    umma_ss(tmem + kColdP, sdesc_sw128(sV(kvs) + kk * 32u, 16, 1024),
+                            sdesc_sw128(sdO(st) + kk * 32u, 16, 1024), idSS, kk > 0 ? 1u : 0u);
+                umma_commit(bar(kBardPFull));
+            };
+            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++n) {
+                const int kt = w / BH;
+                const int niter = n_t - kt;
+                const int kvs = n & 1;
+                if (!(ok = mbar_wait(bar(kBarKVFull + kvs), (uint32_t)(n >> 1) & 1u, g))) break;
+                // first S and dP of this item
+                if (!(ok = mbar_wait(bar(kBarQFull + gi % kQStages), (uint32_t)(gi / kQStages) & 1u, g))) break;
+                if (gi > 0 && !(ok = mbar_wait(bar(kBarSEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                tc_fence_after();
+                issue_S(kvs, gi % kQStages);
+                any = true;
+                if (gi > 0 && !(ok = mbar_wait(bar(kBardPEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                tc_fence_after();
+                issue_dP(kvs, gi % kQStages);
+                for (int it = 0; it < niter; ++it, ++gi) {
+                    const int st = gi % kQStages;
+                    const int st1 = (gi + 1) % kQStages;
+                    const bool more = it + 1 < niter;
+                    const uint32_t ph = (uint32_t)gi & 1u;
+                    if (more) {  // S^T of the next query tile
+                        if (!(ok = mbar_wait(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u, g))) break;
+                        if (!(ok = mbar_wait(bar(kBarSEmpty), ph, g))) break;
+                        tc_fence_after();
+                        issue_S(kvs, st1);
+                    }
+                    // dV += P^T dO
+                    if (!(ok = mbar_wait(bar(kBarPFull), ph, g))) break;
+                    if (it == 0 && n > 0 && !(ok = mbar_wait(bar(kBarAccFree), (uint32_t)(n - 1) & 1u, g))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, sdesc_sw128(sdO(st) + kk * 2048u, kSlabBytes, 1024),
+                                idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(bar(kBarPEmpty));
+                    // dK += dS^T Q ; dQ = dS K
+                    if (!(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
+                        umma_ss(tmem + kColdK, sdesc_sw128(sdS + koff, 16, 1024),
+                                sdesc_sw128(sQ(st) + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    if (gi > 0 && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ss(tmem + kColdQ, sdesc_sw128(sdS + kk * 2048u, kSlabBytes, 1024),
+                                sdesc_sw128(sK(kvs) + kk * 2048u, kSlabBytes, 1024), idQ, kk > 0 ? 1u : 0u);
+                    umma_commit(bar(kBardQFull));
+                    umma_commit(bar(kBardSEmpty));
+                    umma_commit(bar(kBarQEmpty + st));
+                    if (more) {  // dP^T of the next query tile
+                        if (!(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
+                        tc_fence_after();
+                        issue_dP(kvs, st1);
+                    }
+                }
+                if (!ok) break;
+                umma_commit(bar(kBarKdV));
+                umma_commit(bar(kBarKVEmpty + kvs));
+            }
+            if (any) {
+                umma_commit(bar(kBarDone));
+                drain_wait(bar(kBarDone), 0, budget_ns);
+            }
+        }
+    } else if (warp < 10) {
+        // ================================================================ softmax warps
+        const int sp = warp & 3;                 // TMEM sub-partition: key rows 32*sp .. 32*sp+31
+        const int half = (warp - 2) >> 2;        // query columns 64*half .. 64*half+63
+        const int row = sp * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
+        const float scale_log2 = 0.125f * 1.4426950408889634f;
+        const uint64_t c2 = f32x2_pack(scale_log2, scale_log2);
+        bool ok = true;
+        int n = 0, gi = 0;
+        for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++n) {
+            const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
+            const int niter = n_t - kt;
+            for (int it = 0; it < niter; ++it, ++gi) {
+                const int st = gi % kQStages;
+                const uint32_t ph = (uint32_t)gi & 1u;
+                if (ok) ok = warp_wait(bar(kBarQFull + st), (uint32_t)(gi / kQStages) & 1u, g);
+                if (ok) ok = warp_wait(bar(kBarSFull), ph, g);
+                float pf[64];  // P^T row segment, fp32
+                if (ok) {
+                    tc_fence_after();
+                    uint32_t sr[64];
+                    tmem_ld_x32(trow + kColS + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld_x32(trow + kColS + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                    tc_fence_before();
+                    mbar_arrive(bar(kBarSEmpty));
+                    const float4 *lse4 = reinterpret_cast<const float4 *>(sLse + st * 128 + 64 * half);
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        const float4 l = lse4[c4];
+                        const int c = 4 * c4;
+                        const uint64_t x01 = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2,
+                                                   f32x2_pack(-l.x, -l.y));
+                        const uint64_t x23 = ffma2(f32x2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])),
+                                                   c2, f32x2_pack(-l.z, -l.w));
+                        float x0, x1, x2, x3;
+                        f32x2_unpack(x01, x0, x1);
+                        f32x2_unpack(x23, x2, x3);
+                        pf[c] = ex2_approx(x0);
+                        pf[c + 1] = ex2_approx(x1);
+                        pf[c + 2] = ex2_approx(x2);
+                        pf[c + 3] = ex2_approx(x3);
+                    }
+                    if (it == 0) {  // diagonal tile: query column q sees key `row` only if row <= q
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (64 * half + c < row) pf[c] = 0.f;
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
+                    if (gi > 0) ok = warp_wait(bar(kBarPEmpty), (uint32_t)(gi - 1) & 1u, g);
+                    if (ok) {
+                        tmem_st_x32(trow + kColP + 32 * half, pk);
+                        tmem_st_wait();
+                        tc_fence_before();
+                        mbar_arrive(bar(kBarPFull));
+                    }
+                }
+                if (ok) ok = warp_wait(bar(kBardPFull), ph, g);
+                if (ok && gi > 0) ok = warp_wait(bar(kBardSEmpty), (uint32_t)(gi - 1) & 1u, g);
+                if (ok) {
+                    tc_fence_after();
+                    const float4 *D4 = reinterpret_cast<const float4 *>(sD + st * 128 + 64 * half);
+                    // dS^T row `row`, query columns [64*half, 64*half+64) = slab `half`, chunks 0..7
+                    const uint32_t rbase = sdS + (uint32_t)half * kSlabBytes + (uint32_t)row * 128u;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        uint32_t dr[32];
+                        tmem_ld_x32(trow + kColdP + 64 * half + 32 * part, dr);
+                        if (part == 1) {
+                            tc_fence_before();
+                            mbar_arrive(bar(kBardPEmpty));
+                        }
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+                            const int q = 4 * part + qq;  // 16-byte chunk = 8 query columns
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float4 d = D4[2 * q + e];
+                                const int c = 8 * q + 4 * e;      // column within the half
+                                const int cr = 8 * qq + 4 * e;    // column within this dP chunk
+                                const uint64_t a01 = fadd2(f32x2_pack(__uint_as_float(dr[cr]), __uint_as_float(dr[cr + 1])),
+                                                           f32x2_pack(-d.x, -d.y));
+                                const uint64_t a23 = fadd2(f32x2_pack(__uint_as_float(dr[cr + 2]), __uint_as_float(dr[cr + 3])),
+                                                           f32x2_pack(-d.z, -d.w));
+                                const uint64_t s01 = fmul2(a01, f32x2_pack(pf[c], pf[c + 1]));
+                                const uint64_t s23 = fmul2(a23, f32x2_pack(pf[c + 2], pf[c + 3]));
+                                float s0, s1, s2, s3;
+                                f32x2_unpack(s01, s0, s1);
+                                f32x2_unpack(s23, s2, s3);
+                                wv[2 * e] = pack_bf16x2(s0, s1);
+                                wv[2 * e + 1] = pack_bf16x2(s2, s3);
+                            }
+                            st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), wv[0], wv[1], wv[2], wv[3]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar(kBardSFull));
+                }
+            }
+            // ---------------------------------------------------- dK / dV epilogue of this item
+            // staging: the dS buffer (free once the item's last dQ retired): dV -> slab 0, dK -> slab 1
+            if (ok) ok = warp_wait(bar(kBarKdV), (uint32_t)n & 1u, g);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t col = half == 0 ? kColdV : kColdK;
+                const float mul = half == 0 ? 1.f : 0.125f;
+                uint32_t o[64];
+                tmem_ld_x32(trow + col, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                tmem_ld_x32(trow + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                tc_fence_before();
+                mbar_arrive(bar(kBarAccFree));
+                const uint32_t rbase = sdS + (uint32_t)half * kSlabBytes + (uint32_t)row * 128u;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    uint32_t wv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(o[8 * q + 2 * e]) * mul,
+                                            __uint_as_float(o[8 * q + 2 * e + 1]) * mul);
+                    st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), wv[0], wv[1], wv[2], wv[3]);
+                }
+                fence_proxy_async_smem();
+            }
+            named_bar_sync(1, kSoftmaxThreads);
+            if (warp == 2 && lane == 0 && ok && !*abort_flag) {
+                tma_store_3d(&map_dqkv, sdS, 2 * C + h * HS, kt * kTile, b);
+                tma_store_3d(&map_dqkv, sdS + kSlabBytes, C + h * HS, kt * kTile, b);
+                bulk_commit_group();
+                bulk_wait_group_read_0();  // staging may be overwritten by the next item's dS
+            }
+            named_bar_sync(1, kSoftmaxThreads);
+        }
+        if (warp == 2 && lane == 0) bulk_wait_group_0();
+    } else {
+        // ================================================================ dQ drain warps
+        const int sp = warp & 3;
+        const int row = sp * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
+        const bool leader = (warp == 10 && lane == 0);
+        bool ok = true;
+        int gi = 0;
+        for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+            const int kt = w / BH, bh = w % BH;
+            for (int qt = kt; qt < n_t; ++qt, ++gi) {
+                if (ok) ok = warp_wait(bar(kBardQFull), (uint32_t)gi & 1u, g);
+                uint32_t v[64];
+                if (ok) {
+                    tc_fence_after();
+                    tmem_ld_x32(trow + kColdQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                    tmem_ld_x32(trow + kColdQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                    tc_fence_before();
+                    mbar_arrive(bar(kBardQEmpty));
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {  // two 32-column halves through one 16 KB staging slab
+                    if (leader) bulk_wait_group_read_0();
+                    named_bar_sync(2, kDrainThreads);
+                    if (ok) {
+                        const uint32_t rbase = sdQ + (uint32_t)row * 128u;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), v[32 * hh + 4 * q],
+                                         v[32 * hh + 4 * q + 1], v[32 * hh + 4 * q + 2], v[32 * hh + 4 * q + 3]);
+                        fence_proxy_async_smem();
+                    }
+                    named_bar_sync(2, kDrainThreads);
+                    if (leader && ok && !*abort_flag) {
+                        tma_reduce_add_2d(&map_dq, sdQ, 32 * hh, bh * T_pad + qt * kTile);
+                        bulk_commit_group();
+                    }
+                }
+            }
+        }
+        if (leader) bulk_wait_group_0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
+                                const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
+                                int n_head, int T_pad, DevCtx ctx, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_h64_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int n_t = ceil_div(T, kTile);
+    const long long items = (long long)n_t * B * n_head;
+    const int grid = (int)(items < sms ? items : sms);
+    bwd_h64_persistent<<<dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s>>>(
+        map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace gptattn

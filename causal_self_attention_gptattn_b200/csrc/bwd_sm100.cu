@@ -532,7 +532,7 @@ cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUten
                                  const float *D, int B, int T, int C, int n_head, int T_pad, DevCtx ctx,
                                  cudaStream_t s) {
     if (hs == 64)
-        return launch_main_impl<64>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
+        return launch_bwd_main_h64(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
     if (hs == 128)
         return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
     return cudaErrorInvalidValue;

@@ -213,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
         const float scale_log2 = rsqrtf((float)HS) * 1.4426950408889634f;
         float m = -INFINITY;  // running max of scaled scores (log2 units)
-        float l = 0.f;        // running normaliser
+        float l = 0.f;        // running normaliser (fp32 weights)
+        float l_r = 0.f;      // running normaliser (bf16-rounded weights)
         bool ok = true;
         for (int j = 0; j < nkv; ++j) {
             ok = warp_wait(bar(K::kBarS + (j & 1)), (uint32_t)(j >> 1) & 1u, g);
@@ -231,24 +232,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 128; ++c)
                     if (c > row) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max with 8 independent partial maxima (no 128-long dependency chain)
+            float mp[8];
 #pragma unroll
-            for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-            const float m_new = fmaxf(m, mx * scale_log2);
-            const float alpha = ex2_approx(m - m_new);
+            for (int k = 0; k < 8; ++k) mp[k] = s[k];
+#pragma unroll
+            for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+            // Lazy rescaling: keep the running max unless it grows by more than
+            // 8 (log2 units).  p stays <= 2^8 and l, O use the same stale max,
+            // so y = O / l and lse = m + log2 l are exact; O is rescaled rarely.
+            const float m_cand = mx * scale_log2;
+            const bool grow = m_cand > m + 8.f;
+            const float m_new = grow ? m_cand : m;
+            const float alpha = grow ? ex2_approx(m - m_new) : 1.f;
             const float neg = -m_new;
-            float sum = 0.f;
+            // Two row sums: of the fp32 weights (for lse) and of the bf16-rounded
+            // weights the P V product actually uses (to normalise y, so that a
+            // row dominated by one key returns that key's value exactly).
+            float sp8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            float sr8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[64];
 #pragma unroll
             for (int c = 0; c < 128; c += 2) {
                 const float p0 = ex2_approx(fmaf(s[c], scale_log2, neg));
                 const float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, neg));
-                sum += p0 + p1;
-                pk[c >> 1] = pack_bf16x2(p0, p1);
+                sp8[(c >> 1) & 7] += p0 + p1;
+                const uint32_t w = pack_bf16x2(p0, p1);
+                sr8[(c >> 1) & 7] += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+                pk[c >> 1] = w;
             }
+            const float sum = ((sp8[0] + sp8[1]) + (sp8[2] + sp8[3])) + ((sp8[4] + sp8[5]) + (sp8[6] + sp8[7]));
+            const float sum_r = ((sr8[0] + sr8[1]) + (sr8[2] + sr8[3])) + ((sr8[4] + sr8[5]) + (sr8[6] + sr8[7]));
             tmem_st_x32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
             tmem_st_x32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
             l = l * alpha + sum;
+            l_r = l_r * alpha + sum_r;
             m = m_new;
             if (j > 0) {
                 // rescale O once the previous P V product has landed
@@ -274,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) ok = warp_wait(bar(K::kBarO), (uint32_t)(nkv - 1) & 1u, g);
         if (ok) {
             tc_fence_after();
-            const float inv_l = 1.f / l;
+            const float inv_l = 1.f / l_r;
 #pragma unroll
             for (int c0 = 0; c0 < HS; c0 += 32) {
                 uint32_t o[32];

@@ -39,6 +39,11 @@ cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUten
                                  const float *D, int B, int T, int C, int n_head, int T_pad, DevCtx ctx,
                                  cudaStream_t s);
 
+// Persistent head-size-64 variant of the above (same arguments).
+cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
+                                const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
+                                int n_head, int T_pad, DevCtx ctx, cudaStream_t s);
+
 // dqkv[b][t][h*hs+d] = bf16(dqacc[(b*n_head+h)*T_pad + t][d] / sqrt(hs)).
 cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head,
                                  int T_pad, cudaStream_t s);

@@ -31,6 +31,7 @@ EXPORTED = (
     "gptattn_fwd", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
     "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
+    "gptattn_last_error_string",
 )
 
 
@@ -41,7 +42,13 @@ class LibraryNotBuilt(RuntimeError):
 class GptAttnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == GPTATTN_ERR_CUDA:
+            try:
+                detail = f": {gptattn_last_error_string()}"
+            except LibraryNotBuilt:
+                pass
+        super().__init__(f"{where}: {status_string(status)}{detail} (status {status})")
 
 
 _lock = threading.Lock()
@@ -87,6 +94,8 @@ def lib():
             L.gptattn_selftest_wait_timeout.restype = i
             L.gptattn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, st]
             L.gptattn_bwd_noalloc.restype = i
+            L.gptattn_last_error_string.argtypes = []
+            L.gptattn_last_error_string.restype = ctypes.c_char_p
             _lib = L
     return _lib
 
@@ -144,6 +153,10 @@ def status_string(status: int) -> str:
         return gptattn_status_string(status)
     except LibraryNotBuilt:
         return f"status {status}"
+
+
+def gptattn_last_error_string() -> str:
+    return lib().gptattn_last_error_string().decode()
 
 
 def gptattn_version() -> int:

@@ -130,6 +130,10 @@ GPTATTN_API gptattn_status gptattn_get_device_status(gptattn_stream_t stream);
 /* Static human-readable name of a status code. */
 GPTATTN_API const char *gptattn_status_string(gptattn_status s);
 
+/* Text of the last CUDA error that made a call on this host thread return
+ * GPTATTN_ERR_CUDA ("no error" if none yet).  Static string. */
+GPTATTN_API const char *gptattn_last_error_string(void);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 GPTATTN_API int gptattn_version(void);
 

@@ -49,10 +49,8 @@ def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream
     nbytes = ga.gptattn_bwd_workspace_bytes(B, T, C, n_head, dt)
     ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
-    rc = ga.gptattn_fwd(qkv, y.view, lse.view, B, T, C, n_head, dt, s)
-    assert rc == ga.GPTATTN_OK, ga.status_string(rc)
-    rc = ga.gptattn_bwd(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, dt, s)
-    assert rc == ga.GPTATTN_OK, ga.status_string(rc)
+    ga.check(ga.gptattn_fwd(qkv, y.view, lse.view, B, T, C, n_head, dt, s), "gptattn_fwd")
+    ga.check(ga.gptattn_bwd(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, dt, s), "gptattn_bwd")
     rc = ga.gptattn_get_device_status(s)
     assert rc == ga.GPTATTN_OK, ga.status_string(rc)
     assert y.intact() and lse.intact() and dqkv.intact(), "write outside an output buffer"
