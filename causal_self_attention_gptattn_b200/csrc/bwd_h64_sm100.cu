@@ -5,6 +5,7 @@
 // GPT: from scratch, in code, spelled out"; P recomputed from the saved
 // logsumexp):  dV += P^T dY,  dP = dY V^T,  dS = P o (dP - D),
 //              dK += dS^T Q * scale,  dQ += dS K * scale.
+// The workspace rows hold -D and -lse*log2(e) (negated by the preprocess kernel).
 //
 // Schedule: one persistent CTA per SM walks a static list of work items
 // (key tile j, batch b, head h), ordered longest first (small j first), with
@@ -196,20 +197,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idSS = idesc_bf16_f32(128, 128, false, false);
             constexpr uint32_t idAcc = idesc_bf16_f32(128, HS, false, true);
             constexpr uint32_t idQ = idesc_bf16_f32(128, HS, true, true);
+            // Descriptors of every buffer, built once.  K-major views: rows of 128 B,
+            // 8-row groups 1024 B apart.  N/M-major views: 8-row groups 1024 B apart,
+            // 64-element column blocks one slab apart.  A k-step moves the start address.
+            const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024), dV0 = sdesc_sw128(sV(0), 16, 1024);
+            const uint64_t dQ0 = sdesc_sw128(sQ(0), 16, 1024), ddO0 = sdesc_sw128(sdO(0), 16, 1024);
+            const uint64_t ddOmn0 = sdesc_sw128(sdO(0), kSlabBytes, 1024), dQmn0 = sdesc_sw128(sQ(0), kSlabBytes, 1024);
+            const uint64_t dKmn0 = sdesc_sw128(sK(0), kSlabBytes, 1024);
+            const uint64_t ddS = sdesc_sw128(sdS, 16, 1024), ddSmn = sdesc_sw128(sdS, kSlabBytes, 1024);
+            auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
             bool ok = true, any = false;
             int n = 0, gi = 0;
             auto issue_S = [&](int kvs, int st) {
+                const uint64_t a = at(dK0, kvs * kTileBytes), b = at(dQ0, st * kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < HS / 16; ++kk)
-                    umma_ss(tmem + kColS, sdesc_sw128(sK(kvs) + kk * 32u, 16, 1024),
-                            sdesc_sw128(sQ(st) + kk * 32u, 16, 1024), idSS, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + kColS, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
                 umma_commit(bar(kBarSFull));
             };
             auto issue_dP = [&](int kvs, int st) {
+                const uint64_t a = at(dV0, kvs * kTileBytes), b = at(ddO0, st * kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < HS / 16; ++kk)
-                    umma_ss(tmem + kColdP, sdesc_sw128(sV(kvs) + kk * 32u, 16, 1024),
-                            sdesc_sw128(sdO(st) + kk * 32u, 16, 1024), idSS, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + kColdP, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
                 umma_commit(bar(kBardPFull));
             };
             for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++n) {
@@ -241,26 +251,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!(ok = mbar_wait(bar(kBarPFull), ph, g))) break;
                     if (it == 0 && n > 0 && !(ok = mbar_wait(bar(kBarAccFree), (uint32_t)(n - 1) & 1u, g))) break;
                     tc_fence_after();
+                    {
+                        const uint64_t b = at(ddOmn0, st * kTileBytes);
+                        const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, sdesc_sw128(sdO(st) + kk * 2048u, kSlabBytes, 1024),
-                                idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, at(b, kk * 2048u), idAcc, kk > 0 ? 1u : acc);
+                    }
                     umma_commit(bar(kBarPEmpty));
                     // dK += dS^T Q ; dQ = dS K
                     if (!(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
                     tc_fence_after();
+                    {
+                        const uint64_t b = at(dQmn0, st * kTileBytes);
+                        const uint32_t acc = it > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
-                        umma_ss(tmem + kColdK, sdesc_sw128(sdS + koff, 16, 1024),
-                                sdesc_sw128(sQ(st) + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_ss(tmem + kColdK, at(ddS, (kk >> 2) * kSlabBytes + (kk & 3) * 32u), at(b, kk * 2048u),
+                                    idAcc, kk > 0 ? 1u : acc);
                     }
                     if (gi > 0 && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
                     tc_fence_after();
+                    {
+                        const uint64_t b = at(dKmn0, kvs * kTileBytes);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_ss(tmem + kColdQ, sdesc_sw128(sdS + kk * 2048u, kSlabBytes, 1024),
-                                sdesc_sw128(sK(kvs) + kk * 2048u, kSlabBytes, 1024), idQ, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_ss(tmem + kColdQ, at(ddSmn, kk * 2048u), at(b, kk * 2048u), idQ, kk > 0 ? 1u : 0u);
+                    }
                     umma_commit(bar(kBardQFull));
                     umma_commit(bar(kBardSEmpty));
                     umma_commit(bar(kBarQEmpty + st));
@@ -311,9 +328,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float4 l = lse4[c4];
                         const int c = 4 * c4;
                         const uint64_t x01 = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2,
-                                                   f32x2_pack(-l.x, -l.y));
+                                                   f32x2_pack(l.x, l.y));
                         const uint64_t x23 = ffma2(f32x2_pack(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])),
-                                                   c2, f32x2_pack(-l.z, -l.w));
+                                                   c2, f32x2_pack(l.z, l.w));
                         float x0, x1, x2, x3;
                         f32x2_unpack(x01, x0, x1);
                         f32x2_unpack(x23, x2, x3);
@@ -363,9 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const int c = 8 * q + 4 * e;      // column within the half
                                 const int cr = 8 * qq + 4 * e;    // column within this dP chunk
                                 const uint64_t a01 = fadd2(f32x2_pack(__uint_as_float(dr[cr]), __uint_as_float(dr[cr + 1])),
-                                                           f32x2_pack(-d.x, -d.y));
+                                                           f32x2_pack(d.x, d.y));
                                 const uint64_t a23 = fadd2(f32x2_pack(__uint_as_float(dr[cr + 2]), __uint_as_float(dr[cr + 3])),
-                                                           f32x2_pack(-d.z, -d.w));
+                                                           f32x2_pack(d.z, d.w));
                                 const uint64_t s01 = fmul2(a01, f32x2_pack(pf[c], pf[c + 1]));
                                 const uint64_t s23 = fmul2(a23, f32x2_pack(pf[c + 2], pf[c + 3]));
                                 float s0, s1, s2, s3;

@@ -277,8 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
                     const int c = 32 * ch + e;
-                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, -lse_i[c]));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), scale_log2, -lse_i[c + 1]));
+                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, lse_i[c]));
+                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), scale_log2, lse_i[c + 1]));
                     if (it == 0) {  // diagonal tile: query c sees key row only if row <= c
                         if (c < row) p0 = 0.f;
                         if (c + 1 < row) p1 = 0.f;
@@ -305,8 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; e += 2) {
                     const int c = 32 * ch + e;
                     const uint32_t pp = pk[c >> 1];
-                    const float ds0 = bf16lo_to_f32(pp) * (__uint_as_float(dr[e]) - D_i[c]);
-                    const float ds1 = bf16hi_to_f32(pp) * (__uint_as_float(dr[e + 1]) - D_i[c + 1]);
+                    const float ds0 = bf16lo_to_f32(pp) * (__uint_as_float(dr[e]) + D_i[c]);
+                    const float ds1 = bf16hi_to_f32(pp) * (__uint_as_float(dr[e + 1]) + D_i[c + 1]);
                     w[e >> 1] = pack_bf16x2(ds0, ds1);
                 }
                 // dS^T row `row`, query columns [32ch, 32ch+32): slab ch/2, 16-byte chunks 4*(ch&1)..+3
@@ -420,9 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// preprocess: D = rowsum(dy o y) per (b, h, t); lse2 = lse * log2(e); rows
-// t >= T of each (b, h) get D = 0 and lse2 = +inf (so recomputed P is 0);
-// dQ accumulator zeroed.
+// preprocess: per (b, h, t) store -D = -rowsum(dy o y) and -lse * log2(e)
+// (negated so the main kernels add them); rows t >= T of each (b, h) get
+// 0 and -inf (so the recomputed P there is 0); dQ accumulator zeroed.
 // ---------------------------------------------------------------------------
 template <int HS>
 __global__ void bwd_pre_kernel(const __nv_bfloat16 *__restrict__ y, const __nv_bfloat16 *__restrict__ dy,
@@ -436,7 +436,7 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16 *__restrict__ y, const __nv_b
         const long long bh = idx / T_pad;
         const int h = (int)(bh % n_head);
         const long long b = bh / n_head;
-        float d = 0.f, l2 = INFINITY;
+        float d = 0.f, l2 = INFINITY;  // stored negated below: -D and -lse*log2(e)
         if (t < T) {
             const size_t off = ((size_t)b * T + t) * (size_t)C + (size_t)h * HS;
             const uint4 *yv = reinterpret_cast<const uint4 *>(y + off);
@@ -453,8 +453,8 @@ __global__ void bwd_pre_kernel(const __nv_bfloat16 *__restrict__ y, const __nv_b
             }
             l2 = lse[bh * T + t] * 1.4426950408889634f;
         }
-        D[idx] = d;
-        lse2[idx] = l2;
+        D[idx] = -d;
+        lse2[idx] = -l2;
     }
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
     for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < zero4; idx += stride) dqacc[idx] = z;

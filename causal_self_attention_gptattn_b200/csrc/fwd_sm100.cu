@@ -1,29 +1,40 @@
-// fwd_sm100.cu -- bf16 causal self-attention forward for sm_100a.
+// fwd_sm100.cu -- persistent bf16 causal self-attention forward for sm_100a.
 //
-// Computes, per (batch b, head h) and 128-row query tile i (lecture page
+// Computes, for every (batch b, head h) and 128-row query tile (lecture page
 // "Let's build GPT: from scratch, in code, spelled out", chapters "version 3:
 // adding softmax" and "version 4: self-attention"; note 6 / correction 01:20:05
 // for the 1/sqrt(head_size) scale; correction 00:57:00 for the causal mask):
-//     S_j = Q_i K_j^T                 (tcgen05 MMA, fp32 accumulators in TMEM)
+//     S_j = Q K_j^T                   (tcgen05 MMA, fp32 accumulators in TMEM)
 //     online softmax of S_j * scale   (fp32, one TMEM lane = one query row per thread)
 //     O  += P_j V_j                   (tcgen05 MMA, P read straight from TMEM)
-// for key tiles j = 0..i only (tiles above the diagonal are skipped, the
-// diagonal tile is masked element-wise), then y = O / l and lse = m + ln l.
+// over the key tiles j at or below the diagonal (tiles above it are skipped,
+// the diagonal tile is masked element-wise), then y = O / l and lse = m + ln l.
 //
-// One CTA per (query tile, b, h), six warps with fixed roles:
-//   warp 0      TMA producer: Q once, then K_j / V_j through a smem ring
+// Work item = a pair of consecutive query tiles (A = 2m, B = 2m+1) of one
+// (b, h); both share the K_j / V_j tiles.  One persistent CTA per SM walks
+// the items longest first, in a snake order over the CTAs.  Ten warps:
+//   warp 0      TMA producer: Q_A, Q_B per item, K_j / V_j through a ring
 //   warp 1      TMEM owner + MMA issuer (one elected lane)
-//   warps 2..5  softmax, O rescale and epilogue (128 threads = 128 query rows)
-// TMEM (512 columns): S double buffer at [0,128) and [128,256), O at [256,256+hs).
-// Every barrier wait is bounded (see sm100_ptx.cuh); a timeout sets the CTA's
-// abort flag and the device status word, and all roles drain and exit.
+//   warps 2..5  softmax, O rescale and epilogue of tile A (one query row per thread)
+//   warps 6..9  the same for tile B
+// The two softmax warpgroups ping-pong: the MMA order
+//     S_A0 S_B0 | PV_A0 S_A1 | PV_B0 S_B1 | PV_A1 S_A2 | ...
+// lets one tile's exponentials run while the other tile's P V and next S run.
+// TMEM (512 columns): S_A [0,128), S_B [128,256) (P written back over the
+// first 64 columns of its S), O_A [256, 256+hs), O_B [256+hs, 256+2hs).
+// The softmax keeps the running max lazily (rescaling O only when the max
+// grows by more than 2^8) and normalises y by the sum of the bf16-rounded
+// weights that the P V product used; lse uses the sum of the fp32 weights.
+// Every barrier wait is bounded (sm100_ptx.cuh); on a timeout all roles stop
+// issuing work, drain and exit.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
+
 
 namespace gptattn {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlabBytes = 128 * 128;  // 128 rows x 128 bytes (64 bf16 columns), one swizzle slab
 
@@ -31,23 +42,27 @@ template <int HS>
 struct FwdCfg {
     static constexpr int kSlabs = HS / 64;
     static constexpr uint32_t kTileBytes = 128u * HS * 2u;
-    static constexpr int kStages = (HS == 64) ? 3 : 2;
-    static constexpr uint32_t kOffQ = 0;
-    static constexpr uint32_t kOffK = kOffQ + kTileBytes;
-    static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
-    static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-    static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + slack for 1024-byte alignment
-    static constexpr uint32_t kColS = 0;    // S buffers at kColS + 128 * (j & 1)
-    static constexpr uint32_t kColO = 256;
+    static constexpr int kQStages = (HS == 64) ? 2 : 1;   // pairs of Q tiles
+    static constexpr int kKVStages = (HS == 64) ? 4 : 2;
+    static constexpr uint32_t kOffQ = 0;                                      // kQStages x 2 tiles
+    static constexpr uint32_t kOffK = kOffQ + kQStages * 2 * kTileBytes;     // kKVStages tiles
+    static constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;        // kKVStages tiles
+    static constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
+    static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;             // + slack for 1024-byte alignment
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static constexpr uint32_t kColS = 0;    // + 128 * tile
+    static constexpr uint32_t kColO = 256;  // + HS * tile
     // barrier slots (8 bytes each)
-    static constexpr int kBarQ = 0;
-    static constexpr int kBarK = 1;
-    static constexpr int kBarV = kBarK + kStages;
-    static constexpr int kBarE = kBarV + kStages;
-    static constexpr int kBarS = kBarE + kStages;  // two
-    static constexpr int kBarP = kBarS + 2;
-    static constexpr int kBarO = kBarP + 1;
-    static constexpr int kBarDone = kBarO + 1;
+    static constexpr int kBarQFull = 0;
+    static constexpr int kBarQEmpty = kBarQFull + kQStages;
+    static constexpr int kBarKFull = kBarQEmpty + kQStages;
+    static constexpr int kBarVFull = kBarKFull + kKVStages;
+    static constexpr int kBarKVEmpty = kBarVFull + kKVStages;
+    static constexpr int kBarSFull = kBarKVEmpty + kKVStages;  // 2 (per tile)
+    static constexpr int kBarPFull = kBarSFull + 2;            // 2
+    static constexpr int kBarODone = kBarPFull + 2;            // 2
+    static constexpr int kBarOFree = kBarODone + 2;            // 2
+    static constexpr int kBarDone = kBarOFree + 2;
     static constexpr int kNumBars = kBarDone + 1;
     static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
 };
@@ -66,6 +81,11 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
+// Item k of this CTA in the snake walk over items sorted longest first.
+__device__ __forceinline__ int item_index(int k, int cta, int grid) {
+    return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
+}
+
 template <int HS>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
@@ -80,11 +100,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int BH = B * n_head;
-    const int bh = blockIdx.x % BH;
-    const int qt = n_qt - 1 - blockIdx.x / BH;  // longest rows first
-    const int b = bh / n_head;
-    const int h = bh % n_head;
-    const int nkv = qt + 1;                     // causal: key tiles 0..qt
+    const int n_pairs = (n_qt + 1) >> 1;
+    const int n_items = n_pairs * BH;
+    const int grid = gridDim.x, cta = blockIdx.x;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K::kOffBar);
     auto bar = [&](int idx) -> uint32_t { return smem_u32(&bars[idx]); };
@@ -92,21 +110,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + K::kOffBar + K::kNumBars * 8 + 4);
     const WaitGuard g{abort_flag, status, budget_ns};
 
-    const uint32_t sQ = sbase + K::kOffQ;
-    auto sK = [&](int st) -> uint32_t { return sbase + K::kOffK + st * K::kTileBytes; };
-    auto sV = [&](int st) -> uint32_t { return sbase + K::kOffV + st * K::kTileBytes; };
+    auto sQ = [&](int qs, int t) -> uint32_t { return sbase + K::kOffQ + (uint32_t)(2 * qs + t) * K::kTileBytes; };
+    auto sK = [&](int st) -> uint32_t { return sbase + K::kOffK + (uint32_t)st * K::kTileBytes; };
+    auto sV = [&](int st) -> uint32_t { return sbase + K::kOffV + (uint32_t)st * K::kTileBytes; };
+
+    // item -> (pair m, batch*head); pairs with the most key tiles first
+    auto decode = [&](int w, int &m, int &bh) {
+        m = n_pairs - 1 - w / BH;
+        bh = w % BH;
+    };
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(K::kBarQ), 1);
-        for (int s = 0; s < K::kStages; ++s) {
-            mbar_init(bar(K::kBarK + s), 1);
-            mbar_init(bar(K::kBarV + s), 1);
-            mbar_init(bar(K::kBarE + s), 1);
+        for (int s = 0; s < K::kQStages; ++s) {
+            mbar_init(bar(K::kBarQFull + s), 1);
+            mbar_init(bar(K::kBarQEmpty + s), 2);  // one arrival per softmax warpgroup
         }
-        mbar_init(bar(K::kBarS + 0), 1);
-        mbar_init(bar(K::kBarS + 1), 1);
-        mbar_init(bar(K::kBarP), 128);
-        mbar_init(bar(K::kBarO), 1);
+        for (int s = 0; s < K::kKVStages; ++s) {
+            mbar_init(bar(K::kBarKFull + s), 1);
+            mbar_init(bar(K::kBarVFull + s), 1);
+            mbar_init(bar(K::kBarKVEmpty + s), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(K::kBarSFull + t), 1);
+            mbar_init(bar(K::kBarPFull + t), 128);
+            mbar_init(bar(K::kBarODone + t), 1);
+            mbar_init(bar(K::kBarOFree + t), 128);
+        }
         mbar_init(bar(K::kBarDone), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -121,85 +150,129 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ================================================================ producer
         if (lane == 0) {
             tma_prefetch_map(&map_qkv);
             tma_prefetch_map(&map_y);
-            const int col_q = h * HS, col_k = C + h * HS, col_v = 2 * C + h * HS;
-            mbar_arrive_expect_tx(bar(K::kBarQ), K::kTileBytes);
-            for (int s = 0; s < K::kSlabs; ++s)
-                tma_load_3d(sQ + s * kSlabBytes, &map_qkv, bar(K::kBarQ), col_q + 64 * s, qt * kTile, b);
-            int issued = 0;
             bool ok = true;
-            for (int j = 0; j < nkv; ++j) {
-                const int st = j % K::kStages;
-                const uint32_t ph = (uint32_t)(j / K::kStages) & 1u;
-                if (j >= K::kStages && !mbar_wait(bar(K::kBarE + st), ph ^ 1u, g)) {
-                    ok = false;
+            int nq = 0, gkv = 0;  // Q stages and K/V stages filled so far
+            for (int k = 0; ok; ++k) {
+                const int w = item_index(k, cta, grid);
+                if (w >= n_items) break;
+                int m, bh;
+                decode(w, m, bh);
+                const int b = bh / n_head, h = bh % n_head;
+                const bool hasB = 2 * m + 1 < n_qt;
+                const int nkv = hasB ? 2 * m + 2 : 2 * m + 1;
+                const int qs = nq % K::kQStages;
+                if (nq >= K::kQStages &&
+                    !(ok = mbar_wait(bar(K::kBarQEmpty + qs), (uint32_t)((nq / K::kQStages) & 1) ^ 1u, g)))
                     break;
+                const uint32_t qb = bar(K::kBarQFull + qs);
+                mbar_arrive_expect_tx(qb, (hasB ? 2u : 1u) * K::kTileBytes);
+                for (int t = 0; t < (hasB ? 2 : 1); ++t)
+                    for (int s = 0; s < K::kSlabs; ++s)
+                        tma_load_3d(sQ(qs, t) + s * kSlabBytes, &map_qkv, qb, h * HS + 64 * s, (2 * m + t) * kTile, b);
+                ++nq;
+                for (int j = 0; j < nkv; ++j) {
+                    const int st = gkv % K::kKVStages;
+                    const uint32_t ph = (uint32_t)(gkv / K::kKVStages) & 1u;
+                    if (gkv >= K::kKVStages && !(ok = mbar_wait(bar(K::kBarKVEmpty + st), ph ^ 1u, g))) break;
+                    mbar_arrive_expect_tx(bar(K::kBarKFull + st), K::kTileBytes);
+                    for (int s = 0; s < K::kSlabs; ++s)
+                        tma_load_3d(sK(st) + s * kSlabBytes, &map_qkv, bar(K::kBarKFull + st), C + h * HS + 64 * s,
+                                    j * kTile, b);
+                    mbar_arrive_expect_tx(bar(K::kBarVFull + st), K::kTileBytes);
+                    for (int s = 0; s < K::kSlabs; ++s)
+                        tma_load_3d(sV(st) + s * kSlabBytes, &map_qkv, bar(K::kBarVFull + st), 2 * C + h * HS + 64 * s,
+                                    j * kTile, b);
+                    ++gkv;
                 }
-                mbar_arrive_expect_tx(bar(K::kBarK + st), K::kTileBytes);
-                for (int s = 0; s < K::kSlabs; ++s)
-                    tma_load_3d(sK(st) + s * kSlabBytes, &map_qkv, bar(K::kBarK + st), col_k + 64 * s, j * kTile, b);
-                mbar_arrive_expect_tx(bar(K::kBarV + st), K::kTileBytes);
-                for (int s = 0; s < K::kSlabs; ++s)
-                    tma_load_3d(sV(st) + s * kSlabBytes, &map_qkv, bar(K::kBarV + st), col_v + 64 * s, j * kTile, b);
-                issued = j + 1;
             }
             if (!ok || *abort_flag) {
-                // let this CTA's own copies land before shared memory is released
-                drain_wait(bar(K::kBarQ), 0, budget_ns);
-                for (int j = (issued > K::kStages ? issued - K::kStages : 0); j < issued; ++j) {
-                    const uint32_t ph = (uint32_t)(j / K::kStages) & 1u;
-                    drain_wait(bar(K::kBarK + j % K::kStages), ph, budget_ns);
-                    drain_wait(bar(K::kBarV + j % K::kStages), ph, budget_ns);
+                // let this CTA's last copies land before shared memory is released
+                for (int q = (nq > K::kQStages ? nq - K::kQStages : 0); q < nq; ++q)
+                    drain_wait(bar(K::kBarQFull + q % K::kQStages), (uint32_t)(q / K::kQStages) & 1u, budget_ns);
+                for (int q = (gkv > K::kKVStages ? gkv - K::kKVStages : 0); q < gkv; ++q) {
+                    drain_wait(bar(K::kBarKFull + q % K::kKVStages), (uint32_t)(q / K::kKVStages) & 1u, budget_ns);
+                    drain_wait(bar(K::kBarVFull + q % K::kKVStages), (uint32_t)(q / K::kKVStages) & 1u, budget_ns);
                 }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ================================================================ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // Q, K both K-major
             constexpr uint32_t idPV = idesc_bf16_f32(128, HS, false, true);   // P from TMEM, V N-major
-            bool ok = mbar_wait(bar(K::kBarQ), 0, g);
-            bool any = false;
-            auto issue_s = [&](int j) -> bool {
-                const int st = j % K::kStages;
-                const uint32_t ph = (uint32_t)(j / K::kStages) & 1u;
-                if (!mbar_wait(bar(K::kBarK + st), ph, g)) return false;
-                tc_fence_after();
-                const uint32_t d = tmem + K::kColS + 128u * (uint32_t)(j & 1);
+            const uint64_t dQ0 = sdesc_sw128(sQ(0, 0), 16, 1024);
+            const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
+            const uint64_t dV0 = sdesc_sw128(sV(0), kSlabBytes, 1024);
+            auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+            bool ok = true, any = false;
+            int n = 0, gkv = 0;
+            int it[2] = {0, 0};     // S / P V iterations issued per tile stream
+            int items[2] = {0, 0};  // items that used each tile stream
+            auto issue_S = [&](int qs, int t, int st) {
+                const uint64_t a = at(dQ0, (uint32_t)(2 * qs + t) * K::kTileBytes);
+                const uint64_t bk = at(dK0, (uint32_t)st * K::kTileBytes);
 #pragma unroll
                 for (int kk = 0; kk < HS / 16; ++kk) {
                     const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
-                    umma_ss(d, sdesc_sw128(sQ + koff, 16, 1024), sdesc_sw128(sK(st) + koff, 16, 1024), idS,
-                            kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + K::kColS + 128u * t, at(a, koff), at(bk, koff), idS, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(bar(K::kBarS + (j & 1)));
-                any = true;
-                return true;
+                umma_commit(bar(K::kBarSFull + t));
             };
-            auto issue_pv = [&](int j) -> bool {
-                const int st = j % K::kStages;
-                const uint32_t ph = (uint32_t)(j / K::kStages) & 1u;
-                if (!mbar_wait(bar(K::kBarP), (uint32_t)j & 1u, g)) return false;
-                if (!mbar_wait(bar(K::kBarV + st), ph, g)) return false;
-                tc_fence_after();
-                const uint32_t p = tmem + K::kColS + 128u * (uint32_t)(j & 1);
+            auto issue_PV = [&](int t, int st, bool first) {
+                const uint64_t bv = at(dV0, (uint32_t)st * K::kTileBytes);
+                const uint32_t p = tmem + K::kColS + 128u * t;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    umma_ts(tmem + K::kColO, p + 8u * kk, sdesc_sw128(sV(st) + kk * 2048u, kSlabBytes, 1024), idPV,
-                            (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(bar(K::kBarE + st));
-                umma_commit(bar(K::kBarO));
-                return true;
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + K::kColO + HS * t, p + 8u * kk, at(bv, kk * 2048u), idPV,
+                            (!first || kk > 0) ? 1u : 0u);
+                umma_commit(bar(K::kBarODone + t));
             };
-            for (int j = 0; j < nkv && ok; ++j) {
-                ok = issue_s(j);
-                if (ok && j > 0) ok = issue_pv(j - 1);
+            for (int k = 0; ok; ++k, ++n) {
+                const int w = item_index(k, cta, grid);
+                if (w >= n_items) break;
+                int m, bh;
+                decode(w, m, bh);
+                const bool hasB = 2 * m + 1 < n_qt;
+                const int nt[2] = {2 * m + 1, hasB ? 2 * m + 2 : 0};  // key tiles per tile stream
+                const int nkv = hasB ? nt[1] : nt[0];
+                const int qs = n % K::kQStages;
+                if (!(ok = mbar_wait(bar(K::kBarQFull + qs), (uint32_t)(n / K::kQStages) & 1u, g))) break;
+                if (!(ok = mbar_wait(bar(K::kBarKFull + gkv % K::kKVStages), (uint32_t)(gkv / K::kKVStages) & 1u, g)))
+                    break;
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t)
+                    if (nt[t] > 0) issue_S(qs, t, gkv % K::kKVStages);
+                any = true;
+                for (int j = 0; j < nkv && ok; ++j) {
+                    const int st = (gkv + j) % K::kKVStages;
+                    const int st1 = (gkv + j + 1) % K::kKVStages;
+                    const uint32_t ph1 = (uint32_t)((gkv + j + 1) / K::kKVStages) & 1u;
+                    if (!(ok = mbar_wait(bar(K::kBarVFull + st), (uint32_t)((gkv + j) / K::kKVStages) & 1u, g))) break;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= nt[t]) continue;
+                        if (!(ok = mbar_wait(bar(K::kBarPFull + t), (uint32_t)it[t] & 1u, g))) break;
+                        if (j == 0 && items[t] > 0 &&
+                            !(ok = mbar_wait(bar(K::kBarOFree + t), (uint32_t)(items[t] - 1) & 1u, g)))
+                            break;
+                        tc_fence_after();
+                        issue_PV(t, st, j == 0);
+                        ++it[t];
+                        if (j + 1 < nt[t]) {
+                            if (!(ok = mbar_wait(bar(K::kBarKFull + st1), ph1, g))) break;
+                            tc_fence_after();
+                            issue_S(qs, t, st1);
+                        }
+                    }
+                    if (ok) umma_commit(bar(K::kBarKVEmpty + st));
+                }
+                gkv += nkv;
+                items[0] += 1;
+                items[1] += hasB ? 1 : 0;
             }
-            if (ok) ok = issue_pv(nkv - 1);
             if (any) {
                 // all MMAs of this CTA retired before TMEM can be released
                 umma_commit(bar(K::kBarDone));
@@ -207,121 +280,155 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax warps
+        // ================================================================ softmax warpgroups
+        const int t = (warp - 2) >> 2;           // tile stream: 0 = A, 1 = B
         const int sp = warp & 3;                 // TMEM sub-partition this warp may access
         const int row = sp * 32 + lane;          // query row within the tile
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
-        const float scale_log2 = rsqrtf((float)HS) * 1.4426950408889634f;
-        float m = -INFINITY;  // running max of scaled scores (log2 units)
-        float l = 0.f;        // running normaliser (fp32 weights)
-        float l_r = 0.f;      // running normaliser (bf16-rounded weights)
+        const uint32_t tS = trow + K::kColS + 128u * t;
+        const uint32_t tO = trow + K::kColO + (uint32_t)HS * t;
+        const float scale_log2 = (HS == 64 ? 0.125f : 0.08838834764831845f) * 1.4426950408889634f;
+        const uint64_t c2 = f32x2_pack(scale_log2, scale_log2);
+        const bool leader = (sp == 0 && lane == 0);  // one thread of this warpgroup
         bool ok = true;
-        for (int j = 0; j < nkv; ++j) {
-            ok = warp_wait(bar(K::kBarS + (j & 1)), (uint32_t)(j >> 1) & 1u, g);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t tS = trow + K::kColS + 128u * (uint32_t)(j & 1);
-            uint32_t sr[128];
-            tmem_ld_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_ld_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-            tmem_ld_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-            float *s = reinterpret_cast<float *>(sr);
-            if (j == qt) {
-#pragma unroll
-                for (int c = 0; c < 128; ++c)
-                    if (c > row) s[c] = -INFINITY;
+        int it = 0, n = 0;
+        for (int k = 0;; ++k, ++n) {
+            const int w = item_index(k, cta, grid);
+            if (w >= n_items) break;
+            int m, bh;
+            decode(w, m, bh);
+            const int b = bh / n_head, h = bh % n_head;
+            const int qt = 2 * m + t;
+            const int qs = n % K::kQStages;
+            if (qt >= n_qt) {
+                // this tile stream has no work in this item; release its share of the Q stage
+                if (leader) mbar_arrive(bar(K::kBarQEmpty + qs));
+                continue;
             }
-            // row max with 8 independent partial maxima (no 128-long dependency chain)
-            float mp[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mp[k] = s[k];
-#pragma unroll
-            for (int c = 8; c < 128; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                   fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-            // Lazy rescaling: keep the running max unless it grows by more than
-            // 8 (log2 units).  p stays <= 2^8 and l, O use the same stale max,
-            // so y = O / l and lse = m + log2 l are exact; O is rescaled rarely.
-            const float m_cand = mx * scale_log2;
-            const bool grow = m_cand > m + 8.f;
-            const float m_new = grow ? m_cand : m;
-            const float alpha = grow ? ex2_approx(m - m_new) : 1.f;
-            const float neg = -m_new;
-            // Two row sums: of the fp32 weights (for lse) and of the bf16-rounded
-            // weights the P V product actually uses (to normalise y, so that a
-            // row dominated by one key returns that key's value exactly).
-            float sp8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            float sr8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[64];
-#pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                const float p0 = ex2_approx(fmaf(s[c], scale_log2, neg));
-                const float p1 = ex2_approx(fmaf(s[c + 1], scale_log2, neg));
-                sp8[(c >> 1) & 7] += p0 + p1;
-                const uint32_t w = pack_bf16x2(p0, p1);
-                sr8[(c >> 1) & 7] += bf16lo_to_f32(w) + bf16hi_to_f32(w);
-                pk[c >> 1] = w;
-            }
-            const float sum = ((sp8[0] + sp8[1]) + (sp8[2] + sp8[3])) + ((sp8[4] + sp8[5]) + (sp8[6] + sp8[7]));
-            const float sum_r = ((sr8[0] + sr8[1]) + (sr8[2] + sr8[3])) + ((sr8[4] + sr8[5]) + (sr8[6] + sr8[7]));
-            tmem_st_x32(tS + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
-            tmem_st_x32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-            l = l * alpha + sum;
-            l_r = l_r * alpha + sum_r;
-            m = m_new;
-            if (j > 0) {
-                // rescale O once the previous P V product has landed
-                ok = warp_wait(bar(K::kBarO), (uint32_t)(j - 1) & 1u, g);
-                if (!ok) break;
+            const int ntile = qt + 1;
+            float mrow = -INFINITY;  // reference max of scaled scores (log2 units), lazily updated
+            float l = 0.f;           // running normaliser of the fp32 weights
+            float l_r = 0.f;         // running normaliser of the bf16-rounded weights
+            for (int j = 0; j < ntile; ++j, ++it) {
+                if (ok) ok = warp_wait(bar(K::kBarSFull + t), (uint32_t)it & 1u, g);
+                if (!ok) continue;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                const bool diag = (j == qt);
+                // pass 1: row maximum
+                float mx = -INFINITY;
 #pragma unroll
-                    for (int c0 = 0; c0 < HS; c0 += 32) {
-                        uint32_t o[32];
-                        tmem_ld_x32(trow + K::kColO + c0, o);
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t sr[32];
+                    tmem_ld_x32(tS + 32 * ch, sr);
+                    if (diag) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                        tmem_st_x32(trow + K::kColO + c0, o);
+                        for (int c = 0; c < 32; ++c)
+                            if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
+                    }
+                    float a = __uint_as_float(sr[0]), bb = __uint_as_float(sr[1]);
+#pragma unroll
+                    for (int c = 2; c < 32; c += 2) a = fmax3(a, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                    mx = fmax3(mx, a, bb);
+                }
+                // lazy max: keep the reference unless it grows by more than 8 (log2 units)
+                const float m_cand = mx * scale_log2;
+                const bool grow = m_cand > mrow + 8.f;
+                const float m_new = grow ? m_cand : mrow;
+                const float alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
+                const uint64_t negm2 = f32x2_pack(-m_new, -m_new);
+                // pass 2: weights, sums, P back into TMEM (bf16 pairs over columns already read)
+                uint64_t sum2 = f32x2_pack(0.f, 0.f), sumr2 = f32x2_pack(0.f, 0.f);
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t sr[32];
+                    tmem_ld_x32(tS + 32 * ch, sr);
+                    if (diag) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
+                    }
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
+                        float x0, x1;
+                        f32x2_unpack(x, x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        const uint32_t wv = pack_bf16x2(p0, p1);
+                        pk[c >> 1] = wv;
+                        sum2 = fadd2(sum2, f32x2_pack(p0, p1));
+                        sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                    }
+                    tmem_st_x16(tS + 16 * ch, pk);
+                }
+                float s0, s1, r0, r1;
+                f32x2_unpack(sum2, s0, s1);
+                f32x2_unpack(sumr2, r0, r1);
+                l = l * alpha + (s0 + s1);
+                l_r = l_r * alpha + (r0 + r1);
+                mrow = m_new;
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // rescale O once the previous P V product of this tile has landed
+                    ok = warp_wait(bar(K::kBarODone + t), (uint32_t)(it - 1) & 1u, g);
+                    if (ok) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int c0 = 0; c0 < HS; c0 += 32) {
+                            uint32_t o[32];
+                            tmem_ld_x32(tO + c0, o);
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                            tmem_st_x32(tO + c0, o);
+                        }
                     }
                 }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar(K::kBarPFull + t));
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(bar(K::kBarP));
-        }
-        // -------------------------------------------------------- epilogue
-        if (ok) ok = warp_wait(bar(K::kBarO), (uint32_t)(nkv - 1) & 1u, g);
-        if (ok) {
-            tc_fence_after();
-            const float inv_l = 1.f / l_r;
+            // ------------------------------------------------------------ epilogue of this tile
+            // staging: this tile's Q buffer (its last S MMA retired before the last P V)
+            const uint32_t stg = sQ(qs, t);
+            if (ok) ok = warp_wait(bar(K::kBarODone + t), (uint32_t)(it - 1) & 1u, g);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = 1.f / l_r;
 #pragma unroll
-            for (int c0 = 0; c0 < HS; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld_x32(trow + K::kColO + c0, o);
-                uint32_t w[16];
+                for (int c0 = 0; c0 < HS; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld_x32(tO + c0, o);
+                    if (c0 + 32 == HS) {
+                        tc_fence_before();
+                        mbar_arrive(bar(K::kBarOFree + t));  // O may be overwritten by the next item
+                    }
+                    uint32_t wv[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
-                // staging tile in the Q buffer (Q is dead once the last S MMA retired)
-                const uint32_t slab = sQ + (uint32_t)(c0 >> 6) * kSlabBytes + (uint32_t)row * 128u;
+                    for (int c = 0; c < 16; ++c)
+                        wv[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
+                    const uint32_t slab = stg + (uint32_t)(c0 >> 6) * kSlabBytes + (uint32_t)row * 128u;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t chunk = (uint32_t)(((c0 & 63) >> 3) + q);
-                    st_shared_v4(slab + ((chunk ^ (uint32_t)(row & 7)) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2],
-                                 w[4 * q + 3]);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t chunk = (uint32_t)(((c0 & 63) >> 3) + q);
+                        st_shared_v4(slab + ((chunk ^ (uint32_t)(row & 7)) << 4), wv[4 * q], wv[4 * q + 1],
+                                     wv[4 * q + 2], wv[4 * q + 3]);
+                    }
                 }
+                fence_proxy_async_smem();
+                const int tq = qt * kTile + row;
+                if (tq < T) lse[(size_t)bh * (size_t)T + (size_t)tq] = (mrow + __log2f(l)) * 0.6931471805599453f;
             }
-            fence_proxy_async_smem();
-            const int t = qt * kTile + row;
-            if (t < T) lse[(size_t)bh * (size_t)T + (size_t)t] = (m + __log2f(l)) * 0.6931471805599453f;
+            named_bar_sync(1 + t, 128);
+            if (leader) {
+                if (ok && !*abort_flag) {
+                    for (int s = 0; s < K::kSlabs; ++s)
+                        tma_store_3d(&map_y, stg + s * kSlabBytes, h * HS + 64 * s, qt * kTile, b);
+                    bulk_commit_group();
+                    bulk_wait_group_read_0();  // staging (this Q buffer) may now be refilled
+                }
+                mbar_arrive(bar(K::kBarQEmpty + qs));
+            }
         }
-        named_bar_sync(1, 128);
-        if (warp == 2 && lane == 0 && !*abort_flag) {
-            for (int s = 0; s < K::kSlabs; ++s) tma_store_3d(&map_y, sQ + s * kSlabBytes, h * HS + 64 * s, qt * kTile, b);
-            bulk_commit_group();
-            bulk_wait_group_0();
-        }
+        if (leader) bulk_wait_group_0();
     }
 
     tc_fence_before();
@@ -339,9 +446,14 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
     cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     const int n_qt = ceil_div(T, kTile);
-    const long long blocks = (long long)n_qt * B * n_head;
-    fwd_bf16_kernel<HS><<<dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s>>>(
+    const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
+    const int grid = (int)(items < sms ? items : sms);
+    fwd_bf16_kernel<HS><<<dim3((unsigned)grid), dim3(kThreads), K::kSmemBytes, s>>>(
         map_qkv, map_y, lse, B, T, C, n_head, n_qt, ctx.status, ctx.budget_ns);
     return cudaGetLastError();
 }
