@@ -1,0 +1,427 @@
+// fwd_h64_sm100.cu -- persistent bf16 causal self-attention forward, head size 64.
+//
+// Same function as fwd_sm100.cu (lecture page "Let's build GPT: from scratch,
+// in code, spelled out", chapters "version 3: adding softmax" and "version 4:
+// self-attention"; note 6 / correction 01:20:05 for the 1/sqrt(head_size)
+// scale; correction 00:57:00 for the causal mask), organised for head size 64,
+// where all six TMEM buffers fit at once:
+//   TMEM (512 columns): S_A [0,128)  S_B [128,256)  P_A [256,320)  P_B [320,384)
+//                       O_A [384,448)  O_B [448,512)
+// Work item = query tiles A = 2m and B = 2m+1 of one (batch, head), sharing the
+// key/value tiles; one persistent CTA per SM walks the items longest first in
+// a snake order.  Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5
+// softmax of tile A, 6..9 softmax of tile B (one query row per thread).
+// Because P has its own buffer, a softmax warpgroup copies S_j to registers
+// in one pass and releases it immediately; the MMA warp then computes S_{j+1}
+// while the warpgroup exponentiates tile j, and P V of tile j runs while the
+// warpgroup starts tile j+1.  MMA order per key tile j:
+//     S_A(j+1)  S_B(j+1)  PV_A(j)  PV_B(j)
+// Lazy rescaling (O is rescaled only when a row max grows by more than 2^8)
+// and y normalised by the sum of the bf16-rounded weights, as in fwd_sm100.cu.
+// Every barrier wait is bounded; on a timeout all roles stop, drain and exit.
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace gptattn {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSlabBytes = 128 * 128;
+constexpr int HS = 64;
+constexpr uint32_t kTileBytes = 128u * 64u * 2u;
+constexpr int kQStages = 2;   // pairs of Q tiles
+constexpr int kKVStages = 4;
+constexpr uint32_t kOffQ = 0;                                   // kQStages x 2 tiles
+constexpr uint32_t kOffK = kOffQ + kQStages * 2 * kTileBytes;    // kKVStages tiles
+constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;       // kKVStages tiles
+constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // + 128 t, + 64 t, + 64 t
+
+constexpr int kBarQFull = 0;
+constexpr int kBarQEmpty = kBarQFull + kQStages;
+constexpr int kBarKFull = kBarQEmpty + kQStages;
+constexpr int kBarVFull = kBarKFull + kKVStages;
+constexpr int kBarKVEmpty = kBarVFull + kKVStages;
+constexpr int kBarSFull = kBarKVEmpty + kKVStages;  // 2
+constexpr int kBarSEmpty = kBarSFull + 2;           // 2
+constexpr int kBarPFull = kBarSEmpty + 2;           // 2
+constexpr int kBarPVDone = kBarPFull + 2;           // 2
+constexpr int kBarOFree = kBarPVDone + 2;           // 2
+constexpr int kBarDone = kBarOFree + 2;
+constexpr int kNumBars = kBarDone + 1;
+static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitGuard &g) {
+    bool ok = mbar_wait(bar, parity, g);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > budget_ns) break;
+    }
+}
+
+__device__ __forceinline__ int item_index(int k, int cta, int grid) {
+    return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_h64_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
+                   float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int *status,
+                   unsigned long long budget_ns) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int BH = B * n_head;
+    const int n_pairs = (n_qt + 1) >> 1;
+    const int n_items = n_pairs * BH;
+    const int grid = gridDim.x, cta = blockIdx.x;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    auto bar = [&](int idx) -> uint32_t { return smem_u32(&bars[idx]); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffBar + kNumBars * 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + kNumBars * 8 + 4);
+    const WaitGuard g{abort_flag, status, budget_ns};
+
+    auto sQ = [&](int qs, int t) -> uint32_t { return sbase + kOffQ + (uint32_t)(2 * qs + t) * kTileBytes; };
+    auto sK = [&](int st) -> uint32_t { return sbase + kOffK + (uint32_t)st * kTileBytes; };
+    auto sV = [&](int st) -> uint32_t { return sbase + kOffV + (uint32_t)st * kTileBytes; };
+    auto decode = [&](int w, int &m, int &bh) {
+        m = n_pairs - 1 - w / BH;
+        bh = w % BH;
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(bar(kBarQFull + s), 1);
+            mbar_init(bar(kBarQEmpty + s), 2);
+        }
+        for (int s = 0; s < kKVStages; ++s) {
+            mbar_init(bar(kBarKFull + s), 1);
+            mbar_init(bar(kBarVFull + s), 1);
+            mbar_init(bar(kBarKVEmpty + s), 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(kBarSFull + t), 1);
+            mbar_init(bar(kBarSEmpty + t), 128);
+            mbar_init(bar(kBarPFull + t), 128);
+            mbar_init(bar(kBarPVDone + t), 1);
+            mbar_init(bar(kBarOFree + t), 128);
+        }
+        mbar_init(bar(kBarDone), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ================================================================ producer
+        if (lane == 0) {
+            tma_prefetch_map(&map_qkv);
+            tma_prefetch_map(&map_y);
+            bool ok = true;
+            int nq = 0, gkv = 0;
+            for (int k = 0; ok; ++k) {
+                const int w = item_index(k, cta, grid);
+                if (w >= n_items) break;
+                int m, bh;
+                decode(w, m, bh);
+                const int b = bh / n_head, h = bh % n_head;
+                const bool hasB = 2 * m + 1 < n_qt;
+                const int nkv = hasB ? 2 * m + 2 : 2 * m + 1;
+                const int qs = nq % kQStages;
+                if (nq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + qs), (uint32_t)((nq / kQStages) & 1) ^ 1u, g)))
+                    break;
+                const uint32_t qb = bar(kBarQFull + qs);
+                mbar_arrive_expect_tx(qb, (hasB ? 2u : 1u) * kTileBytes);
+                for (int t = 0; t < (hasB ? 2 : 1); ++t)
+                    tma_load_3d(sQ(qs, t), &map_qkv, qb, h * HS, (2 * m + t) * kTile, b);
+                ++nq;
+                for (int j = 0; j < nkv; ++j) {
+                    const int st = gkv % kKVStages;
+                    const uint32_t ph = (uint32_t)(gkv / kKVStages) & 1u;
+                    if (gkv >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + st), ph ^ 1u, g))) break;
+                    mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
+                    tma_load_3d(sK(st), &map_qkv, bar(kBarKFull + st), C + h * HS, j * kTile, b);
+                    mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
+                    tma_load_3d(sV(st), &map_qkv, bar(kBarVFull + st), 2 * C + h * HS, j * kTile, b);
+                    ++gkv;
+                }
+            }
+            if (!ok || *abort_flag) {
+                for (int q = (nq > kQStages ? nq - kQStages : 0); q < nq; ++q)
+                    drain_wait(bar(kBarQFull + q % kQStages), (uint32_t)(q / kQStages) & 1u, budget_ns);
+                for (int q = (gkv > kKVStages ? gkv - kKVStages : 0); q < gkv; ++q) {
+                    drain_wait(bar(kBarKFull + q % kKVStages), (uint32_t)(q / kKVStages) & 1u, budget_ns);
+                    drain_wait(bar(kBarVFull + q % kKVStages), (uint32_t)(q / kKVStages) & 1u, budget_ns);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+            constexpr uint32_t idPV = idesc_bf16_f32(128, HS, false, true);
+            const uint64_t dQ0 = sdesc_sw128(sQ(0, 0), 16, 1024);
+            const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
+            const uint64_t dV0 = sdesc_sw128(sV(0), kSlabBytes, 1024);
+            auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+            bool ok = true, any = false;
+            int n = 0, gkv = 0;
+            int sc[2] = {0, 0};     // S issued per stream
+            int pc[2] = {0, 0};     // P V issued per stream
+            int items[2] = {0, 0};  // items that used each stream
+            auto issue_S = [&](int qs, int t, int st) {
+                const uint64_t a = at(dQ0, (uint32_t)(2 * qs + t) * kTileBytes);
+                const uint64_t bk = at(dK0, (uint32_t)st * kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < HS / 16; ++kk)
+                    umma_ss(tmem + kColS + 128u * t, at(a, kk * 32u), at(bk, kk * 32u), idS, kk > 0 ? 1u : 0u);
+                umma_commit(bar(kBarSFull + t));
+                ++sc[t];
+            };
+            auto issue_PV = [&](int t, int st, bool first) {
+                const uint64_t bv = at(dV0, (uint32_t)st * kTileBytes);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tmem + kColO + 64u * t, tmem + kColP + 64u * t + 8u * kk, at(bv, kk * 2048u), idPV,
+                            (!first || kk > 0) ? 1u : 0u);
+                umma_commit(bar(kBarPVDone + t));
+                ++pc[t];
+            };
+            for (int k = 0; ok; ++k, ++n) {
+                const int w = item_index(k, cta, grid);
+                if (w >= n_items) break;
+                int m, bh;
+                decode(w, m, bh);
+                const bool hasB = 2 * m + 1 < n_qt;
+                const int nt[2] = {2 * m + 1, hasB ? 2 * m + 2 : 0};
+                const int nkv = hasB ? nt[1] : nt[0];
+                const int qs = n % kQStages;
+                if (!(ok = mbar_wait(bar(kBarQFull + qs), (uint32_t)(n / kQStages) & 1u, g))) break;
+                if (!(ok = mbar_wait(bar(kBarKFull + gkv % kKVStages), (uint32_t)(gkv / kKVStages) & 1u, g))) break;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (nt[t] == 0) continue;
+                    if (sc[t] > 0 && !(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
+                    tc_fence_after();
+                    issue_S(qs, t, gkv % kKVStages);
+                    any = true;
+                }
+                for (int j = 0; j < nkv && ok; ++j) {
+                    const int st = (gkv + j) % kKVStages;
+                    // S of the next key tile for each stream, as soon as its S buffer is free
+                    if (j + 1 < nkv) {
+                        const int st1 = (gkv + j + 1) % kKVStages;
+                        if (!(ok = mbar_wait(bar(kBarKFull + st1), (uint32_t)((gkv + j + 1) / kKVStages) & 1u, g))) break;
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (j + 1 >= nt[t]) continue;
+                            if (!(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
+                            tc_fence_after();
+                            issue_S(qs, t, st1);
+                        }
+                        if (!ok) break;
+                    }
+                    // P V of key tile j for each stream
+                    if (!(ok = mbar_wait(bar(kBarVFull + st), (uint32_t)((gkv + j) / kKVStages) & 1u, g))) break;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= nt[t]) continue;
+                        if (!(ok = mbar_wait(bar(kBarPFull + t), (uint32_t)pc[t] & 1u, g))) break;
+                        if (j == 0 && items[t] > 0 &&
+                            !(ok = mbar_wait(bar(kBarOFree + t), (uint32_t)(items[t] - 1) & 1u, g)))
+                            break;
+                        tc_fence_after();
+                        issue_PV(t, st, j == 0);
+                    }
+                    if (ok) umma_commit(bar(kBarKVEmpty + st));
+                }
+                gkv += nkv;
+                items[0] += 1;
+                items[1] += hasB ? 1 : 0;
+            }
+            if (any) {
+                umma_commit(bar(kBarDone));
+                drain_wait(bar(kBarDone), 0, budget_ns);
+            }
+        }
+    } else {
+        // ================================================================ softmax warpgroups
+        const int t = (warp - 2) >> 2;
+        const int sp = warp & 3;
+        const int row = sp * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
+        const uint32_t tS = trow + kColS + 128u * t;
+        const uint32_t tP = trow + kColP + 64u * t;
+        const uint32_t tO = trow + kColO + 64u * t;
+        const float scale_log2 = 0.125f * 1.4426950408889634f;
+        const uint64_t c2 = f32x2_pack(scale_log2, scale_log2);
+        const bool leader = (sp == 0 && lane == 0);
+        bool ok = true;
+        int it = 0, n = 0;
+        for (int k = 0;; ++k, ++n) {
+            const int w = item_index(k, cta, grid);
+            if (w >= n_items) break;
+            int m, bh;
+            decode(w, m, bh);
+            const int b = bh / n_head, h = bh % n_head;
+            const int qt = 2 * m + t;
+            const int qs = n % kQStages;
+            if (qt >= n_qt) {
+                if (leader) mbar_arrive(bar(kBarQEmpty + qs));
+                continue;
+            }
+            const int ntile = qt + 1;
+            float mrow = -INFINITY, l = 0.f, l_r = 0.f;
+            for (int j = 0; j < ntile; ++j, ++it) {
+                if (ok) ok = warp_wait(bar(kBarSFull + t), (uint32_t)it & 1u, g);
+                if (!ok) continue;
+                tc_fence_after();
+                uint32_t sr[128];
+                tmem_ld_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                tmem_ld_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                tc_fence_before();
+                mbar_arrive(bar(kBarSEmpty + t));  // S buffer may take the next tile
+                if (j == qt) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c > row) sr[c] = __float_as_uint(-INFINITY);
+                }
+                float mp[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mp[q] = __uint_as_float(sr[32 * q]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int c = 1; c < 31; c += 2)
+                        mp[q] = fmax3(mp[q], __uint_as_float(sr[32 * q + c]), __uint_as_float(sr[32 * q + c + 1]));
+                const float mx = fmax3(fmax3(mp[0], mp[1], __uint_as_float(sr[31])),
+                                       fmax3(mp[2], mp[3], __uint_as_float(sr[63])),
+                                       fmax3(__uint_as_float(sr[95]), __uint_as_float(sr[127]), -INFINITY));
+                const float m_cand = mx * scale_log2;
+                const bool grow = m_cand > mrow + 8.f;
+                const float m_new = grow ? m_cand : mrow;
+                const float alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
+                const uint64_t negm2 = f32x2_pack(-m_new, -m_new);
+                uint64_t sum2 = f32x2_pack(0.f, 0.f), sumr2 = f32x2_pack(0.f, 0.f);
+                uint32_t pk[64];
+#pragma unroll
+                for (int c = 0; c < 128; c += 2) {
+                    const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
+                    float x0, x1;
+                    f32x2_unpack(x, x0, x1);
+                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                    const uint32_t wv = pack_bf16x2(p0, p1);
+                    pk[c >> 1] = wv;
+                    sum2 = fadd2(sum2, f32x2_pack(p0, p1));
+                    sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                }
+                float s0, s1, r0, r1;
+                f32x2_unpack(sum2, s0, s1);
+                f32x2_unpack(sumr2, r0, r1);
+                l = l * alpha + (s0 + s1);
+                l_r = l_r * alpha + (r0 + r1);
+                mrow = m_new;
+                // P buffer and O are free once the previous P V of this stream retired
+                if (j > 0) {
+                    ok = warp_wait(bar(kBarPVDone + t), (uint32_t)(it - 1) & 1u, g);
+                    if (!ok) continue;
+                    tc_fence_after();
+                }
+                tmem_st_x32(tP + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
+                tmem_st_x32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int c0 = 0; c0 < HS; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld_x32(tO + c0, o);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tmem_st_x32(tO + c0, o);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar(kBarPFull + t));
+            }
+            // ------------------------------------------------------------ epilogue of this tile
+            const uint32_t stg = sQ(qs, t);
+            if (ok) ok = warp_wait(bar(kBarPVDone + t), (uint32_t)(it - 1) & 1u, g);
+            if (ok) {
+                tc_fence_after();
+                uint32_t o[64];
+                tmem_ld_x32(tO + 0, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                tmem_ld_x32(tO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                tc_fence_before();
+                mbar_arrive(bar(kBarOFree + t));
+                const float inv_l = 1.f / l_r;
+                const uint32_t rbase = stg + (uint32_t)row * 128u;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    uint32_t wv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(o[8 * q + 2 * e]) * inv_l,
+                                            __uint_as_float(o[8 * q + 2 * e + 1]) * inv_l);
+                    st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), wv[0], wv[1], wv[2], wv[3]);
+                }
+                fence_proxy_async_smem();
+                const int tq = qt * kTile + row;
+                if (tq < T) lse[(size_t)bh * (size_t)T + (size_t)tq] = (mrow + __log2f(l)) * 0.6931471805599453f;
+            }
+            named_bar_sync(1 + t, 128);
+            if (leader) {
+                if (ok && !*abort_flag) {
+                    tma_store_3d(&map_y, stg, h * HS, qt * kTile, b);
+                    bulk_commit_group();
+                    bulk_wait_group_read_0();
+                }
+                mbar_arrive(bar(kBarQEmpty + qs));
+            }
+        }
+        if (leader) bulk_wait_group_0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
+                           int n_head, DevCtx ctx, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_h64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int n_qt = ceil_div(T, kTile);
+    const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
+    const int grid = (int)(items < sms ? items : sms);
+    fwd_h64_kernel<<<dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s>>>(map_qkv, map_y, lse, B, T, C, n_head, n_qt,
+                                                                            ctx.status, ctx.budget_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace gptattn

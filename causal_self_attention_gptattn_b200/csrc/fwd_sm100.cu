@@ -462,7 +462,7 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
 
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T,
                             int C, int n_head, DevCtx ctx, cudaStream_t s) {
-    if (hs == 64) return launch_fwd_impl<64>(map_qkv, map_y, lse, B, T, C, n_head, ctx, s);
+    if (hs == 64) return launch_fwd_h64(map_qkv, map_y, lse, B, T, C, n_head, ctx, s);
     if (hs == 128) return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, ctx, s);
     return cudaErrorInvalidValue;
 }

@@ -27,6 +27,10 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse,
                             int B, int T, int C, int n_head, DevCtx ctx, cudaStream_t s);
 
+// Head-size-64 forward with separate P buffers (same arguments as above).
+cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
+                           int n_head, DevCtx ctx, cudaStream_t s);
+
 // D[bh][t] = sum_d y*dy, lse2[bh][t] = lse*log2(e) (rows t >= T: 0 and +inf),
 // dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].
 cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
