@@ -131,6 +131,7 @@ gptattn_status check_shape(int B, int T, int C, int n_head, gptattn_dtype dt, in
     const long long tiles = (long long)((T + kTile - 1) / kTile) * B * n_head;
     if (tiles > 0x7fffffffLL) return GPTATTN_ERR_UNSUPPORTED;
     if ((long long)B * n_head > 65535LL && dt == GPTATTN_F32) return GPTATTN_ERR_UNSUPPORTED;  // grid.y
+    if (dt == GPTATTN_BF16 && (B > 65535 || (T + kTile - 1) / kTile > 65535)) return GPTATTN_ERR_UNSUPPORTED;  // grid.y
     *hs_out = hs;
     return GPTATTN_OK;
 }

@@ -424,74 +424,78 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (negated so the main kernels add them); rows t >= T of each (b, h) get
 // 0 and -inf (so the recomputed P there is 0); dQ accumulator zeroed.
 // ---------------------------------------------------------------------------
+// 128-thread blocks, so that a whole (B * n_head, T_pad / 128) grid is resident at once
+// for the usual sizes (16 blocks per SM).
+constexpr int kPPThreads = 128;
+
+// Grid (B * n_head, T_pad / 128): a block takes one 128-row tile of one (b, h).
+// HS/8 lanes share a row (16 bytes of y and of dy each), so every warp load is a
+// set of whole 128-byte rows; the dot product is finished with shuffles.  The
+// block also zeroes its tile of the dQ accumulator.
 template <int HS>
-__global__ void bwd_pre_kernel(const __nv_bfloat16 *__restrict__ y, const __nv_bfloat16 *__restrict__ dy,
-                               const float *__restrict__ lse, float *__restrict__ D, float *__restrict__ lse2,
-                               float4 *__restrict__ dqacc, int B, int T, int C, int n_head, int T_pad) {
-    const long long rows = (long long)B * n_head * T_pad;
-    const long long zero4 = rows * HS / 4;
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < rows; idx += stride) {
-        const int t = (int)(idx % T_pad);
-        const long long bh = idx / T_pad;
-        const int h = (int)(bh % n_head);
-        const long long b = bh / n_head;
-        float d = 0.f, l2 = INFINITY;  // stored negated below: -D and -lse*log2(e)
+__global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16 *__restrict__ y,
+                                                      const __nv_bfloat16 *__restrict__ dy,
+                                                      const float *__restrict__ lse, float *__restrict__ D,
+                                                      float *__restrict__ lse2, float4 *__restrict__ dqacc, int T,
+                                                      int C, int n_head, int T_pad) {
+    constexpr int kLanesPerRow = HS / 8;
+    constexpr int kRowsPerPass = kPPThreads / kLanesPerRow;
+    const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
+    const int sub = threadIdx.x / kLanesPerRow, part = threadIdx.x % kLanesPerRow;
+    const size_t row0 = (size_t)bh * T_pad + (size_t)blockIdx.y * kTile;
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRowsPerPass) {
+        const int t = blockIdx.y * kTile + r + sub;
+        float d = 0.f;
         if (t < T) {
-            const size_t off = ((size_t)b * T + t) * (size_t)C + (size_t)h * HS;
-            const uint4 *yv = reinterpret_cast<const uint4 *>(y + off);
-            const uint4 *gv = reinterpret_cast<const uint4 *>(dy + off);
+            const size_t off = ((size_t)b * T + t) * (size_t)C + (size_t)h * HS + (size_t)part * 8;
+            const uint4 a = *reinterpret_cast<const uint4 *>(y + off);
+            const uint4 c = *reinterpret_cast<const uint4 *>(dy + off);
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-            for (int k = 0; k < HS / 8; ++k) {
-                const uint4 a = yv[k], c = gv[k];
-                const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    d = fmaf(bf16lo_to_f32(av[q]), bf16lo_to_f32(cv[q]), d);
-                    d = fmaf(bf16hi_to_f32(av[q]), bf16hi_to_f32(cv[q]), d);
-                }
+            for (int q = 0; q < 4; ++q) {
+                d = fmaf(bf16lo_to_f32(av[q]), bf16lo_to_f32(cv[q]), d);
+                d = fmaf(bf16hi_to_f32(av[q]), bf16hi_to_f32(cv[q]), d);
             }
-            l2 = lse[bh * T + t] * 1.4426950408889634f;
         }
-        D[idx] = -d;
-        lse2[idx] = -l2;
+#pragma unroll
+        for (int o = kLanesPerRow / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (part == 0) {  // stored negated: -D and -lse*log2(e); padded rows 0 and -inf
+            D[row0 + r + sub] = -d;
+            lse2[row0 + r + sub] = t < T ? -lse[(size_t)bh * T + t] * 1.4426950408889634f : -INFINITY;
+        }
     }
+    float4 *acc = dqacc + row0 * (HS / 4);
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < zero4; idx += stride) dqacc[idx] = z;
+#pragma unroll 4
+    for (int i = threadIdx.x; i < kTile * HS / 4; i += kPPThreads) acc[i] = z;
 }
 
-// postprocess: dq = bf16(dqacc * scale) into dqkv[..., 0:C]
+// postprocess: dq = bf16(dqacc * scale) into dqkv[..., 0:C].  Grid (B * n_head,
+// T_pad / 128): a block converts one 128-row tile of one (b, h), which is 32 KB
+// contiguous in the accumulator; a thread moves 8 elements at a time.
 template <int HS>
-__global__ void bwd_post_kernel(const float *__restrict__ dqacc, __nv_bfloat16 *__restrict__ dqkv, int B, int T,
-                                int C, int n_head, int T_pad) {
+__global__ void __launch_bounds__(kPPThreads) bwd_post_kernel(const float *__restrict__ dqacc, __nv_bfloat16 *__restrict__ dqkv,
+                                                       int T, int C, int n_head, int T_pad) {
+    constexpr int kPerRow = HS / 8;
     const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
-    const long long n8 = (long long)B * T * n_head * (HS / 8);
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < n8; idx += stride) {
-        const int k = (int)(idx % (HS / 8));
-        long long r = idx / (HS / 8);
-        const int h = (int)(r % n_head);
-        r /= n_head;
-        const int t = (int)(r % T);
-        const long long b = r / T;
-        const float4 *src = reinterpret_cast<const float4 *>(
-            dqacc + (((size_t)b * n_head + h) * (size_t)T_pad + (size_t)t) * HS + (size_t)k * 8);
-        const float4 a = src[0], c = src[1];
-        uint4 o;
-        o.x = pack_bf16x2(a.x * scale, a.y * scale);
-        o.y = pack_bf16x2(a.z * scale, a.w * scale);
-        o.z = pack_bf16x2(c.x * scale, c.y * scale);
-        o.w = pack_bf16x2(c.z * scale, c.w * scale);
-        *reinterpret_cast<uint4 *>(dqkv + ((size_t)b * T + t) * (size_t)(3 * C) + (size_t)h * HS + (size_t)k * 8) = o;
+    const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
+    const int t0 = blockIdx.y * kTile;
+    const float4 *src = reinterpret_cast<const float4 *>(dqacc + ((size_t)bh * T_pad + t0) * HS);
+    __nv_bfloat16 *dst = dqkv + ((size_t)b * T + t0) * (size_t)(3 * C) + (size_t)h * HS;
+#pragma unroll
+    for (int i = threadIdx.x; i < kTile * kPerRow; i += kPPThreads) {
+        const int r = i / kPerRow, k = i % kPerRow;
+        if (t0 + r < T) {
+            const float4 a = src[2 * i], c = src[2 * i + 1];
+            uint4 o;
+            o.x = pack_bf16x2(a.x * scale, a.y * scale);
+            o.y = pack_bf16x2(a.z * scale, a.w * scale);
+            o.z = pack_bf16x2(c.x * scale, c.y * scale);
+            o.w = pack_bf16x2(c.z * scale, c.w * scale);
+            *reinterpret_cast<uint4 *>(dst + (size_t)r * (size_t)(3 * C) + (size_t)k * 8) = o;
+        }
     }
-}
-
-inline unsigned grid_for(long long work, int threads) {
-    long long blocks = (work + threads - 1) / threads;
-    const long long cap = 148LL * 16;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    return (unsigned)blocks;
 }
 
 template <int HS>
@@ -513,15 +517,14 @@ cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_
 
 cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
                                 float *dqacc, int B, int T, int C, int n_head, int T_pad, cudaStream_t s) {
-    const long long work = (long long)B * n_head * T_pad * hs / 4;
-    const unsigned grid = grid_for(work, 256);
+    const dim3 grid((unsigned)(B * n_head), (unsigned)(T_pad / kTile));
     auto yy = static_cast<const __nv_bfloat16 *>(y);
     auto gg = static_cast<const __nv_bfloat16 *>(dy);
     auto zz = reinterpret_cast<float4 *>(dqacc);
     if (hs == 64)
-        bwd_pre_kernel<64><<<grid, 256, 0, s>>>(yy, gg, lse, D, lse2, zz, B, T, C, n_head, T_pad);
+        bwd_pre_kernel<64><<<grid, kPPThreads, 0, s>>>(yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
     else if (hs == 128)
-        bwd_pre_kernel<128><<<grid, 256, 0, s>>>(yy, gg, lse, D, lse2, zz, B, T, C, n_head, T_pad);
+        bwd_pre_kernel<128><<<grid, kPPThreads, 0, s>>>(yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
@@ -540,16 +543,14 @@ cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUten
 
 cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head, int T_pad,
                                  cudaStream_t s) {
-    const long long work = (long long)B * T * n_head * hs / 8;
-    const unsigned grid = grid_for(work, 256);
+    const dim3 grid((unsigned)(B * n_head), (unsigned)(T_pad / kTile));
     auto out = static_cast<__nv_bfloat16 *>(dqkv);
     if (hs == 64)
-        bwd_post_kernel<64><<<grid, 256, 0, s>>>(dqacc, out, B, T, C, n_head, T_pad);
+        bwd_post_kernel<64><<<grid, kPPThreads, 0, s>>>(dqacc, out, T, C, n_head, T_pad);
     else if (hs == 128)
-        bwd_post_kernel<128><<<grid, 256, 0, s>>>(dqacc, out, B, T, C, n_head, T_pad);
+        bwd_post_kernel<128><<<grid, kPPThreads, 0, s>>>(dqacc, out, T, C, n_head, T_pad);
     else
         return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
-
 }  // namespace gptattn
