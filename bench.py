@@ -52,6 +52,35 @@ def parse_args():
     return p.parse_args()
 
 
+# DRAM traffic per launch of the dominant kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum) of the same workload; reported
+# only while the sources it was taken on are unchanged (sha256 over the files).
+MEASURED_TRAFFIC = {
+    ("bwd_bf16_sm100", "gpt2_124m"): {
+        "bytes": 202.071552e6 + 83.947776e6,
+        "sources": ("bwd_h64_sm100.cu", "sm100_ptx.cuh", "kernels.h"),
+        "sha256": "139e3df576d4bebbdc2826aface4ec533f42215f7f92f3c28f8191ab4706114c",
+        "capture": "profiles/bwd_h64_persistent_gpt2_124m.md",
+    },
+}
+
+
+def measured_traffic(kernel: str, workload: str):
+    import hashlib
+    rec = MEASURED_TRAFFIC.get((kernel, workload))
+    if rec is None:
+        return None
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "causal_self_attention_gptattn_b200", "csrc")
+    try:
+        for f in rec["sources"]:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return rec["bytes"] if h.hexdigest() == rec["sha256"] else None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -317,7 +346,8 @@ def run_ours(args, w, rank, world, local_rank):
         peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "peak_source": f"{peak_src} bf16 burst",
-                    "traffic": None, "avg_ms": dom_ms}
+                    "traffic": measured_traffic(dominant, args.workload), "traffic_unit": "bytes per launch",
+                    "avg_ms": dom_ms}
 
     cpu = None
     if world == 1 and not (args.skip_cpu_baseline or args.profile_run):
