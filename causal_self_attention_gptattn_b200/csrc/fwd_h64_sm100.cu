@@ -319,7 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_new = grow ? m_cand : mrow;
                 const float alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
                 const uint64_t negm2 = f32x2_pack(-m_new, -m_new);
-                uint64_t sum2 = f32x2_pack(0.f, 0.f), sumr2 = f32x2_pack(0.f, 0.f);
+                // four independent partial sums each, so the adds do not form one long chain
+                uint64_t sum2[4], sumr2[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) sum2[a] = sumr2[a] = f32x2_pack(0.f, 0.f);
                 uint32_t pk[64];
 #pragma unroll
                 for (int c = 0; c < 128; c += 2) {
@@ -329,12 +332,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                     const uint32_t wv = pack_bf16x2(p0, p1);
                     pk[c >> 1] = wv;
-                    sum2 = fadd2(sum2, f32x2_pack(p0, p1));
-                    sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                    const int a = (c >> 1) & 3;
+                    sum2[a] = fadd2(sum2[a], f32x2_pack(p0, p1));
+                    sumr2[a] = fadd2(sumr2[a], f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
                 }
                 float s0, s1, r0, r1;
-                f32x2_unpack(sum2, s0, s1);
-                f32x2_unpack(sumr2, r0, r1);
+                f32x2_unpack(fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3])), s0, s1);
+                f32x2_unpack(fadd2(fadd2(sumr2[0], sumr2[1]), fadd2(sumr2[2], sumr2[3])), r0, r1);
                 l = l * alpha + (s0 + s1);
                 l_r = l_r * alpha + (r0 + r1);
                 mrow = m_new;
