@@ -153,6 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_launch_dependents();
+    griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
     if (warp == 0) {
         // ================================================================ producer
@@ -498,9 +500,8 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
     const int n_t = ceil_div(T, kTile);
     const long long items = (long long)n_t * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    bwd_h64_persistent<<<dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s>>>(
-        map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
-    return cudaGetLastError();
+    return launch_pdl(bwd_h64_persistent, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_dy, map_dqkv,
+                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

@@ -145,6 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_launch_dependents();
+    griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -440,6 +442,8 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
                                                       int C, int n_head, int T_pad) {
     constexpr int kLanesPerRow = HS / 8;
     constexpr int kRowsPerPass = kPPThreads / kLanesPerRow;
+    griddep_launch_dependents();
+    griddep_wait();
     const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
     const int sub = threadIdx.x / kLanesPerRow, part = threadIdx.x % kLanesPerRow;
     const size_t row0 = (size_t)bh * T_pad + (size_t)blockIdx.y * kTile;
@@ -479,6 +483,8 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_kernel(const float *__res
                                                        int T, int C, int n_head, int T_pad) {
     constexpr int kPerRow = HS / 8;
     const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
+    griddep_launch_dependents();
+    griddep_wait();
     const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
     const int t0 = blockIdx.y * kTile;
     const float4 *src = reinterpret_cast<const float4 *>(dqacc + ((size_t)bh * T_pad + t0) * HS);
@@ -508,9 +514,8 @@ cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_
     if (e != cudaSuccess) return e;
     const int n_t = ceil_div(T, kTile);
     const long long blocks = (long long)n_t * B * n_head;
-    bwd_bf16_kernel<HS><<<dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s>>>(
-        map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
-    return cudaGetLastError();
+    return launch_pdl(bwd_bf16_kernel<HS>, dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_dy,
+                      map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace
@@ -521,13 +526,9 @@ cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const flo
     auto yy = static_cast<const __nv_bfloat16 *>(y);
     auto gg = static_cast<const __nv_bfloat16 *>(dy);
     auto zz = reinterpret_cast<float4 *>(dqacc);
-    if (hs == 64)
-        bwd_pre_kernel<64><<<grid, kPPThreads, 0, s>>>(yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
-    else if (hs == 128)
-        bwd_pre_kernel<128><<<grid, kPPThreads, 0, s>>>(yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
-    else
-        return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    if (hs == 64) return launch_pdl(bwd_pre_kernel<64>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
+    if (hs == 128) return launch_pdl(bwd_pre_kernel<128>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
@@ -545,12 +546,8 @@ cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, 
                                  cudaStream_t s) {
     const dim3 grid((unsigned)(B * n_head), (unsigned)(T_pad / kTile));
     auto out = static_cast<__nv_bfloat16 *>(dqkv);
-    if (hs == 64)
-        bwd_post_kernel<64><<<grid, kPPThreads, 0, s>>>(dqacc, out, T, C, n_head, T_pad);
-    else if (hs == 128)
-        bwd_post_kernel<128><<<grid, kPPThreads, 0, s>>>(dqacc, out, T, C, n_head, T_pad);
-    else
-        return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    if (hs == 64) return launch_pdl(bwd_post_kernel<64>, grid, dim3(kPPThreads), 0, s, dqacc, out, T, C, n_head, T_pad);
+    if (hs == 128) return launch_pdl(bwd_post_kernel<128>, grid, dim3(kPPThreads), 0, s, dqacc, out, T, C, n_head, T_pad);
+    return cudaErrorInvalidValue;
 }
 }  // namespace gptattn

@@ -129,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_launch_dependents();
+    griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
     if (warp == 0) {
         // ================================================================ producer
@@ -423,9 +425,8 @@ cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y,
     const int n_qt = ceil_div(T, kTile);
     const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    fwd_h64_kernel<<<dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s>>>(map_qkv, map_y, lse, B, T, C, n_head, n_qt,
-                                                                            ctx.status, ctx.budget_ns);
-    return cudaGetLastError();
+    return launch_pdl(fwd_h64_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_y, lse, B, T, C,
+                      n_head, n_qt, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

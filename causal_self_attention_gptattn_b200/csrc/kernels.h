@@ -21,6 +21,26 @@ constexpr int kTile = 128;
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Launch with programmatic stream serialisation: the kernel's CTAs may start
+// (and run their prologue) while the previous kernel of the stream finishes;
+// every kernel launched this way calls griddep_wait() before touching global
+// memory, so results are as with an ordinary launch.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // ---- bf16 tensor-core path (sm_100a) --------------------------------------
 // map_qkv: 3-D view (3C, T, B) of qkv, box (64, 128, 1), 128-byte swizzle.
 // map_y:   3-D view (C, T, B) of y, same box.

@@ -95,6 +95,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     }
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel of the
+// stream (launched with programmatic stream serialisation) start its CTAs as
+// SMs free up; wait blocks until the previous kernel of the stream has completed
+// and its memory is visible.  Both are no-ops without such a launch.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Named barrier for a subset of warps (ids 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
