@@ -8,8 +8,10 @@
 // The workspace rows hold -D and -lse*log2(e) (negated by the preprocess kernel).
 //
 // Schedule: one persistent CTA per SM walks a static list of work items
-// (key tile j, batch b, head h), ordered longest first (small j first), with
-// stride gridDim.x.  Per item the CTA loops over query tiles i >= j.
+// (key tile j, batch b, head h), ordered longest first (small j first), in a
+// snake order over the CTAs (round k takes items k*grid .. k*grid+grid-1,
+// reversed on odd rounds), which evens out the causal triangle's work across
+// CTAs.  Per item the CTA loops over query tiles i >= j.
 //
 // Warp roles (14 warps):
 //   warp 0        TMA producer: K_j, V_j (double-buffered across items), and
@@ -91,6 +93,10 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
+__device__ __forceinline__ int item_index(int k, int cta, int grid) {
+    return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_h64_persistent(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
                        const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
@@ -164,7 +170,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             int n = 0;   // items started
             int gq = 0;  // query tiles issued (ring position)
-            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++n) {
+            for (int k = 0; ok; ++k, ++n) {
+                const int w = item_index(k, blockIdx.x, gridDim.x);
+                if (w >= n_items) break;
                 const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
                 const int kvs = n & 1;
                 if (n >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + kvs), (uint32_t)((n >> 1) & 1) ^ 1u, g)))
@@ -224,7 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_ss(tmem + kColdP, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
                 umma_commit(bar(kBardPFull));
             };
-            for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x, ++n) {
+            for (int k = 0; ok; ++k, ++n) {
+                const int w = item_index(k, blockIdx.x, gridDim.x);
+                if (w >= n_items) break;
                 const int kt = w / BH;
                 const int niter = n_t - kt;
                 const int kvs = n & 1;
@@ -308,7 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t c2 = f32x2_pack(scale_log2, scale_log2);
         bool ok = true;
         int n = 0, gi = 0;
-        for (int w = blockIdx.x; w < n_items; w += gridDim.x, ++n) {
+        for (int k = 0;; ++k, ++n) {
+            const int w = item_index(k, blockIdx.x, gridDim.x);
+            if (w >= n_items) break;
             const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
             const int niter = n_t - kt;
             for (int it = 0; it < niter; ++it, ++gi) {
@@ -442,7 +454,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool leader = (warp == 10 && lane == 0);
         bool ok = true;
         int gi = 0;
-        for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+        for (int k = 0;; ++k) {
+            const int w = item_index(k, blockIdx.x, gridDim.x);
+            if (w >= n_items) break;
             const int kt = w / BH, bh = w % BH;
             for (int qt = kt; qt < n_t; ++qt, ++gi) {
                 if (ok) ok = warp_wait(bar(kBardQFull), (uint32_t)gi & 1u, g);
