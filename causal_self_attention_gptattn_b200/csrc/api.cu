@@ -278,6 +278,22 @@ gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse, int B, int T, i
     return from_cuda(run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, ctx, s); }));
 }
 
+gptattn_status gptattn_decode(const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C, int n_head,
+                              gptattn_dtype dt, gptattn_stream_t stream) {
+    int hs = 0;
+    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
+    if (st != GPTATTN_OK) return st;
+    if (T_cap < T) return GPTATTN_ERR_INVALID_ARG;
+    if ((long long)B * n_head > 65535LL) return GPTATTN_ERR_UNSUPPORTED;  // grid.y
+    if (B == 0 || T == 0) return GPTATTN_OK;
+    if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return from_cuda(run_kernel(kKDecode, s, [&] {
+        return launch_decode(hs, dt == GPTATTN_BF16, qkv, y, lse, B, T, T_cap, C, n_head, s);
+    }));
+}
+
 size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt) {
     int hs = 0;
     if (check_shape(B, T, C, n_head, dt, &hs) != GPTATTN_OK) return (size_t)-1;
@@ -395,7 +411,7 @@ int gptattn_profile_read(int *kernel_ids, float *ms, int capacity) {
 const char *gptattn_kernel_name(int kernel_id) {
     static const char *names[kKNumKernels] = {
         "fwd_bf16_sm100", "bwd_pre_bf16", "bwd_bf16_sm100", "bwd_post_bf16", "fwd_f32_simt",
-        "bwd_pre_f32",    "bwd_dq_f32",   "bwd_dkv_f32",    "selftest_timeout"};
+        "bwd_pre_f32",    "bwd_dq_f32",   "bwd_dkv_f32",    "selftest_timeout", "decode"};
     if (kernel_id < 0 || kernel_id >= kKNumKernels) return "unknown";
     return names[kernel_id];
 }

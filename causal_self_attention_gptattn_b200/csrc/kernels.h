@@ -82,6 +82,10 @@ cudaError_t launch_bwd_f32_dq(int hs, const float *qkv, const float *dy, const f
 cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
                                float *dqkv, int B, int T, int C, int n_head, cudaStream_t s);
 
+// ---- decode: last position over a key/value cache (cluster of 8 CTAs per (b, h))
+cudaError_t launch_decode(int hs, bool bf16, const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C,
+                          int n_head, cudaStream_t s);
+
 // ---- bounded-wait self-test -----------------------------------------------
 cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s);
 
@@ -96,7 +100,8 @@ enum KernelId {
     kKBwdDqF32 = 6,
     kKBwdDkvF32 = 7,
     kKSelftest = 8,
-    kKNumKernels = 9
+    kKDecode = 9,
+    kKNumKernels = 10
 };
 
 }  // namespace gptattn

@@ -83,6 +83,24 @@ GPTATTN_API gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse,
                            int B, int T, int C, int n_head,
                            gptattn_dtype dt, gptattn_stream_t stream);
 
+/* Decode: attention of the last position over a key/value cache (no
+ * counterpart on the pages beyond the operation itself: it is row T-1 of
+ * gptattn_fwd, the only row the pages' generate loop reads, computed without
+ * the other rows).  For every batch b and head h, with q the head's query of
+ * position T-1 and k_s, v_s its keys and values of positions 0..T-1 (all
+ * visible to the last position):
+ *     y[b][h*hs + d] = sum_s P[s] v_s[d],  P = softmax_s(q . k_s / sqrt(hs)),
+ *     lse[b][h]      = ln sum_s exp(q . k_s / sqrt(hs)).
+ * The cache is a packed qkv buffer [B][T_cap][3C] (same column layout as
+ * gptattn_fwd's qkv, batch stride T_cap rows) of which rows 0..T-1 are read;
+ * y is [B][C] (dtype dt), lse is [B][n_head] float32.  T_cap >= T; B * n_head
+ * <= 65535.  Same dtypes, head sizes, pointer rules and error codes as
+ * gptattn_fwd; B == 0 or T == 0 is a valid empty call.  Memory-bound; it reads
+ * each key and value row once and allocates nothing. */
+GPTATTN_API gptattn_status gptattn_decode(const void *qkv, void *y, float *lse,
+                              int B, int T, int T_cap, int C, int n_head,
+                              gptattn_dtype dt, gptattn_stream_t stream);
+
 /* Bytes of device scratch gptattn_bwd needs for this shape (0 for an empty
  * shape; (size_t)-1 for an invalid one).  Pure host function. */
 GPTATTN_API size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt);

@@ -108,3 +108,16 @@ def test_profile_enable_rejects_negative():
     assert ga.gptattn_profile_enable(-1) == ga.GPTATTN_ERR_INVALID_ARG
     assert ga.gptattn_profile_enable(0) == ga.GPTATTN_OK
     assert ga.gptattn_profile_read(8) == []
+
+
+def test_decode_validation():
+    bf, f32 = ga.GPTATTN_BF16, ga.GPTATTN_F32
+    assert ga.gptattn_decode(FAKE, FAKE, FAKE, 2, 9, 8, 128, 2, bf, None) == ga.GPTATTN_ERR_INVALID_ARG  # T > T_cap
+    assert ga.gptattn_decode(FAKE, FAKE, FAKE, 2, 8, 8, 96, 3, bf, None) == ga.GPTATTN_ERR_UNSUPPORTED  # hs = 32 on bf16
+    assert ga.gptattn_decode(FAKE, FAKE, FAKE, 2, 8, 8, 96, 4, f32, None) == ga.GPTATTN_ERR_UNSUPPORTED  # hs = 24
+    assert ga.gptattn_decode(FAKE, FAKE, FAKE, 40000, 8, 8, 128, 2, bf, None) == ga.GPTATTN_ERR_UNSUPPORTED  # grid.y
+    assert ga.gptattn_decode(None, FAKE, FAKE, 2, 8, 8, 128, 2, bf, None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_decode(FAKE, FAKE + 2, FAKE, 2, 8, 8, 128, 2, bf, None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_decode(None, None, None, 0, 8, 8, 128, 2, bf, None) == ga.GPTATTN_OK
+    assert ga.gptattn_decode(None, None, None, 2, 0, 8, 128, 2, f32, None) == ga.GPTATTN_OK
+    assert ga.gptattn_kernel_name(9) == "decode"
