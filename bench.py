@@ -374,6 +374,51 @@ def run_ours(args, w, rank, world, local_rank):
     h2d = qkv_h.numel() * qkv_h.element_size() + dy_h.numel() * dy_h.element_size()
     d2h = y_h.numel() * y_h.element_size() + dqkv_h.numel() * dqkv_h.element_size()
 
+    # ---- decode (gptattn_decode): the last position of every sequence over the same qkv as a
+    # key/value cache; HBM-bound, so its roofline is the measured copy bandwidth.  L2 flushed
+    # before every call.  Also a large cache (B=64, T=4096 at this head layout) for the
+    # asymptotic bandwidth.
+    decode = None
+    if not args.profile_run:
+        peaks_d, src_d = load_peaks()
+        hbm = float(peaks_d.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        yd = torch.empty(B, C, dtype=w.torch_dtype, device=dev)
+        ld = torch.empty(B, nh, dtype=torch.float32, device=dev)
+
+        def time_decode(q, Bq, Tq, reps, flush_each):
+            for _ in range(3):
+                ga.check(ga.gptattn_decode(q, yd if Bq == B else yl, ld if Bq == B else ll, Bq, Tq, Tq, C, nh, dt, s),
+                         "gptattn_decode")
+            torch.cuda.synchronize()
+            tot = 0.0
+            for _ in range(reps):
+                if flush_each:
+                    flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b_ = torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                ga.check(ga.gptattn_decode(q, yd if Bq == B else yl, ld if Bq == B else ll, Bq, Tq, Tq, C, nh, dt, s),
+                         "gptattn_decode")
+                b_.record(s)
+                torch.cuda.synchronize()
+                tot += a.elapsed_time(b_)
+            return tot / reps
+
+        ms_d = time_decode(qkv, B, T, 50, True)
+        kv_bytes = B * T * 2 * C * qkv.element_size()
+        BL, TL = 64, 4096
+        ql = torch.empty(BL, TL, 3 * C, dtype=w.torch_dtype, device=dev).normal_()
+        yl = torch.empty(BL, C, dtype=w.torch_dtype, device=dev)
+        ll = torch.empty(BL, nh, dtype=torch.float32, device=dev)
+        ms_l = time_decode(ql, BL, TL, 20, False)
+        kv_l = BL * TL * 2 * C * ql.element_size()
+        del ql
+        decode = {"workload": f"{w.name}: last position of each of the B={B} sequences over T={T} cached keys",
+                  "us_per_call": ms_d * 1e3, "kv_bytes": kv_bytes, "achieved_gbs": kv_bytes / ms_d / 1e6,
+                  "frac_of_hbm": kv_bytes / ms_d / 1e6 / hbm, "peak_source": f"{src_d} copy bandwidth",
+                  "large_cache": {"B": BL, "T": TL, "us_per_call": ms_l * 1e3, "kv_bytes": kv_l,
+                                  "achieved_gbs": kv_l / ms_l / 1e6, "frac_of_hbm": kv_l / ms_l / 1e6 / hbm}}
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -423,6 +468,7 @@ def run_ours(args, w, rank, world, local_rank):
                 "steps": Ke, "ms_per_step": (e2e_ms / Ke if Ke else None),
                 "overlap": "copies in / compute / copies out on three streams, device buffers double-buffered"},
         "gpu_launches": launches,
+        "decode": decode,
         "clocks": clocks,
         "wall_s_timed": wall1 - wall0,
     }
