@@ -82,6 +82,12 @@ class Oracle:
         lib.oracle_bwd.restype = i
         lib.oracle_probs.argtypes = [dp, i, i, i, i, i, i, dp]
         lib.oracle_probs.restype = i
+        lib.oracle_fwd_window.argtypes = [dp, i, i, i, i, i, dp, dp]
+        lib.oracle_fwd_window.restype = i
+        lib.oracle_bwd_window.argtypes = [dp, dp, i, i, i, i, i, dp]
+        lib.oracle_bwd_window.restype = i
+        lib.oracle_probs_window.argtypes = [dp, i, i, i, i, i, i, i, dp]
+        lib.oracle_probs_window.restype = i
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i
         lib.oracle_set_num_threads.argtypes = [i]
@@ -95,36 +101,46 @@ class Oracle:
     def set_num_threads(self, n: int) -> None:
         self.lib.oracle_set_num_threads(int(n))
 
-    def forward(self, qkv, n_head: int):
-        """Return (y[B,T,C], lse[B,n_head,T]) in float64."""
+    def forward(self, qkv, n_head: int, window=None):
+        """Return (y[B,T,C], lse[B,n_head,T]) in float64.  window: local band width
+        (token t sees t-window < s <= t); None = causal (every past position)."""
         q = _f64(qkv)
         B, T, C = _shape(q, n_head)
         y = np.zeros((B, T, C), dtype=np.float64)
         lse = np.zeros((B, n_head, T), dtype=np.float64)
-        rc = self.lib.oracle_fwd(_ptr(q), B, T, C, n_head, _ptr(y), _ptr(lse))
+        if window is None:
+            rc = self.lib.oracle_fwd(_ptr(q), B, T, C, n_head, _ptr(y), _ptr(lse))
+        else:
+            rc = self.lib.oracle_fwd_window(_ptr(q), B, T, C, n_head, int(window), _ptr(y), _ptr(lse))
         if rc:
             raise RuntimeError(f"oracle_fwd failed with code {rc}")
         return y, lse
 
-    def backward(self, qkv, dy, n_head: int):
-        """Return dqkv[B,T,3C] = d(sum(y*dy))/d(qkv) in float64."""
+    def backward(self, qkv, dy, n_head: int, window=None):
+        """Return dqkv[B,T,3C] = d(sum(y*dy))/d(qkv) in float64 (window as in forward)."""
         q = _f64(qkv)
         g = _f64(dy)
         B, T, C = _shape(q, n_head)
         if g.shape != (B, T, C):
             raise ValueError(f"dy must be {(B, T, C)}, got {g.shape}")
         dqkv = np.zeros((B, T, 3 * C), dtype=np.float64)
-        rc = self.lib.oracle_bwd(_ptr(q), _ptr(g), B, T, C, n_head, _ptr(dqkv))
+        if window is None:
+            rc = self.lib.oracle_bwd(_ptr(q), _ptr(g), B, T, C, n_head, _ptr(dqkv))
+        else:
+            rc = self.lib.oracle_bwd_window(_ptr(q), _ptr(g), B, T, C, n_head, int(window), _ptr(dqkv))
         if rc:
             raise RuntimeError(f"oracle_bwd failed with code {rc}")
         return dqkv
 
-    def probs(self, qkv, n_head: int, b: int, h: int):
-        """Return the T x T attention weights of batch b, head h."""
+    def probs(self, qkv, n_head: int, b: int, h: int, window=None):
+        """Return the T x T attention weights of batch b, head h (window as in forward)."""
         q = _f64(qkv)
         B, T, C = _shape(q, n_head)
         P = np.zeros((T, T), dtype=np.float64)
-        rc = self.lib.oracle_probs(_ptr(q), B, T, C, n_head, int(b), int(h), _ptr(P))
+        if window is None:
+            rc = self.lib.oracle_probs(_ptr(q), B, T, C, n_head, int(b), int(h), _ptr(P))
+        else:
+            rc = self.lib.oracle_probs_window(_ptr(q), B, T, C, n_head, int(window), int(b), int(h), _ptr(P))
         if rc:
             raise RuntimeError(f"oracle_probs failed with code {rc}")
         return P
@@ -146,13 +162,13 @@ def set_num_threads(n: int) -> None:
     default().set_num_threads(n)
 
 
-def forward(qkv, n_head: int):
-    return default().forward(qkv, n_head)
+def forward(qkv, n_head: int, window=None):
+    return default().forward(qkv, n_head, window)
 
 
-def backward(qkv, dy, n_head: int):
-    return default().backward(qkv, dy, n_head)
+def backward(qkv, dy, n_head: int, window=None):
+    return default().backward(qkv, dy, n_head, window)
 
 
-def probs(qkv, n_head: int, b: int, h: int):
-    return default().probs(qkv, n_head, b, h)
+def probs(qkv, n_head: int, b: int, h: int, window=None):
+    return default().probs(qkv, n_head, b, h, window)

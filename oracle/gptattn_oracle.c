@@ -27,6 +27,12 @@
  *    self-attention": all heads at once, heads treated as one more batch
  *    dimension; head h owns columns [h*hs, (h+1)*hs) of each of q, k, v.
  *  - same page, note 3: no communication across the batch dimension.
+ *  - minGPT README page ("卡帕西(氏)MinGPT"), reference notes on GPT-3: the
+ *    layers alternate dense attention with locally banded sparse attention
+ *    (no band width is given).  Read here as a local window of `window`
+ *    positions: token t sees s with t - window < s <= t (itself and the
+ *    window-1 before it); window >= T is the dense causal case above, with the
+ *    same arithmetic.
  *
  * Input packing (the projection output of a GPT-2 style block): qkv[B][T][3C]
  * row-major, q = columns [0,C), k = [C,2C), v = [2C,3C).  Output y[B][T][C]
@@ -68,43 +74,50 @@ static inline double qkv_at(const double *qkv, int T, int C, int hs, int b, int 
     return qkv[row * (size_t)(3 * C) + (size_t)part * (size_t)C + (size_t)h * (size_t)hs + (size_t)d];
 }
 
-/* Attention weights of one (b, h): P[t][s] for s <= t, 0 for s > t, and the
- * per-row logsumexp of the masked scaled scores.  P is a T*T buffer. */
-static void head_probs(const double *qkv, int T, int C, int hs, int b, int h,
+/* First key position visible to query t, and last query position that sees key s. */
+static inline int band_lo(int t, int window) { return t - window + 1 > 0 ? t - window + 1 : 0; }
+static inline int band_hi(int s, int window, int T) { return s + window - 1 < T - 1 ? s + window - 1 : T - 1; }
+
+/* Attention weights of one (b, h): P[t][s] for the visible band lo(t) <= s <= t,
+ * 0 elsewhere, and the per-row logsumexp of the masked scaled scores.  P is a
+ * T*T buffer. */
+static void head_probs(const double *qkv, int T, int C, int hs, int window, int b, int h,
                        double *P, double *lse_row) {
     const double scale = 1.0 / sqrt((double)hs);
     for (int t = 0; t < T; ++t) {
         double *Pt = P + (size_t)t * (size_t)T;
-        /* scores S[t][s] = q_t . k_s / sqrt(hs) for the visible past s <= t */
+        const int lo = band_lo(t, window);
+        /* scores S[t][s] = q_t . k_s / sqrt(hs) for the visible s */
         double m = -INFINITY;
-        for (int s = 0; s <= t; ++s) {
+        for (int s = lo; s <= t; ++s) {
             double acc = 0.0;
             for (int d = 0; d < hs; ++d)
                 acc += qkv_at(qkv, T, C, hs, b, t, 0, h, d) * qkv_at(qkv, T, C, hs, b, s, 1, h, d);
             Pt[s] = acc * scale;
             if (Pt[s] > m) m = Pt[s];
         }
-        /* softmax over the visible row; the future gets weight zero */
+        /* softmax over the visible row; the future (and the past outside the band) gets weight zero */
         double l = 0.0;
-        for (int s = 0; s <= t; ++s) {
+        for (int s = lo; s <= t; ++s) {
             Pt[s] = exp(Pt[s] - m);
             l += Pt[s];
         }
-        for (int s = 0; s <= t; ++s) Pt[s] /= l;
+        for (int s = lo; s <= t; ++s) Pt[s] /= l;
+        for (int s = 0; s < lo; ++s) Pt[s] = 0.0;
         for (int s = t + 1; s < T; ++s) Pt[s] = 0.0;
         if (lse_row) lse_row[t] = m + log(l);
     }
 }
 
 /* y[b,t,h*hs+d] = sum_s P[t][s] v_s[d] */
-static void head_output(const double *qkv, int T, int C, int hs, int b, int h,
+static void head_output(const double *qkv, int T, int C, int hs, int window, int b, int h,
                         const double *P, double *y) {
     for (int t = 0; t < T; ++t) {
         const double *Pt = P + (size_t)t * (size_t)T;
         double *yt = y + ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)h * (size_t)hs;
         for (int d = 0; d < hs; ++d) {
             double acc = 0.0;
-            for (int s = 0; s <= t; ++s) acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);
+            for (int s = band_lo(t, window); s <= t; ++s) acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);
             yt[d] = acc;
         }
     }
@@ -126,10 +139,12 @@ void oracle_set_num_threads(int n) {
 #endif
 }
 
-/* Forward: y[B][T][C] and lse[B][n_head][T] (either may be NULL). */
-int oracle_fwd(const double *qkv, int B, int T, int C, int n_head, double *y, double *lse) {
+/* Forward over a local window: y[B][T][C] and lse[B][n_head][T] (either may be
+ * NULL).  window >= 1. */
+int oracle_fwd_window(const double *qkv, int B, int T, int C, int n_head, int window, double *y, double *lse) {
     int rc = check_shape(B, T, C, n_head);
     if (rc) return rc;
+    if (window < 1) return ORACLE_EINVAL;
     if (B == 0 || T == 0) return ORACLE_OK;
     const int hs = C / n_head;
     const int pairs = B * n_head;
@@ -146,30 +161,41 @@ int oracle_fwd(const double *qkv, int B, int T, int C, int n_head, double *y, do
             if (!P) continue;
             const int b = p / n_head, h = p % n_head;
             double *lse_row = lse ? lse + ((size_t)b * (size_t)n_head + (size_t)h) * (size_t)T : NULL;
-            head_probs(qkv, T, C, hs, b, h, P, lse_row);
-            if (y) head_output(qkv, T, C, hs, b, h, P, y);
+            head_probs(qkv, T, C, hs, window, b, h, P, lse_row);
+            if (y) head_output(qkv, T, C, hs, window, b, h, P, y);
         }
         free(P);
     }
     return err ? ORACLE_ENOMEM : ORACLE_OK;
 }
 
+/* Forward, causal (every past position visible). */
+int oracle_fwd(const double *qkv, int B, int T, int C, int n_head, double *y, double *lse) {
+    return oracle_fwd_window(qkv, B, T, C, n_head, T > 0 ? T : 1, y, lse);
+}
+
 /* Attention weights of one (b, h) as a dense T*T matrix (the "wei" of the
  * lecture's versions 2-4), for tests that inspect the weights directly. */
-int oracle_probs(const double *qkv, int B, int T, int C, int n_head, int b, int h, double *P) {
+int oracle_probs_window(const double *qkv, int B, int T, int C, int n_head, int window, int b, int h, double *P) {
     int rc = check_shape(B, T, C, n_head);
     if (rc) return rc;
-    if (b < 0 || b >= B || h < 0 || h >= n_head) return ORACLE_EINVAL;
+    if (window < 1 || b < 0 || b >= B || h < 0 || h >= n_head) return ORACLE_EINVAL;
     if (T == 0) return ORACLE_OK;
-    head_probs(qkv, T, C, C / n_head, b, h, P, NULL);
+    head_probs(qkv, T, C, C / n_head, window, b, h, P, NULL);
     return ORACLE_OK;
 }
 
-/* Backward: dqkv[B][T][3C] = d(sum y o dy)/d(qkv), by the chain rule through
- * the weighted sum, the row softmax and the scaled dot products. */
-int oracle_bwd(const double *qkv, const double *dy, int B, int T, int C, int n_head, double *dqkv) {
+int oracle_probs(const double *qkv, int B, int T, int C, int n_head, int b, int h, double *P) {
+    return oracle_probs_window(qkv, B, T, C, n_head, T > 0 ? T : 1, b, h, P);
+}
+
+/* Backward over a local window: dqkv[B][T][3C] = d(sum y o dy)/d(qkv), by the
+ * chain rule through the weighted sum, the row softmax and the scaled dot
+ * products.  window >= 1. */
+int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, int n_head, int window, double *dqkv) {
     int rc = check_shape(B, T, C, n_head);
     if (rc) return rc;
+    if (window < 1) return ORACLE_EINVAL;
     if (B == 0 || T == 0) return ORACLE_OK;
     const int hs = C / n_head;
     const double scale = 1.0 / sqrt((double)hs);
@@ -187,7 +213,7 @@ int oracle_bwd(const double *qkv, const double *dy, int B, int T, int C, int n_h
         for (int p = 0; p < pairs; ++p) {
             if (!P || !dS) continue;
             const int b = p / n_head, h = p % n_head;
-            head_probs(qkv, T, C, hs, b, h, P, NULL);
+            head_probs(qkv, T, C, hs, window, b, h, P, NULL);
             const double *dyb = dy + (size_t)b * (size_t)T * (size_t)C + (size_t)h * (size_t)hs;
             double *dq = dqkv + (size_t)b * (size_t)T * (size_t)(3 * C) + (size_t)h * (size_t)hs;
             double *dk = dq + C;
@@ -199,35 +225,40 @@ int oracle_bwd(const double *qkv, const double *dy, int B, int T, int C, int n_h
             for (int t = 0; t < T; ++t) {
                 const double *Pt = P + (size_t)t * (size_t)T;
                 double *dSt = dS + (size_t)t * (size_t)T;
+                const int lo = band_lo(t, window);
                 double rowdot = 0.0;
-                for (int s = 0; s <= t; ++s) {
+                for (int s = lo; s <= t; ++s) {
                     double acc = 0.0;
                     for (int d = 0; d < hs; ++d) acc += dyb[(size_t)t * ld_dy + d] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);
                     dSt[s] = acc;
                     rowdot += Pt[s] * acc;
                 }
-                for (int s = 0; s <= t; ++s) dSt[s] = Pt[s] * (dSt[s] - rowdot);
+                for (int s = lo; s <= t; ++s) dSt[s] = Pt[s] * (dSt[s] - rowdot);
+                for (int s = 0; s < lo; ++s) dSt[s] = 0.0;
                 for (int s = t + 1; s < T; ++s) dSt[s] = 0.0;
             }
-            /* dV[s] = sum_{t>=s} P[t][s] dy_t */
+            /* dV[s] = sum over the queries t that see s of P[t][s] dy_t */
             for (int s = 0; s < T; ++s)
                 for (int d = 0; d < hs; ++d) {
                     double acc = 0.0;
-                    for (int t = s; t < T; ++t) acc += P[(size_t)t * (size_t)T + s] * dyb[(size_t)t * ld_dy + d];
+                    for (int t = s; t <= band_hi(s, window, T); ++t)
+                        acc += P[(size_t)t * (size_t)T + s] * dyb[(size_t)t * ld_dy + d];
                     dv[(size_t)s * ld_dqkv + d] = acc;
                 }
-            /* dQ[t] = scale * sum_{s<=t} dS[t][s] k_s */
+            /* dQ[t] = scale * sum over the visible s of dS[t][s] k_s */
             for (int t = 0; t < T; ++t)
                 for (int d = 0; d < hs; ++d) {
                     double acc = 0.0;
-                    for (int s = 0; s <= t; ++s) acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);
+                    for (int s = band_lo(t, window); s <= t; ++s)
+                        acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);
                     dq[(size_t)t * ld_dqkv + d] = acc * scale;
                 }
-            /* dK[s] = scale * sum_{t>=s} dS[t][s] q_t */
+            /* dK[s] = scale * sum over the queries t that see s of dS[t][s] q_t */
             for (int s = 0; s < T; ++s)
                 for (int d = 0; d < hs; ++d) {
                     double acc = 0.0;
-                    for (int t = s; t < T; ++t) acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);
+                    for (int t = s; t <= band_hi(s, window, T); ++t)
+                        acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);
                     dk[(size_t)s * ld_dqkv + d] = acc * scale;
                 }
         }
@@ -235,4 +266,9 @@ int oracle_bwd(const double *qkv, const double *dy, int B, int T, int C, int n_h
         free(dS);
     }
     return err ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+/* Backward, causal (every past position visible). */
+int oracle_bwd(const double *qkv, const double *dy, int B, int T, int C, int n_head, double *dqkv) {
+    return oracle_bwd_window(qkv, dy, B, T, C, n_head, T > 0 ? T : 1, dqkv);
 }

@@ -8,7 +8,10 @@ fixture.  ``tests/test_oracle.py`` runs them against the real oracle;
 oracle and checks that every planted mistake trips at least one pin.
 
 Page cited throughout: "Let's build GPT: from scratch, in code, spelled out"
-(the lecture page with the chapter list and corrections).
+(the lecture page with the chapter list and corrections).  The local-window
+pins (``pin_window_*``) follow the minGPT README page's reference notes on
+GPT-3 (alternating dense and locally banded sparse attention), read as: token
+t sees positions t-window < s <= t.
 """
 from __future__ import annotations
 
@@ -288,10 +291,134 @@ def pin_empty(orc):
     assert g.shape == (2, 0, 12)
 
 
+# ---- local window (banded) attention ------------------------------------------
+
+def pin_window_one(orc):
+    """window = 1: each token sees only itself, so y = v exactly, lse = q.k/sqrt(hs),
+    and the backward is dV = dy, dQ = dK = 0 (the softmax of one element has zero
+    derivative)."""
+    B, T, n_head, hs = 2, 11, 2, 4
+    C = n_head * hs
+    r = _rng(30)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    y, lse = orc.forward(qkv, n_head, window=1)
+    assert np.array_equal(y, qkv[:, :, 2 * C:])
+    q, k, _ = _split(qkv, n_head)
+    assert np.allclose(lse, (q * k).sum(-1) / math.sqrt(hs), rtol=0, atol=1e-14)
+    g = orc.backward(qkv, dy, n_head, window=1)
+    assert np.allclose(g[:, :, 2 * C:], dy, rtol=0, atol=1e-15)
+    assert np.abs(g[:, :, :2 * C]).max() < 1e-15
+
+
+def pin_window_covers_all(orc):
+    """A window at least T wide hides nothing the causal mask does not: the
+    results equal the causal oracle's bit for bit."""
+    B, T, n_head, hs = 2, 13, 2, 3
+    C = n_head * hs
+    r = _rng(31)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    y0, l0 = orc.forward(qkv, n_head)
+    g0 = orc.backward(qkv, dy, n_head)
+    for w in (T, T + 5):
+        y, l = orc.forward(qkv, n_head, window=w)
+        assert np.array_equal(y, y0) and np.array_equal(l, l0)
+        assert np.array_equal(orc.backward(qkv, dy, n_head, window=w), g0)
+
+
+def pin_window_uniform_scores(orc):
+    """Zero queries: the weights are uniform over the band, so y[t] is the mean of
+    v over max(0, t-window+1)..t and lse[t] = ln(band size)."""
+    B, T, n_head, hs, w = 2, 17, 2, 3, 5
+    C = n_head * hs
+    qkv = _rng(32).standard_normal((B, T, 3 * C))
+    qkv[:, :, :C] = 0.0
+    y, lse = orc.forward(qkv, n_head, window=w)
+    v = qkv[:, :, 2 * C:]
+    for t in range(T):
+        lo = max(0, t - w + 1)
+        total = np.zeros((B, C))
+        for s in range(lo, t + 1):
+            total += v[:, s]
+        assert np.allclose(y[:, t], total / (t - lo + 1), rtol=0, atol=1e-14)
+        assert np.allclose(lse[:, :, t], math.log(t - lo + 1), rtol=0, atol=1e-14)
+
+
+def pin_window_locality(orc):
+    """Tokens before the band of position t (s <= t-window) do not reach it:
+    perturbing them leaves y[t], lse[t] bit-identical; perturbing a token inside
+    the band changes y[t]."""
+    B, T, n_head, hs, w = 1, 16, 2, 4, 4
+    C = n_head * hs
+    r = _rng(33)
+    qkv = r.standard_normal((B, T, 3 * C))
+    y0, l0 = orc.forward(qkv, n_head, window=w)
+    t = 12
+    q2 = qkv.copy()
+    q2[:, :t - w + 1] += r.standard_normal(q2[:, :t - w + 1].shape)
+    y1, l1 = orc.forward(q2, n_head, window=w)
+    assert np.array_equal(y1[:, t], y0[:, t]) and np.array_equal(l1[:, :, t], l0[:, :, t])
+    q3 = qkv.copy()
+    q3[:, t - w + 1] += 1.0
+    y2, _ = orc.forward(q3, n_head, window=w)
+    assert not np.allclose(y2[:, t], y0[:, t])
+
+
+def pin_window_library_special_case(orc):
+    """A different implementation: PyTorch scaled_dot_product_attention with an
+    explicit boolean band mask, and autograd, in fp64 on the CPU."""
+    B, T, n_head, hs, w = 2, 29, 2, 8, 7
+    C = n_head * hs
+    r = _rng(34)
+    qkv = r.standard_normal((B, T, 3 * C))
+    dy = r.standard_normal((B, T, C))
+    x = torch.tensor(qkv, dtype=torch.float64, requires_grad=True)
+    q, k, v = x.split(C, dim=2)
+    heads = lambda a: a.view(B, T, n_head, hs).transpose(1, 2)
+    tt = torch.arange(T)
+    band = (tt[None, :] <= tt[:, None]) & (tt[None, :] > tt[:, None] - w)   # [t, s] visible
+    out = torch.nn.functional.scaled_dot_product_attention(heads(q), heads(k), heads(v), attn_mask=band)
+    y_ref = out.transpose(1, 2).reshape(B, T, C)
+    (y_ref * torch.tensor(dy)).sum().backward()
+    y, lse = orc.forward(qkv, n_head, window=w)
+    g = orc.backward(qkv, dy, n_head, window=w)
+    assert np.abs(y - y_ref.detach().numpy()).max() < 1e-12
+    assert np.abs(g - x.grad.numpy()).max() < 1e-12
+    s = heads(q).detach() @ heads(k).detach().transpose(-1, -2) / math.sqrt(hs)
+    s = s.masked_fill(~band, float("-inf"))
+    assert np.abs(lse - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+def pin_window_finite_differences(orc):
+    """The windowed backward is the gradient of sum(y * dy): central differences."""
+    B, T, n_head, hs, w = 1, 7, 2, 3, 3
+    C = n_head * hs
+    r = _rng(35)
+    qkv = r.standard_normal((B, T, 3 * C))
+    G = r.standard_normal((B, T, C))
+    grad = orc.backward(qkv, G, n_head, window=w)
+    h = 1e-6
+    fd = np.zeros_like(qkv)
+    flat = qkv.reshape(-1)
+    for i in range(flat.size):
+        xp = flat.copy()
+        xm = flat.copy()
+        xp[i] += h
+        xm[i] -= h
+        yp, _ = orc.forward(xp.reshape(qkv.shape), n_head, window=w)
+        ym, _ = orc.forward(xm.reshape(qkv.shape), n_head, window=w)
+        fd.reshape(-1)[i] = ((yp * G).sum() - (ym * G).sum()) / (2 * h)
+    err = np.abs(fd - grad).max() / np.abs(grad).max()
+    assert err < 1e-6, f"finite-difference mismatch {err:.3e}"
+
+
 ALL_PINS = [
     pin_single_token, pin_uniform_scores_prefix_mean, pin_tril_average_fixture,
     pin_rows_are_distributions, pin_weights_from_softmax_of_scaled_scores,
     pin_worked_two_heads, pin_causality, pin_batch_independence, pin_head_permutation,
     pin_set_semantics, pin_finite_differences, pin_library_special_case,
     pin_regression_fixture, pin_empty,
+    pin_window_one, pin_window_covers_all, pin_window_uniform_scores, pin_window_locality,
+    pin_window_library_special_case, pin_window_finite_differences,
 ]

@@ -34,6 +34,9 @@ MUTANTS = [
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);",
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 0, h, d);"),
     ("dK_missing_scale", "dk[(size_t)s * ld_dqkv + d] = acc * scale;", "dk[(size_t)s * ld_dqkv + d] = acc;"),
+    ("band_one_key_too_many", "return t - window + 1 > 0 ? t - window + 1 : 0;", "return t - window > 0 ? t - window : 0;"),
+    ("band_last_query_dropped", "return s + window - 1 < T - 1 ? s + window - 1 : T - 1;",
+     "return s + window - 2 < T - 1 ? s + window - 2 : T - 1;"),
     ("dK_transposed_dS",
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);",
      "acc += dS[(size_t)s * (size_t)T + t] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);"),
