@@ -236,6 +236,111 @@ cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s) {
 
 using namespace gptattn;
 
+namespace {
+// Shape checks shared by the windowed entry points: window >= 1; a window
+// narrower than T needs the head-size-64 kernels on the bf16 path.  Returns the
+// window the kernels get (kCausalWindow when nothing is cut).
+gptattn_status check_window(int window, int T, int hs, gptattn_dtype dt, int *kernel_window) {
+    if (window < 1) return GPTATTN_ERR_INVALID_ARG;
+    if (window >= T) {
+        *kernel_window = kCausalWindow;
+        return GPTATTN_OK;
+    }
+    if (dt == GPTATTN_BF16 && hs != 64) return GPTATTN_ERR_UNSUPPORTED;
+    *kernel_window = window;
+    return GPTATTN_OK;
+}
+
+gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, int window,
+                        gptattn_dtype dt, gptattn_stream_t stream) {
+    int hs = 0;
+    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
+    if (st != GPTATTN_OK) return st;
+    int kw = kCausalWindow;
+    st = check_window(window, T, hs, dt, &kw);
+    if (st != GPTATTN_OK) return st;
+    if (B == 0 || T == 0) return GPTATTN_OK;
+    if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    if (dt == GPTATTN_F32) {
+        return from_cuda(run_kernel(kKFwdF32, s, [&] {
+            return launch_fwd_f32(hs, static_cast<const float *>(qkv), static_cast<float *>(y), lse, B, T, C, n_head, kw,
+                                  s);
+        }));
+    }
+    int *status = nullptr;
+    cudaError_t e = status_ptr(&status);
+    if (e != cudaSuccess) return GPTATTN_ERR_CUDA;
+    CUtensorMap mq, my;
+    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&my, y, C, T, B)) return GPTATTN_ERR_CUDA;
+    const DevCtx ctx{status, kDefaultBudgetNs};
+    return from_cuda(
+        run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, kw, ctx, s); }));
+}
+}  // namespace
+
+namespace {
+gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv, void *workspace,
+                        size_t workspace_bytes, int B, int T, int C, int n_head, int window, gptattn_dtype dt,
+                        gptattn_stream_t stream) {
+    int hs = 0;
+    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
+    if (st != GPTATTN_OK) return st;
+    int kw = kCausalWindow;
+    st = check_window(window, T, hs, dt, &kw);
+    if (st != GPTATTN_OK) return st;
+    if (B == 0 || T == 0) return GPTATTN_OK;
+    if (!qkv || !y || !lse || !dy || !dqkv) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse) || !aligned16(dy) || !aligned16(dqkv))
+        return GPTATTN_ERR_INVALID_ARG;
+    const BwdWorkspace w = workspace_layout(B, T, n_head, hs, dt);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < w.total)
+        return GPTATTN_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+
+    if (dt == GPTATTN_F32) {
+        const float *fq = static_cast<const float *>(qkv);
+        const float *fy = static_cast<const float *>(y);
+        const float *fg = static_cast<const float *>(dy);
+        float *fo = static_cast<float *>(dqkv);
+        float *D = reinterpret_cast<float *>(ws + w.D);
+        cudaError_t e = run_kernel(kKBwdPreF32, s, [&] { return launch_bwd_f32_pre(hs, fy, fg, D, B, T, C, n_head, s); });
+        if (e == cudaSuccess)
+            e = run_kernel(kKBwdDqF32, s,
+                           [&] { return launch_bwd_f32_dq(hs, fq, fg, lse, D, fo, B, T, C, n_head, kw, s); });
+        if (e == cudaSuccess)
+            e = run_kernel(kKBwdDkvF32, s,
+                           [&] { return launch_bwd_f32_dkv(hs, fq, fg, lse, D, fo, B, T, C, n_head, kw, s); });
+        return from_cuda(e);
+    }
+
+    int *status = nullptr;
+    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    const int T_pad = padded_T(T);
+    float *D = reinterpret_cast<float *>(ws + w.D);
+    float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
+    float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
+    CUtensorMap mq, mdy, mdqkv, mdq;
+    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&mdy, dy, C, T, B) ||
+        !map_bf16_rows(&mdqkv, dqkv, 3 * C, T, B) || !map_f32_acc(&mdq, dqacc, hs, (long long)B * n_head * T_pad))
+        return GPTATTN_ERR_CUDA;
+    const DevCtx ctx{status, kDefaultBudgetNs};
+    cudaError_t e = run_kernel(kKBwdPreBf16, s, [&] {
+        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, s);
+    });
+    if (e == cudaSuccess)
+        e = run_kernel(kKBwdMainBf16, s, [&] {
+            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, kw, ctx, s);
+        });
+    if (e == cudaSuccess)
+        e = run_kernel(kKBwdPostBf16, s, [&] { return launch_bwd_post_bf16(hs, dqacc, dqkv, B, T, C, n_head, T_pad, s); });
+    return from_cuda(e);
+}
+}  // namespace
+
 extern "C" {
 
 const char *gptattn_status_string(gptattn_status s) {
@@ -254,28 +359,15 @@ int gptattn_version(void) { return 100; }
 
 const char *gptattn_last_error_string(void) { return t_last_error; }
 
+
 gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, gptattn_dtype dt,
                            gptattn_stream_t stream) {
-    int hs = 0;
-    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
-    if (st != GPTATTN_OK) return st;
-    if (B == 0 || T == 0) return GPTATTN_OK;
-    if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
-    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return fwd_impl(qkv, y, lse, B, T, C, n_head, kCausalWindow, dt, stream);
+}
 
-    if (dt == GPTATTN_F32) {
-        return from_cuda(run_kernel(kKFwdF32, s, [&] {
-            return launch_fwd_f32(hs, static_cast<const float *>(qkv), static_cast<float *>(y), lse, B, T, C, n_head, s);
-        }));
-    }
-    int *status = nullptr;
-    cudaError_t e = status_ptr(&status);
-    if (e != cudaSuccess) return GPTATTN_ERR_CUDA;
-    CUtensorMap mq, my;
-    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&my, y, C, T, B)) return GPTATTN_ERR_CUDA;
-    const DevCtx ctx{status, kDefaultBudgetNs};
-    return from_cuda(run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, ctx, s); }));
+gptattn_status gptattn_fwd_window(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, int window,
+                                  gptattn_dtype dt, gptattn_stream_t stream) {
+    return fwd_impl(qkv, y, lse, B, T, C, n_head, window, dt, stream);
 }
 
 gptattn_status gptattn_decode(const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C, int n_head,
@@ -301,57 +393,17 @@ size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtyp
     return workspace_layout(B, T, n_head, hs, dt).total;
 }
 
+
 gptattn_status gptattn_bwd(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
                            void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, gptattn_dtype dt,
                            gptattn_stream_t stream) {
-    int hs = 0;
-    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
-    if (st != GPTATTN_OK) return st;
-    if (B == 0 || T == 0) return GPTATTN_OK;
-    if (!qkv || !y || !lse || !dy || !dqkv) return GPTATTN_ERR_INVALID_ARG;
-    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse) || !aligned16(dy) || !aligned16(dqkv))
-        return GPTATTN_ERR_INVALID_ARG;
-    const BwdWorkspace w = workspace_layout(B, T, n_head, hs, dt);
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < w.total)
-        return GPTATTN_ERR_WORKSPACE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    char *ws = static_cast<char *>(workspace);
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, kCausalWindow, dt, stream);
+}
 
-    if (dt == GPTATTN_F32) {
-        const float *fq = static_cast<const float *>(qkv);
-        const float *fy = static_cast<const float *>(y);
-        const float *fg = static_cast<const float *>(dy);
-        float *fo = static_cast<float *>(dqkv);
-        float *D = reinterpret_cast<float *>(ws + w.D);
-        cudaError_t e = run_kernel(kKBwdPreF32, s, [&] { return launch_bwd_f32_pre(hs, fy, fg, D, B, T, C, n_head, s); });
-        if (e == cudaSuccess)
-            e = run_kernel(kKBwdDqF32, s, [&] { return launch_bwd_f32_dq(hs, fq, fg, lse, D, fo, B, T, C, n_head, s); });
-        if (e == cudaSuccess)
-            e = run_kernel(kKBwdDkvF32, s, [&] { return launch_bwd_f32_dkv(hs, fq, fg, lse, D, fo, B, T, C, n_head, s); });
-        return from_cuda(e);
-    }
-
-    int *status = nullptr;
-    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
-    const int T_pad = padded_T(T);
-    float *D = reinterpret_cast<float *>(ws + w.D);
-    float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
-    float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
-    CUtensorMap mq, mdy, mdqkv, mdq;
-    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&mdy, dy, C, T, B) ||
-        !map_bf16_rows(&mdqkv, dqkv, 3 * C, T, B) || !map_f32_acc(&mdq, dqacc, hs, (long long)B * n_head * T_pad))
-        return GPTATTN_ERR_CUDA;
-    const DevCtx ctx{status, kDefaultBudgetNs};
-    cudaError_t e = run_kernel(kKBwdPreBf16, s, [&] {
-        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, s);
-    });
-    if (e == cudaSuccess)
-        e = run_kernel(kKBwdMainBf16, s, [&] {
-            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
-        });
-    if (e == cudaSuccess)
-        e = run_kernel(kKBwdPostBf16, s, [&] { return launch_bwd_post_bf16(hs, dqacc, dqkv, B, T, C, n_head, T_pad, s); });
-    return from_cuda(e);
+gptattn_status gptattn_bwd_window(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
+                                  void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, int window,
+                                  gptattn_dtype dt, gptattn_stream_t stream) {
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, dt, stream);
 }
 
 gptattn_status gptattn_get_device_status(gptattn_stream_t stream) {

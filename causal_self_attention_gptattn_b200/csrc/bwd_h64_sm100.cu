@@ -6,6 +6,10 @@
 // logsumexp):  dV += P^T dY,  dP = dY V^T,  dS = P o (dP - D),
 //              dK += dS^T Q * scale,  dQ += dS K * scale.
 // The workspace rows hold -D and -lse*log2(e) (negated by the preprocess kernel).
+// Local window (minGPT README page, reference notes on GPT-3: locally banded
+// attention): key s is seen by queries s <= t < s + window, so a key tile's
+// item stops at the last query tile its band reaches and the band's far edge
+// is masked element-wise like the diagonal.  window >= T is the causal case.
 //
 // Schedule: one persistent CTA per SM walks a static list of work items
 // (key tile j, batch b, head h), ordered longest first (small j first), in a
@@ -93,6 +97,12 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
+// Last query tile that key tile kt's band reaches.
+__device__ __forceinline__ int band_hi_tile(int kt, int window, int n_t) {
+    const long long t = (long long)kt * kTile + kTile - 2 + window;  // largest key + window - 1
+    return t / kTile < n_t ? (int)(t / kTile) : n_t - 1;
+}
+
 __device__ __forceinline__ int item_index(int k, int cta, int grid) {
     return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
 }
@@ -101,7 +111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_h64_persistent(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
                        const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
                        const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C,
-                       int n_head, int T_pad, int n_t, int *status, unsigned long long budget_ns) {
+                       int n_head, int T_pad, int n_t, int window, int *status, unsigned long long budget_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -180,7 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(bar(kBarKVFull + kvs), 2 * kTileBytes);
                 tma_load_3d(sK(kvs), &map_qkv, bar(kBarKVFull + kvs), C + h * HS, kt * kTile, b);
                 tma_load_3d(sV(kvs), &map_qkv, bar(kBarKVFull + kvs), 2 * C + h * HS, kt * kTile, b);
-                for (int qt = kt; qt < n_t; ++qt, ++gq) {
+                const int qt_end = band_hi_tile(kt, window, n_t);
+                for (int qt = kt; qt <= qt_end; ++qt, ++gq) {
                     const int st = gq % kQStages;
                     const uint32_t ph = (uint32_t)(gq / kQStages) & 1u;
                     if (gq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + st), ph ^ 1u, g))) break;
@@ -236,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int w = item_index(k, blockIdx.x, gridDim.x);
                 if (w >= n_items) break;
                 const int kt = w / BH;
-                const int niter = n_t - kt;
+                const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
                 const int kvs = n & 1;
                 if (!(ok = mbar_wait(bar(kBarKVFull + kvs), (uint32_t)(n >> 1) & 1u, g))) break;
                 // first S and dP of this item
@@ -322,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int w = item_index(k, blockIdx.x, gridDim.x);
             if (w >= n_items) break;
             const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
-            const int niter = n_t - kt;
+            const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
             for (int it = 0; it < niter; ++it, ++gi) {
                 const int st = gi % kQStages;
                 const uint32_t ph = (uint32_t)gi & 1u;
@@ -357,6 +368,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < 64; ++c)
                             if (64 * half + c < row) pf[c] = 0.f;
+                    }
+                    if (it * kTile + kTile - 1 >= window) {  // band's far edge: t sees s only if t - s < window
+                        const int cut = window + row - it * kTile - 64 * half;  // columns c >= cut are masked
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (c >= cut) pf[c] = 0.f;
                     }
                     uint32_t pk[32];
 #pragma unroll
@@ -458,7 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int w = item_index(k, blockIdx.x, gridDim.x);
             if (w >= n_items) break;
             const int kt = w / BH, bh = w % BH;
-            for (int qt = kt; qt < n_t; ++qt, ++gi) {
+            const int qt_end = band_hi_tile(kt, window, n_t);
+            for (int qt = kt; qt <= qt_end; ++qt, ++gi) {
                 if (ok) ok = warp_wait(bar(kBardQFull), (uint32_t)gi & 1u, g);
                 uint32_t v[64];
                 if (ok) {
@@ -503,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                                int n_head, int T_pad, DevCtx ctx, cudaStream_t s) {
+                                int n_head, int T_pad, int window, DevCtx ctx, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(bwd_h64_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -515,7 +533,7 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
     const long long items = (long long)n_t * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
     return launch_pdl(bwd_h64_persistent, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_dy, map_dqkv,
-                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
+                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

@@ -18,6 +18,10 @@
 //     S_A(j+1)  S_B(j+1)  PV_A(j)  PV_B(j)
 // Lazy rescaling (O is rescaled only when a row max grows by more than 2^8)
 // and y normalised by the sum of the bf16-rounded weights, as in fwd_sm100.cu.
+// Local window (minGPT README page, reference notes on GPT-3: locally banded
+// attention): query t sees keys t-window < s <= t; key tiles below a query
+// tile's band are skipped, and the band's lower edge is masked element-wise
+// like the diagonal.  window >= T is the causal case.
 // Every barrier wait is bounded; on a timeout all roles stop, drain and exit.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -66,13 +70,19 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
+// First key tile that query tile qt's band reaches.
+__device__ __forceinline__ int band_lo_tile(int qt, int window) {
+    const int s = qt * kTile - window + 1;
+    return s > 0 ? s / kTile : 0;
+}
+
 __device__ __forceinline__ int item_index(int k, int cta, int grid) {
     return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_h64_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
-                   float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int *status,
+                   float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, int *status,
                    unsigned long long budget_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -146,7 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode(w, m, bh);
                 const int b = bh / n_head, h = bh % n_head;
                 const bool hasB = 2 * m + 1 < n_qt;
-                const int nkv = hasB ? 2 * m + 2 : 2 * m + 1;
+                const int jlo = band_lo_tile(2 * m, window);
+                const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
                 const int qs = nq % kQStages;
                 if (nq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + qs), (uint32_t)((nq / kQStages) & 1) ^ 1u, g)))
                     break;
@@ -160,9 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (uint32_t)(gkv / kKVStages) & 1u;
                     if (gkv >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + st), ph ^ 1u, g))) break;
                     mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
-                    tma_load_3d(sK(st), &map_qkv, bar(kBarKFull + st), C + h * HS, j * kTile, b);
+                    tma_load_3d(sK(st), &map_qkv, bar(kBarKFull + st), C + h * HS, (jlo + j) * kTile, b);
                     mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
-                    tma_load_3d(sV(st), &map_qkv, bar(kBarVFull + st), 2 * C + h * HS, j * kTile, b);
+                    tma_load_3d(sV(st), &map_qkv, bar(kBarVFull + st), 2 * C + h * HS, (jlo + j) * kTile, b);
                     ++gkv;
                 }
             }
@@ -213,13 +224,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int m, bh;
                 decode(w, m, bh);
                 const bool hasB = 2 * m + 1 < n_qt;
-                const int nt[2] = {2 * m + 1, hasB ? 2 * m + 2 : 0};
-                const int nkv = hasB ? nt[1] : nt[0];
+                // key tiles of each stream: [lo, hi]; the item walks their union [jlo, jlo + nkv)
+                const int lo[2] = {band_lo_tile(2 * m, window), hasB ? band_lo_tile(2 * m + 1, window) : 1};
+                const int hi[2] = {2 * m, hasB ? 2 * m + 1 : 0};
+                const int jlo = lo[0];
+                const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
+                auto part = [&](int t, int j) { return j >= lo[t] && j <= hi[t]; };
                 const int qs = n % kQStages;
                 if (!(ok = mbar_wait(bar(kBarQFull + qs), (uint32_t)(n / kQStages) & 1u, g))) break;
                 if (!(ok = mbar_wait(bar(kBarKFull + gkv % kKVStages), (uint32_t)(gkv / kKVStages) & 1u, g))) break;
                 for (int t = 0; t < 2 && ok; ++t) {
-                    if (nt[t] == 0) continue;
+                    if (!part(t, jlo)) continue;
                     if (sc[t] > 0 && !(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
                     tc_fence_after();
                     issue_S(qs, t, gkv % kKVStages);
@@ -232,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int st1 = (gkv + j + 1) % kKVStages;
                         if (!(ok = mbar_wait(bar(kBarKFull + st1), (uint32_t)((gkv + j + 1) / kKVStages) & 1u, g))) break;
                         for (int t = 0; t < 2 && ok; ++t) {
-                            if (j + 1 >= nt[t]) continue;
+                            if (!part(t, jlo + j + 1)) continue;
                             if (!(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
                             tc_fence_after();
                             issue_S(qs, t, st1);
@@ -242,13 +257,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // P V of key tile j for each stream
                     if (!(ok = mbar_wait(bar(kBarVFull + st), (uint32_t)((gkv + j) / kKVStages) & 1u, g))) break;
                     for (int t = 0; t < 2 && ok; ++t) {
-                        if (j >= nt[t]) continue;
+                        if (!part(t, jlo + j)) continue;
                         if (!(ok = mbar_wait(bar(kBarPFull + t), (uint32_t)pc[t] & 1u, g))) break;
-                        if (j == 0 && items[t] > 0 &&
+                        if (jlo + j == lo[t] && items[t] > 0 &&
                             !(ok = mbar_wait(bar(kBarOFree + t), (uint32_t)(items[t] - 1) & 1u, g)))
                             break;
                         tc_fence_after();
-                        issue_PV(t, st, j == 0);
+                        issue_PV(t, st, jlo + j == lo[t]);
                     }
                     if (ok) umma_commit(bar(kBarKVEmpty + st));
                 }
@@ -287,9 +302,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (leader) mbar_arrive(bar(kBarQEmpty + qs));
                 continue;
             }
-            const int ntile = qt + 1;
+            const int jlo_t = band_lo_tile(qt, window);
+            // key tiles at or below this one need the band's lower edge masked
+            const int j_edge = (qt * kTile + kTile - 1 - window) / kTile;
             float mrow = -INFINITY, l = 0.f, l_r = 0.f;
-            for (int j = 0; j < ntile; ++j, ++it) {
+            for (int j = jlo_t; j <= qt; ++j, ++it) {
                 if (ok) ok = warp_wait(bar(kBarSFull + t), (uint32_t)it & 1u, g);
                 if (!ok) continue;
                 tc_fence_after();
@@ -304,6 +321,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 128; ++c)
                         if (c > row) sr[c] = __float_as_uint(-INFINITY);
+                }
+                if (j <= j_edge && qt * kTile + kTile - 1 - window >= 0) {  // key s visible only if s > t - window
+                    const int cut = (qt - j) * kTile + row - window;       // columns c <= cut are masked
+#pragma unroll
+                    for (int c = 0; c < 128; ++c)
+                        if (c <= cut) sr[c] = __float_as_uint(-INFINITY);
                 }
                 float mp[4];
 #pragma unroll
@@ -320,7 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool grow = m_cand > mrow + 8.f;
                 const float m_new = grow ? m_cand : mrow;
                 const float alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
-                const uint64_t negm2 = f32x2_pack(-m_new, -m_new);
+                // a row with no visible key yet (band edge) keeps weight 0, not NaN
+                const float m_use = m_new == -INFINITY ? 0.f : m_new;
+                const uint64_t negm2 = f32x2_pack(-m_use, -m_use);
                 // four independent partial sums each, so the adds do not form one long chain
                 uint64_t sum2[4], sumr2[4];
 #pragma unroll
@@ -345,14 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l_r = l_r * alpha + (r0 + r1);
                 mrow = m_new;
                 // P buffer and O are free once the previous P V of this stream retired
-                if (j > 0) {
+                if (j > jlo_t) {
                     ok = warp_wait(bar(kBarPVDone + t), (uint32_t)(it - 1) & 1u, g);
                     if (!ok) continue;
                     tc_fence_after();
                 }
                 tmem_st_x32(tP + 0, *reinterpret_cast<const uint32_t(*)[32]>(&pk[0]));
                 tmem_st_x32(tP + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32]));
-                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (j > jlo_t && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
                     for (int c0 = 0; c0 < HS; c0 += 32) {
                         uint32_t o[32];
@@ -415,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
-                           int n_head, DevCtx ctx, cudaStream_t s) {
+                           int n_head, int window, DevCtx ctx, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(fwd_h64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -426,7 +451,7 @@ cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y,
     const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
     return launch_pdl(fwd_h64_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_y, lse, B, T, C,
-                      n_head, n_qt, ctx.status, ctx.budget_ns);
+                      n_head, n_qt, window, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

@@ -21,6 +21,10 @@ constexpr int kTile = 128;
 
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// The window the causal entry points pass: wider than any sequence, so no band
+// edge ever falls inside a tile.
+constexpr int kCausalWindow = 1 << 30;
+
 // Launch with programmatic stream serialisation: the kernel's CTAs may start
 // (and run their prologue) while the previous kernel of the stream finishes;
 // every kernel launched this way calls griddep_wait() before touching global
@@ -44,12 +48,14 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // ---- bf16 tensor-core path (sm_100a) --------------------------------------
 // map_qkv: 3-D view (3C, T, B) of qkv, box (64, 128, 1), 128-byte swizzle.
 // map_y:   3-D view (C, T, B) of y, same box.
+// window: query t sees keys t-window < s <= t (kCausalWindow or any value >= T: causal);
+// the head-size-128 kernels support the causal case only.
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse,
-                            int B, int T, int C, int n_head, DevCtx ctx, cudaStream_t s);
+                            int B, int T, int C, int n_head, int window, DevCtx ctx, cudaStream_t s);
 
 // Head-size-64 forward with separate P buffers (same arguments as above).
 cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
-                           int n_head, DevCtx ctx, cudaStream_t s);
+                           int n_head, int window, DevCtx ctx, cudaStream_t s);
 
 // D[bh][t] = sum_d y*dy, lse2[bh][t] = lse*log2(e) (rows t >= T: 0 and +inf),
 // dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].
@@ -60,27 +66,27 @@ cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const flo
 // map_dq: 2-D view (hs, B*n_head*T_pad) of dqacc (fp32), box (32, 128), 128-byte swizzle.
 cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
                                  const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
-                                 const float *D, int B, int T, int C, int n_head, int T_pad, DevCtx ctx,
+                                 const float *D, int B, int T, int C, int n_head, int T_pad, int window, DevCtx ctx,
                                  cudaStream_t s);
 
 // Persistent head-size-64 variant of the above (same arguments).
 cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                                int n_head, int T_pad, DevCtx ctx, cudaStream_t s);
+                                int n_head, int T_pad, int window, DevCtx ctx, cudaStream_t s);
 
 // dqkv[b][t][h*hs+d] = bf16(dqacc[(b*n_head+h)*T_pad + t][d] / sqrt(hs)).
 cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head,
                                  int T_pad, cudaStream_t s);
 
 // ---- fp32 CUDA-core path --------------------------------------------------
-cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head,
+cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,
                            cudaStream_t s);
 cudaError_t launch_bwd_f32_pre(int hs, const float *y, const float *dy, float *D, int B, int T, int C,
                                int n_head, cudaStream_t s);
 cudaError_t launch_bwd_f32_dq(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
-                              float *dqkv, int B, int T, int C, int n_head, cudaStream_t s);
+                              float *dqkv, int B, int T, int C, int n_head, int window, cudaStream_t s);
 cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
-                               float *dqkv, int B, int T, int C, int n_head, cudaStream_t s);
+                               float *dqkv, int B, int T, int C, int n_head, int window, cudaStream_t s);
 
 // ---- decode: last position over a key/value cache (cluster of 8 CTAs per (b, h))
 cudaError_t launch_decode(int hs, bool bf16, const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C,

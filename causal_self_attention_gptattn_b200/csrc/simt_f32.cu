@@ -3,7 +3,10 @@
 // Same function as the bf16 tensor-core path (lecture page "Let's build GPT:
 // from scratch, in code, spelled out": "version 4: self-attention", causal
 // mask per correction 00:57:00, 1/sqrt(head_size) per correction 01:20:05),
-// kept in full fp32 (no TF32) for callers that need fp32 accuracy.  Every
+// kept in full fp32 (no TF32) for callers that need fp32 accuracy.  A local
+// window (token t sees t-window < s <= t; minGPT README page, reference notes
+// on GPT-3: locally banded attention) narrows every key or query range; the
+// causal case passes window = T.  Every
 // thread owns one query row (forward, dQ) or one key row (dK/dV); key or query
 // rows are staged through shared memory in tiles of kRows.  Deterministic: no
 // atomics.  Accurate expf/logf (no approximate intrinsics).
@@ -25,7 +28,7 @@ __device__ __forceinline__ float dot_row(const float *a, const float *b) {
 // y[b,t,h*HS+d] and lse[b,h,t] for query rows of one (b, h).
 template <int HS>
 __global__ void __launch_bounds__(kRows) fwd_f32_kernel(const float *__restrict__ qkv, float *__restrict__ y,
-                                                        float *__restrict__ lse, int T, int C, int n_head) {
+                                                        float *__restrict__ lse, int T, int C, int n_head, int window) {
     extern __shared__ float sm[];
     float *sk = sm;              // [kRows][HS]
     float *sv = sm + kRows * HS;  // [kRows][HS]
@@ -46,7 +49,9 @@ __global__ void __launch_bounds__(kRows) fwd_f32_kernel(const float *__restrict_
     float m = -INFINITY, l = 0.f;
 
     const int last = min(T - 1, (int)(blockIdx.x * kRows + kRows - 1));  // largest query row of the block
-    for (int s0 = 0; s0 <= last; s0 += kRows) {
+    const int lo_t = max(0, t - window + 1);                              // first key this row sees
+    const int lo_blk = max(0, (int)(blockIdx.x * kRows) - window + 1);    // first key any row of the block sees
+    for (int s0 = lo_blk / kRows * kRows; s0 <= last; s0 += kRows) {
         __syncthreads();
         for (int e = threadIdx.x; e < kRows * HS; e += kRows) {
             const int r = e / HS, d = e % HS;
@@ -56,8 +61,8 @@ __global__ void __launch_bounds__(kRows) fwd_f32_kernel(const float *__restrict_
         }
         __syncthreads();
         if (t < T) {
-            const int smax = min(kRows, t - s0 + 1);  // visible keys in this tile: s <= t
-            for (int r = 0; r < smax; ++r) {
+            const int smax = min(kRows, t - s0 + 1);  // visible keys in this tile: lo_t <= s <= t
+            for (int r = max(0, lo_t - s0); r < smax; ++r) {
                 const float sc = dot_row<HS>(q, sk + r * HS);
                 const float m_new = fmaxf(m, sc);
                 const float corr = expf(m - m_new);
@@ -101,7 +106,8 @@ __global__ void bwd_f32_pre_kernel(const float *__restrict__ y, const float *__r
 template <int HS>
 __global__ void __launch_bounds__(kRows) bwd_f32_dq_kernel(const float *__restrict__ qkv, const float *__restrict__ dy,
                                                            const float *__restrict__ lse, const float *__restrict__ D,
-                                                           float *__restrict__ dqkv, int T, int C, int n_head) {
+                                                           float *__restrict__ dqkv, int T, int C, int n_head,
+                                                           int window) {
     extern __shared__ float sm[];
     float *sk = sm;
     float *sv = sm + kRows * HS;
@@ -128,7 +134,9 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dq_kernel(const float *__restri
     for (int d = 0; d < HS; ++d) acc[d] = 0.f;
 
     const int last = min(T - 1, (int)(blockIdx.x * kRows + kRows - 1));
-    for (int s0 = 0; s0 <= last; s0 += kRows) {
+    const int lo_t = max(0, t - window + 1);
+    const int lo_blk = max(0, (int)(blockIdx.x * kRows) - window + 1);
+    for (int s0 = lo_blk / kRows * kRows; s0 <= last; s0 += kRows) {
         __syncthreads();
         for (int e = threadIdx.x; e < kRows * HS; e += kRows) {
             const int r = e / HS, d = e % HS;
@@ -139,7 +147,7 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dq_kernel(const float *__restri
         __syncthreads();
         if (t < T) {
             const int smax = min(kRows, t - s0 + 1);
-            for (int r = 0; r < smax; ++r) {
+            for (int r = max(0, lo_t - s0); r < smax; ++r) {
                 const float p = expf(dot_row<HS>(q, sk + r * HS) - lse_t);
                 const float ds = p * (dot_row<HS>(g, sv + r * HS) - D_t);
 #pragma unroll
@@ -158,7 +166,8 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dq_kernel(const float *__restri
 template <int HS>
 __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restrict__ qkv, const float *__restrict__ dy,
                                                             const float *__restrict__ lse, const float *__restrict__ D,
-                                                            float *__restrict__ dqkv, int T, int C, int n_head) {
+                                                            float *__restrict__ dqkv, int T, int C, int n_head,
+                                                            int window) {
     extern __shared__ float sm[];
     float *sq = sm;                   // [kRows][HS] queries (pre-scaled)
     float *sg = sm + kRows * HS;      // [kRows][HS] dy rows
@@ -184,7 +193,9 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restr
     for (int d = 0; d < HS; ++d) dk[d] = dv[d] = 0.f;
 
     const int first = blockIdx.x * kRows;  // smallest key row of the block
-    for (int t0 = first; t0 < T; t0 += kRows) {
+    // last query that sees any key of the block: (largest key row) + window - 1
+    const int t_end = min(T, (int)min((long long)first + kRows - 1 + window, (long long)T));
+    for (int t0 = first; t0 < t_end; t0 += kRows) {
         __syncthreads();
         for (int e = threadIdx.x; e < kRows * HS; e += kRows) {
             const int r = e / HS, d = e % HS;
@@ -199,8 +210,8 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restr
         }
         __syncthreads();
         if (s < T) {
-            const int rmin = max(0, s - t0);          // queries t >= s
-            const int rmax = min(kRows, T - t0);
+            const int rmin = max(0, s - t0);                                       // queries t >= s
+            const int rmax = (int)min((long long)min(kRows, T - t0), (long long)s + window - t0);  // t < s + window
             for (int r = rmin; r < rmax; ++r) {
                 const float p = expf(dot_row<HS>(sq + r * HS, k) - sl[r]);
                 const float ds = p * (dot_row<HS>(sg + r * HS, v) - sD[r]);
@@ -223,30 +234,31 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restr
 }
 
 template <int HS>
-cudaError_t launch_fwd_t(const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, cudaStream_t s) {
+cudaError_t launch_fwd_t(const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,
+                         cudaStream_t s) {
     const size_t smem = 2 * kRows * HS * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fwd_f32_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, y, lse, T, C, n_head);
+    fwd_f32_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, y, lse, T, C, n_head, window);
     return cudaGetLastError();
 }
 template <int HS>
 cudaError_t launch_dq_t(const float *qkv, const float *dy, const float *lse, const float *D, float *dqkv, int B, int T,
-                        int C, int n_head, cudaStream_t s) {
+                        int C, int n_head, int window, cudaStream_t s) {
     const size_t smem = 2 * kRows * HS * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_f32_dq_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_f32_dq_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, dy, lse, D, dqkv, T, C, n_head);
+    bwd_f32_dq_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, dy, lse, D, dqkv, T, C, n_head, window);
     return cudaGetLastError();
 }
 template <int HS>
 cudaError_t launch_dkv_t(const float *qkv, const float *dy, const float *lse, const float *D, float *dqkv, int B, int T,
-                         int C, int n_head, cudaStream_t s) {
+                         int C, int n_head, int window, cudaStream_t s) {
     const size_t smem = (2 * kRows * HS + 2 * kRows) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_f32_dkv_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bwd_f32_dkv_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, dy, lse, D, dqkv, T, C,
-                                                                                     n_head);
+                                                                                     n_head, window);
     return cudaGetLastError();
 }
 
@@ -261,9 +273,9 @@ cudaError_t launch_dkv_t(const float *qkv, const float *dy, const float *lse, co
 
 }  // namespace
 
-cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head,
+cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,
                            cudaStream_t s) {
-#define CALL(H) launch_fwd_t<H>(qkv, y, lse, B, T, C, n_head, s)
+#define CALL(H) launch_fwd_t<H>(qkv, y, lse, B, T, C, n_head, window, s)
     GPTATTN_HS_DISPATCH(hs, CALL)
 #undef CALL
 }
@@ -280,15 +292,15 @@ cudaError_t launch_bwd_f32_pre(int hs, const float *y, const float *dy, float *D
 }
 
 cudaError_t launch_bwd_f32_dq(int hs, const float *qkv, const float *dy, const float *lse, const float *D, float *dqkv,
-                              int B, int T, int C, int n_head, cudaStream_t s) {
-#define CALL(H) launch_dq_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, s)
+                              int B, int T, int C, int n_head, int window, cudaStream_t s) {
+#define CALL(H) launch_dq_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, window, s)
     GPTATTN_HS_DISPATCH(hs, CALL)
 #undef CALL
 }
 
 cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
-                               float *dqkv, int B, int T, int C, int n_head, cudaStream_t s) {
-#define CALL(H) launch_dkv_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, s)
+                               float *dqkv, int B, int T, int C, int n_head, int window, cudaStream_t s) {
+#define CALL(H) launch_dkv_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, window, s)
     GPTATTN_HS_DISPATCH(hs, CALL)
 #undef CALL
 }

@@ -28,7 +28,7 @@ GPTATTN_BF16 = 1
 
 # Every symbol include/gptattn.h declares.
 EXPORTED = (
-    "gptattn_fwd", "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
+    "gptattn_fwd", "gptattn_fwd_window", "gptattn_bwd_window", "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
     "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
     "gptattn_last_error_string",
@@ -72,6 +72,10 @@ def lib():
             vp, i, sz, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
             L.gptattn_fwd.argtypes = [vp, vp, vp, i, i, i, i, i, st]
             L.gptattn_fwd.restype = i
+            L.gptattn_fwd_window.argtypes = [vp, vp, vp, i, i, i, i, i, i, st]
+            L.gptattn_fwd_window.restype = i
+            L.gptattn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, st]
+            L.gptattn_bwd_window.restype = i
             L.gptattn_decode.argtypes = [vp, vp, vp, i, i, i, i, i, i, st]
             L.gptattn_decode.restype = i
             L.gptattn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -120,6 +124,16 @@ def _stream(s):
 
 def gptattn_fwd(qkv, y, lse, B, T, C, n_head, dt, stream=None) -> int:
     return lib().gptattn_fwd(_ptr(qkv), _ptr(y), _ptr(lse), B, T, C, n_head, dt, _stream(stream))
+
+
+def gptattn_fwd_window(qkv, y, lse, B, T, C, n_head, window, dt, stream=None) -> int:
+    return lib().gptattn_fwd_window(_ptr(qkv), _ptr(y), _ptr(lse), B, T, C, n_head, window, dt, _stream(stream))
+
+
+def gptattn_bwd_window(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, dt,
+                       stream=None) -> int:
+    return lib().gptattn_bwd_window(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), _ptr(workspace),
+                                    workspace_bytes, B, T, C, n_head, window, dt, _stream(stream))
 
 
 def gptattn_decode(qkv, y, lse, B, T, T_cap, C, n_head, dt, stream=None) -> int:

@@ -83,6 +83,25 @@ GPTATTN_API gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse,
                            int B, int T, int C, int n_head,
                            gptattn_dtype dt, gptattn_stream_t stream);
 
+/* Local-window (banded) variants of gptattn_fwd / gptattn_bwd: token t sees
+ * only positions t-window < s <= t (itself and the window-1 before it), the
+ * locally banded attention that the minGPT README page's reference notes on
+ * GPT-3 describe alternating with dense layers.  window >= 1; window >= T is
+ * exactly the causal operation (the same kernels and results as gptattn_fwd /
+ * gptattn_bwd).  Key tiles outside every query tile's band are skipped.
+ * Supported: every fp32 head size; bf16 head size 64 for any window, bf16 head
+ * size 128 only for window >= T (GPTATTN_ERR_UNSUPPORTED otherwise).
+ * window < 1 -> GPTATTN_ERR_INVALID_ARG.  Other arguments, layouts, the
+ * workspace (gptattn_bwd_workspace_bytes) and errors as in gptattn_fwd /
+ * gptattn_bwd; the backward takes the y and lse of the windowed forward. */
+GPTATTN_API gptattn_status gptattn_fwd_window(const void *qkv, void *y, float *lse,
+                                  int B, int T, int C, int n_head, int window,
+                                  gptattn_dtype dt, gptattn_stream_t stream);
+GPTATTN_API gptattn_status gptattn_bwd_window(const void *qkv, const void *y, const float *lse, const void *dy,
+                                  void *dqkv, void *workspace, size_t workspace_bytes,
+                                  int B, int T, int C, int n_head, int window,
+                                  gptattn_dtype dt, gptattn_stream_t stream);
+
 /* Decode: attention of the last position over a key/value cache (no
  * counterpart on the pages beyond the operation itself: it is row T-1 of
  * gptattn_fwd, the only row the pages' generate loop reads, computed without

@@ -34,8 +34,9 @@ class Guarded:
         return bool((lo == self.fill).all().item() and (hi == self.fill).all().item())
 
 
-def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream=None):
-    """Forward + backward through the C ABI.  Returns float64 numpy (y, lse, dqkv)."""
+def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream=None, window=None):
+    """Forward + backward through the C ABI (the local-window entry points when
+    window is given).  Returns float64 numpy (y, lse, dqkv)."""
     dev = torch.device("cuda", 0)
     dtype = qkv_cpu.dtype
     dt = ga.GPTATTN_BF16 if dtype == torch.bfloat16 else ga.GPTATTN_F32
@@ -49,8 +50,14 @@ def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream
     nbytes = ga.gptattn_bwd_workspace_bytes(B, T, C, n_head, dt)
     ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
-    ga.check(ga.gptattn_fwd(qkv, y.view, lse.view, B, T, C, n_head, dt, s), "gptattn_fwd")
-    ga.check(ga.gptattn_bwd(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, dt, s), "gptattn_bwd")
+    if window is None:
+        ga.check(ga.gptattn_fwd(qkv, y.view, lse.view, B, T, C, n_head, dt, s), "gptattn_fwd")
+        ga.check(ga.gptattn_bwd(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, dt, s),
+                 "gptattn_bwd")
+    else:
+        ga.check(ga.gptattn_fwd_window(qkv, y.view, lse.view, B, T, C, n_head, window, dt, s), "gptattn_fwd_window")
+        ga.check(ga.gptattn_bwd_window(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, window, dt,
+                                       s), "gptattn_bwd_window")
     rc = ga.gptattn_get_device_status(s)
     assert rc == ga.GPTATTN_OK, ga.status_string(rc)
     assert y.intact() and lse.intact() and dqkv.intact(), "write outside an output buffer"

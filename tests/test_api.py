@@ -121,3 +121,18 @@ def test_decode_validation():
     assert ga.gptattn_decode(None, None, None, 0, 8, 8, 128, 2, bf, None) == ga.GPTATTN_OK
     assert ga.gptattn_decode(None, None, None, 2, 0, 8, 128, 2, f32, None) == ga.GPTATTN_OK
     assert ga.gptattn_kernel_name(9) == "decode"
+
+
+def test_window_validation():
+    bf, f32 = ga.GPTATTN_BF16, ga.GPTATTN_F32
+    assert ga.gptattn_fwd_window(FAKE, FAKE, FAKE, 2, 8, 128, 2, 0, bf, None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd_window(FAKE, FAKE, FAKE, 2, 8, 128, 2, -3, f32, None) == ga.GPTATTN_ERR_INVALID_ARG
+    # bf16 head size 128 has no banded kernel: a window narrower than T is refused
+    assert ga.gptattn_fwd_window(FAKE, FAKE, FAKE, 2, 300, 256, 2, 100, bf, None) == ga.GPTATTN_ERR_UNSUPPORTED
+    ws = ga.gptattn_bwd_workspace_bytes(2, 300, 256, 2, bf)
+    assert ga.gptattn_bwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 2, 300, 256, 2, 100, bf,
+                                 None) == ga.GPTATTN_ERR_UNSUPPORTED
+    assert ga.gptattn_bwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 2, 300, 256, 2, 0, bf,
+                                 None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd_window(None, None, None, 0, 8, 128, 2, 4, bf, None) == ga.GPTATTN_OK
+    assert ga.gptattn_bwd_window(None, None, None, None, None, None, 0, 2, 0, 64, 4, 4, f32, None) == ga.GPTATTN_OK
