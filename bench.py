@@ -374,6 +374,41 @@ def run_ours(args, w, rank, world, local_rank):
     h2d = qkv_h.numel() * qkv_h.element_size() + dy_h.numel() * dy_h.element_size()
     d2h = y_h.numel() * y_h.element_size() + dqkv_h.numel() * dqkv_h.element_size()
 
+    # ---- local window (gptattn_fwd_window + gptattn_bwd_window), 256-token band: the same step
+    # with only the band's key tiles; FLOPs counted over the visible (query, key) pairs,
+    # 14 * hs per pair (4 fwd + 10 bwd), which is the causal count 7*B*nh*T^2*hs for a full band.
+    banded = None
+    if not args.profile_run and (dt == ga.GPTATTN_F32 or w.hs == 64):
+        W = 256
+        pairs = sum(min(t + 1, W) for t in range(T))
+        flops_w = 14.0 * w.hs * B * nh * pairs
+
+        def step_w():
+            ga.check(ga.gptattn_fwd_window(qkv, y, lse, B, T, C, nh, W, dt, s), "gptattn_fwd_window")
+            ga.check(ga.gptattn_bwd_window(qkv, y, lse, dy, dqkv, ws, nbytes, B, T, C, nh, W, dt, s),
+                     "gptattn_bwd_window")
+
+        for _ in range(5):
+            flush.zero_()
+            step_w()
+        torch.cuda.synchronize()
+        Kw = max(1, min(K, 200))
+        tw = 0.0
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Kw)]
+        for a, b_ in evs:
+            flush.zero_()
+            a.record(s)
+            step_w()
+            b_.record(s)
+        torch.cuda.synchronize()
+        tw = sum(a.elapsed_time(b_) for a, b_ in evs)
+        ga.check(ga.gptattn_get_device_status(s), "device status after the banded steps")
+        banded = {"window": W, "steps": Kw, "ms_per_step": tw / Kw, "flops_per_step": flops_w,
+                  "value": flops_w * Kw / (tw / 1e3) / 1e12, "unit": "TFLOP/s",
+                  "flop_count": "14*hs per visible (query, key) pair, exact band",
+                  "pct_of_measured_bf16_burst": flops_w * Kw / (tw / 1e3) / 1e12 /
+                  float(load_peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))}
+
     # ---- decode (gptattn_decode): the last position of every sequence over the same qkv as a
     # key/value cache; HBM-bound, so its roofline is the measured copy bandwidth.  L2 flushed
     # before every call.  Also a large cache (B=64, T=4096 at this head layout) for the
@@ -469,6 +504,7 @@ def run_ours(args, w, rank, world, local_rank):
                 "overlap": "copies in / compute / copies out on three streams, device buffers double-buffered"},
         "gpu_launches": launches,
         "decode": decode,
+        "window": banded,
         "clocks": clocks,
         "wall_s_timed": wall1 - wall0,
     }
