@@ -114,3 +114,17 @@ def test_bf16_rows_sum_to_one_at_full_size():
     qkv[:, :, 2 * w.C:] = 1.0
     y, lse, _ = run_fwd_bwd(qkv, dy, w.n_head)
     assert np.abs(y - 1.0).max() <= 1e-2
+
+
+def test_bf16_long_sequence():
+    """T = 4096 (32 query tiles: the longest items of the persistent schedules), two heads."""
+    qkv, dy = make_inputs(1, 4096, 2, 64, dtype=torch.bfloat16, seed=4096)
+    got = run_fwd_bwd(qkv, dy, 2)
+    compare(got, oracle_all(qkv, dy, 2), torch.bfloat16, "T=4096")
+
+
+def test_bf16_many_short_sequences():
+    """B * n_head = 1024 pairs of 130 tokens: many short work items with a ragged tail."""
+    qkv, dy = make_inputs(32, 130, 32, 64, dtype=torch.bfloat16, seed=130)
+    got = run_fwd_bwd(qkv, dy, 32)
+    compare(got, oracle_all(qkv, dy, 32), torch.bfloat16, "1024 x 130")
