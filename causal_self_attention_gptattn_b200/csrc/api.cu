@@ -144,7 +144,13 @@ struct BwdWorkspace {
     size_t D, lse2, dqacc, total;
 };
 
-BwdWorkspace workspace_layout(int B, int T, int n_head, int hs, gptattn_dtype dt) {
+// Partial dQ tiles per (b, h) in deterministic mode: one per (query tile i, key tile j <= i).
+long long det_slots(int T) {
+    const long long n_t = (T + kTile - 1) / kTile;
+    return n_t * (n_t + 1) / 2;
+}
+
+BwdWorkspace workspace_layout(int B, int T, int n_head, int hs, gptattn_dtype dt, bool det = false) {
     BwdWorkspace w{};
     if (dt == GPTATTN_F32) {
         w.D = 0;
@@ -152,10 +158,11 @@ BwdWorkspace workspace_layout(int B, int T, int n_head, int hs, gptattn_dtype dt
         return w;
     }
     const size_t rows = (size_t)B * n_head * padded_T(T);
+    const size_t acc_rows = det ? (size_t)B * n_head * (size_t)det_slots(T) * kTile : rows;
     w.D = 0;
     w.lse2 = align256(rows * sizeof(float));
     w.dqacc = w.lse2 + align256(rows * sizeof(float));
-    w.total = w.dqacc + align256(rows * (size_t)hs * sizeof(float));
+    w.total = w.dqacc + align256(acc_rows * (size_t)hs * sizeof(float));
     return w;
 }
 
@@ -282,20 +289,30 @@ gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int 
 }  // namespace
 
 namespace {
+// Deterministic mode on the bf16 path needs the head-size-64 kernels and row
+// indices of the partial-tile buffer that fit 32-bit TMA coordinates.
+gptattn_status check_det(int B, int T, int n_head, int hs, gptattn_dtype dt) {
+    if (dt != GPTATTN_BF16) return GPTATTN_OK;
+    if (hs != 64) return GPTATTN_ERR_UNSUPPORTED;
+    if ((long long)B * n_head * det_slots(T) * kTile > 0x7fffffffLL) return GPTATTN_ERR_UNSUPPORTED;
+    return GPTATTN_OK;
+}
+
 gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv, void *workspace,
-                        size_t workspace_bytes, int B, int T, int C, int n_head, int window, gptattn_dtype dt,
-                        gptattn_stream_t stream) {
+                        size_t workspace_bytes, int B, int T, int C, int n_head, int window, bool det,
+                        gptattn_dtype dt, gptattn_stream_t stream) {
     int hs = 0;
     gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
     if (st != GPTATTN_OK) return st;
     int kw = kCausalWindow;
     st = check_window(window, T, hs, dt, &kw);
     if (st != GPTATTN_OK) return st;
+    if (det && (st = check_det(B, T, n_head, hs, dt)) != GPTATTN_OK) return st;
     if (B == 0 || T == 0) return GPTATTN_OK;
     if (!qkv || !y || !lse || !dy || !dqkv) return GPTATTN_ERR_INVALID_ARG;
     if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse) || !aligned16(dy) || !aligned16(dqkv))
         return GPTATTN_ERR_INVALID_ARG;
-    const BwdWorkspace w = workspace_layout(B, T, n_head, hs, dt);
+    const BwdWorkspace w = workspace_layout(B, T, n_head, hs, dt, det);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < w.total)
         return GPTATTN_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -325,18 +342,23 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
     float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
     CUtensorMap mq, mdy, mdqkv, mdq;
     if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&mdy, dy, C, T, B) ||
-        !map_bf16_rows(&mdqkv, dqkv, 3 * C, T, B) || !map_f32_acc(&mdq, dqacc, hs, (long long)B * n_head * T_pad))
+        !map_bf16_rows(&mdqkv, dqkv, 3 * C, T, B) ||
+        !map_f32_acc(&mdq, dqacc, hs, det ? (long long)B * n_head * det_slots(T) * kTile : (long long)B * n_head * T_pad))
         return GPTATTN_ERR_CUDA;
+    const int n_slots = det ? (int)det_slots(T) : 0;
     const DevCtx ctx{status, kDefaultBudgetNs};
     cudaError_t e = run_kernel(kKBwdPreBf16, s, [&] {
-        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, s);
+        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, !det, s);
     });
     if (e == cudaSuccess)
         e = run_kernel(kKBwdMainBf16, s, [&] {
-            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, kw, ctx, s);
+            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, kw, n_slots, ctx, s);
         });
     if (e == cudaSuccess)
-        e = run_kernel(kKBwdPostBf16, s, [&] { return launch_bwd_post_bf16(hs, dqacc, dqkv, B, T, C, n_head, T_pad, s); });
+        e = run_kernel(kKBwdPostBf16, s, [&] {
+            return det ? launch_bwd_post_det_bf16(hs, dqacc, dqkv, B, T, C, n_head, T_pad, n_slots, kw, s)
+                       : launch_bwd_post_bf16(hs, dqacc, dqkv, B, T, C, n_head, T_pad, s);
+        });
     return from_cuda(e);
 }
 }  // namespace
@@ -397,13 +419,28 @@ size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtyp
 gptattn_status gptattn_bwd(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
                            void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, gptattn_dtype dt,
                            gptattn_stream_t stream) {
-    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, kCausalWindow, dt, stream);
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, kCausalWindow, false, dt,
+                    stream);
 }
 
 gptattn_status gptattn_bwd_window(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
                                   void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, int window,
                                   gptattn_dtype dt, gptattn_stream_t stream) {
-    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, dt, stream);
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, false, dt, stream);
+}
+
+size_t gptattn_bwd_det_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt) {
+    int hs = 0;
+    if (check_shape(B, T, C, n_head, dt, &hs) != GPTATTN_OK) return (size_t)-1;
+    if (check_det(B, T, n_head, hs, dt) != GPTATTN_OK) return (size_t)-1;
+    if (B == 0 || T == 0) return 0;
+    return workspace_layout(B, T, n_head, hs, dt, true).total;
+}
+
+gptattn_status gptattn_bwd_det(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
+                               void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, int window,
+                               gptattn_dtype dt, gptattn_stream_t stream) {
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, true, dt, stream);
 }
 
 gptattn_status gptattn_get_device_status(gptattn_stream_t stream) {

@@ -10,6 +10,10 @@
 // attention): key s is seen by queries s <= t < s + window, so a key tile's
 // item stops at the last query tile its band reaches and the band's far edge
 // is masked element-wise like the diagonal.  window >= T is the causal case.
+// Deterministic mode (n_slots > 0): instead of adding dQ_i into an fp32
+// accumulator with TMA reduce-adds (whose order across CTAs varies run to run),
+// each (query tile i, key tile j) partial is stored in its own slot i(i+1)/2 + j
+// and the postprocess kernel sums the slots of a query tile in a fixed order.
 //
 // Schedule: one persistent CTA per SM walks a static list of work items
 // (key tile j, batch b, head h), ordered longest first (small j first), in a
@@ -111,7 +115,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_h64_persistent(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
                        const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
                        const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C,
-                       int n_head, int T_pad, int n_t, int window, int *status, unsigned long long budget_ns) {
+                       int n_head, int T_pad, int n_t, int window, int n_slots, int *status,
+                       unsigned long long budget_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -500,7 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     named_bar_sync(2, kDrainThreads);
                     if (leader && ok && !*abort_flag) {
-                        tma_reduce_add_2d(&map_dq, sdQ, 32 * hh, bh * T_pad + qt * kTile);
+                        if (n_slots == 0)  // add into the (b, h, query tile) rows of the accumulator
+                            tma_reduce_add_2d(&map_dq, sdQ, 32 * hh, bh * T_pad + qt * kTile);
+                        else  // deterministic: a slot of its own per (query tile, key tile)
+                            tma_store_2d(&map_dq, sdQ, 32 * hh, (bh * n_slots + qt * (qt + 1) / 2 + kt) * kTile);
                         bulk_commit_group();
                     }
                 }
@@ -521,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                                int n_head, int T_pad, int window, DevCtx ctx, cudaStream_t s) {
+                                int n_head, int T_pad, int window, int n_slots, DevCtx ctx, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(bwd_h64_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -533,7 +541,7 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
     const long long items = (long long)n_t * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
     return launch_pdl(bwd_h64_persistent, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_dy, map_dqkv,
-                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, ctx.status, ctx.budget_ns);
+                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
                                                       const __nv_bfloat16 *__restrict__ dy,
                                                       const float *__restrict__ lse, float *__restrict__ D,
                                                       float *__restrict__ lse2, float4 *__restrict__ dqacc, int T,
-                                                      int C, int n_head, int T_pad) {
+                                                      int C, int n_head, int T_pad, int zero_acc) {
     constexpr int kLanesPerRow = HS / 8;
     constexpr int kRowsPerPass = kPPThreads / kLanesPerRow;
     griddep_launch_dependents();
@@ -469,6 +469,7 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
             lse2[row0 + r + sub] = t < T ? -lse[(size_t)bh * T + t] * 1.4426950408889634f : -INFINITY;
         }
     }
+    if (!zero_acc) return;
     float4 *acc = dqacc + row0 * (HS / 4);
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
@@ -504,6 +505,44 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_kernel(const float *__res
     }
 }
 
+// deterministic postprocess: dq = bf16(scale * sum over key tiles j of partial(i, j)),
+// the partials of query tile i summed in increasing j, so the result does not
+// depend on the order in which CTAs produced them.  Same grid as above; slots
+// of key tiles outside the band (window) were never written and are not read.
+template <int HS>
+__global__ void __launch_bounds__(kPPThreads) bwd_post_det_kernel(const float *__restrict__ part,
+                                                           __nv_bfloat16 *__restrict__ dqkv, int T, int C, int n_head,
+                                                           int n_slots, int window) {
+    griddep_launch_dependents();
+    griddep_wait();
+    constexpr int kPerRow = HS / 8;
+    const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
+    const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
+    const int qt = blockIdx.y, t0 = qt * kTile;
+    const int s_first = qt * kTile - window + 1;
+    const int jlo = s_first > 0 ? s_first / kTile : 0;
+    __nv_bfloat16 *dst = dqkv + ((size_t)b * T + t0) * (size_t)(3 * C) + (size_t)h * HS;
+#pragma unroll
+    for (int i = threadIdx.x; i < kTile * kPerRow; i += kPPThreads) {
+        const int r = i / kPerRow, k = i % kPerRow;
+        if (t0 + r >= T) continue;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = jlo; j <= qt; ++j) {
+            const float4 *src = reinterpret_cast<const float4 *>(
+                part + ((size_t)bh * n_slots + (size_t)(qt * (qt + 1) / 2 + j)) * kTile * HS);
+            const float4 a = src[2 * i], c = src[2 * i + 1];
+            acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+            acc[4] += c.x; acc[5] += c.y; acc[6] += c.z; acc[7] += c.w;
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0] * scale, acc[1] * scale);
+        o.y = pack_bf16x2(acc[2] * scale, acc[3] * scale);
+        o.z = pack_bf16x2(acc[4] * scale, acc[5] * scale);
+        o.w = pack_bf16x2(acc[6] * scale, acc[7] * scale);
+        *reinterpret_cast<uint4 *>(dst + (size_t)r * (size_t)(3 * C) + (size_t)k * 8) = o;
+    }
+}
+
 template <int HS>
 cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                              const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
@@ -521,23 +560,29 @@ cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_
 }  // namespace
 
 cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
-                                float *dqacc, int B, int T, int C, int n_head, int T_pad, cudaStream_t s) {
+                                float *dqacc, int B, int T, int C, int n_head, int T_pad, bool zero_acc, cudaStream_t s) {
     const dim3 grid((unsigned)(B * n_head), (unsigned)(T_pad / kTile));
     auto yy = static_cast<const __nv_bfloat16 *>(y);
     auto gg = static_cast<const __nv_bfloat16 *>(dy);
     auto zz = reinterpret_cast<float4 *>(dqacc);
-    if (hs == 64) return launch_pdl(bwd_pre_kernel<64>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
-    if (hs == 128) return launch_pdl(bwd_pre_kernel<128>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad);
+    const int za = zero_acc ? 1 : 0;
+    if (hs == 64)
+        return launch_pdl(bwd_pre_kernel<64>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad,
+                          za);
+    if (hs == 128)
+        return launch_pdl(bwd_pre_kernel<128>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad,
+                          za);
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
                                  const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
-                                 const float *D, int B, int T, int C, int n_head, int T_pad, int window, DevCtx ctx,
-                                 cudaStream_t s) {
+                                 const float *D, int B, int T, int C, int n_head, int T_pad, int window, int n_slots,
+                                 DevCtx ctx, cudaStream_t s) {
     if (hs == 64)
-        return launch_bwd_main_h64(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, ctx, s);
-    if (hs == 128 && window >= T)
+        return launch_bwd_main_h64(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots,
+                                   ctx, s);
+    if (hs == 128 && window >= T && n_slots == 0)
         return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
     return cudaErrorInvalidValue;
 }
@@ -550,4 +595,13 @@ cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, 
     if (hs == 128) return launch_pdl(bwd_post_kernel<128>, grid, dim3(kPPThreads), 0, s, dqacc, out, T, C, n_head, T_pad);
     return cudaErrorInvalidValue;
 }
+cudaError_t launch_bwd_post_det_bf16(int hs, const float *part, void *dqkv, int B, int T, int C, int n_head, int T_pad,
+                                     int n_slots, int window, cudaStream_t s) {
+    const dim3 grid((unsigned)(B * n_head), (unsigned)(T_pad / kTile));
+    auto out = static_cast<__nv_bfloat16 *>(dqkv);
+    if (hs == 64)
+        return launch_pdl(bwd_post_det_kernel<64>, grid, dim3(kPPThreads), 0, s, part, out, T, C, n_head, n_slots, window);
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace gptattn

@@ -60,23 +60,29 @@ cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y,
 // D[bh][t] = sum_d y*dy, lse2[bh][t] = lse*log2(e) (rows t >= T: 0 and +inf),
 // dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].
 cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
-                                float *dqacc, int B, int T, int C, int n_head, int T_pad, cudaStream_t s);
+                                float *dqacc, int B, int T, int C, int n_head, int T_pad, bool zero_acc, cudaStream_t s);
 
 // map_dy: 3-D view (C, T, B) of dy; map_dqkv: 3-D view (3C, T, B) of dqkv;
 // map_dq: 2-D view (hs, B*n_head*T_pad) of dqacc (fp32), box (32, 128), 128-byte swizzle.
 cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
                                  const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
-                                 const float *D, int B, int T, int C, int n_head, int T_pad, int window, DevCtx ctx,
-                                 cudaStream_t s);
+                                 const float *D, int B, int T, int C, int n_head, int T_pad, int window, int n_slots,
+                                 DevCtx ctx, cudaStream_t s);
 
 // Persistent head-size-64 variant of the above (same arguments).
 cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                                int n_head, int T_pad, int window, DevCtx ctx, cudaStream_t s);
+                                int n_head, int T_pad, int window, int n_slots, DevCtx ctx, cudaStream_t s);
 
 // dqkv[b][t][h*hs+d] = bf16(dqacc[(b*n_head+h)*T_pad + t][d] / sqrt(hs)).
 cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head,
                                  int T_pad, cudaStream_t s);
+
+// Deterministic mode: n_slots = n_t(n_t+1)/2 partial dQ tiles per (b, h), the partial of
+// (query tile i, key tile j) in rows (bh*n_slots + i(i+1)/2 + j)*128 of `part` ([rows][hs]
+// fp32); the postprocess sums a query tile's partials in increasing j (head size 64).
+cudaError_t launch_bwd_post_det_bf16(int hs, const float *part, void *dqkv, int B, int T, int C, int n_head, int T_pad,
+                                     int n_slots, int window, cudaStream_t s);
 
 // ---- fp32 CUDA-core path --------------------------------------------------
 cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,

@@ -28,7 +28,8 @@ GPTATTN_BF16 = 1
 
 # Every symbol include/gptattn.h declares.
 EXPORTED = (
-    "gptattn_fwd", "gptattn_fwd_window", "gptattn_bwd_window", "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
+    "gptattn_fwd", "gptattn_fwd_window", "gptattn_bwd_window", "gptattn_bwd_det_workspace_bytes", "gptattn_bwd_det",
+    "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
     "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
     "gptattn_last_error_string",
@@ -76,6 +77,10 @@ def lib():
             L.gptattn_fwd_window.restype = i
             L.gptattn_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, st]
             L.gptattn_bwd_window.restype = i
+            L.gptattn_bwd_det_workspace_bytes.argtypes = [i, i, i, i, i]
+            L.gptattn_bwd_det_workspace_bytes.restype = sz
+            L.gptattn_bwd_det.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, st]
+            L.gptattn_bwd_det.restype = i
             L.gptattn_decode.argtypes = [vp, vp, vp, i, i, i, i, i, i, st]
             L.gptattn_decode.restype = i
             L.gptattn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -134,6 +139,16 @@ def gptattn_bwd_window(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, 
                        stream=None) -> int:
     return lib().gptattn_bwd_window(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), _ptr(workspace),
                                     workspace_bytes, B, T, C, n_head, window, dt, _stream(stream))
+
+
+def gptattn_bwd_det_workspace_bytes(B, T, C, n_head, dt) -> int:
+    return lib().gptattn_bwd_det_workspace_bytes(B, T, C, n_head, dt)
+
+
+def gptattn_bwd_det(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, dt,
+                    stream=None) -> int:
+    return lib().gptattn_bwd_det(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), _ptr(workspace),
+                                 workspace_bytes, B, T, C, n_head, window, dt, _stream(stream))
 
 
 def gptattn_decode(qkv, y, lse, B, T, T_cap, C, n_head, dt, stream=None) -> int:

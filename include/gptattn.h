@@ -102,6 +102,25 @@ GPTATTN_API gptattn_status gptattn_bwd_window(const void *qkv, const void *y, co
                                   int B, int T, int C, int n_head, int window,
                                   gptattn_dtype dt, gptattn_stream_t stream);
 
+/* Deterministic backward (no counterpart on the pages beyond the operation:
+ * a reproducibility variant of gptattn_bwd_window).  gptattn_bwd adds each
+ * key tile's contribution to dQ into an fp32 accumulator with reduce-adds
+ * whose order varies from run to run, so its bf16 dq can differ in the last
+ * bit between runs.  This variant stores every (query tile, key tile) partial
+ * of dQ in a workspace slot of its own and sums a query tile's partials in a
+ * fixed order, so equal inputs give bit-identical dqkv on every run.  Same
+ * arguments, semantics, support (bf16: head size 64 only, any window) and
+ * errors as gptattn_bwd_window, with a larger workspace:
+ * gptattn_bwd_det_workspace_bytes() (for bf16 it adds B * n_head *
+ * ceil(T/128)(ceil(T/128)+1)/2 tiles of 128 x 64 fp32; (size_t)-1 for an
+ * unsupported or invalid shape).  The fp32 path has no reduce-adds and is
+ * deterministic in both entry points. */
+GPTATTN_API size_t gptattn_bwd_det_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt);
+GPTATTN_API gptattn_status gptattn_bwd_det(const void *qkv, const void *y, const float *lse, const void *dy,
+                               void *dqkv, void *workspace, size_t workspace_bytes,
+                               int B, int T, int C, int n_head, int window,
+                               gptattn_dtype dt, gptattn_stream_t stream);
+
 /* Decode: attention of the last position over a key/value cache (no
  * counterpart on the pages beyond the operation itself: it is row T-1 of
  * gptattn_fwd, the only row the pages' generate loop reads, computed without

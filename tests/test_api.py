@@ -136,3 +136,21 @@ def test_window_validation():
                                  None) == ga.GPTATTN_ERR_INVALID_ARG
     assert ga.gptattn_fwd_window(None, None, None, 0, 8, 128, 2, 4, bf, None) == ga.GPTATTN_OK
     assert ga.gptattn_bwd_window(None, None, None, None, None, None, 0, 2, 0, 64, 4, 4, f32, None) == ga.GPTATTN_OK
+
+
+def test_deterministic_backward_workspace_and_validation():
+    bf, f32 = ga.GPTATTN_BF16, ga.GPTATTN_F32
+    B, T, C, nh = 2, 300, 128, 2  # 3 query tiles -> 6 partial tiles per (b, h)
+    rows = B * nh * 384
+    base = rows * 4 + rows * 4
+    assert ga.gptattn_bwd_det_workspace_bytes(B, T, C, nh, bf) == base + B * nh * 6 * 128 * 64 * 4
+    assert ga.gptattn_bwd_det_workspace_bytes(B, T, C, nh, f32) == ga.gptattn_bwd_workspace_bytes(B, T, C, nh, f32)
+    assert ga.gptattn_bwd_det_workspace_bytes(B, T, 256, nh, bf) == (1 << 64) - 1  # head size 128
+    ws = ga.gptattn_bwd_det_workspace_bytes(B, T, C, nh, bf)
+    assert ga.gptattn_bwd_det(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 1, B, T, C, nh, 10**6, bf,
+                              None) == ga.GPTATTN_ERR_WORKSPACE
+    assert ga.gptattn_bwd_det(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, B, T, 256, nh, 10**6, bf,
+                              None) == ga.GPTATTN_ERR_UNSUPPORTED
+    assert ga.gptattn_bwd_det(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, B, T, C, nh, 0, bf,
+                              None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_bwd_det(None, None, None, None, None, None, 0, 0, T, C, nh, 1, bf, None) == ga.GPTATTN_OK
