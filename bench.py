@@ -409,6 +409,36 @@ def run_ours(args, w, rank, world, local_rank):
                   "pct_of_measured_bf16_burst": flops_w * Kw / (tw / 1e3) / 1e12 /
                   float(load_peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))}
 
+    # ---- deterministic backward (gptattn_bwd_det): the same step with dQ partials stored per
+    # (query tile, key tile) and summed in a fixed order instead of reduce-added.
+    det = None
+    if not args.profile_run and (dt == ga.GPTATTN_F32 or w.hs == 64):
+        nb_det = ga.gptattn_bwd_det_workspace_bytes(B, T, C, nh, dt)
+        ws_det = torch.empty(max(nb_det, 256), dtype=torch.uint8, device=dev)
+
+        def step_det():
+            ga.check(ga.gptattn_fwd(qkv, y, lse, B, T, C, nh, dt, s), "gptattn_fwd")
+            ga.check(ga.gptattn_bwd_det(qkv, y, lse, dy, dqkv, ws_det, nb_det, B, T, C, nh, 1 << 30, dt, s),
+                     "gptattn_bwd_det")
+
+        for _ in range(5):
+            flush.zero_()
+            step_det()
+        torch.cuda.synchronize()
+        Kd = max(1, min(K, 200))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Kd)]
+        for a, b_ in evs:
+            flush.zero_()
+            a.record(s)
+            step_det()
+            b_.record(s)
+        torch.cuda.synchronize()
+        td = sum(a.elapsed_time(b_) for a, b_ in evs)
+        ga.check(ga.gptattn_get_device_status(s), "device status after the deterministic steps")
+        det = {"steps": Kd, "ms_per_step": td / Kd, "value": flops * Kd / (td / 1e3) / 1e12, "unit": "TFLOP/s",
+               "workspace_bytes": nb_det}
+        del ws_det
+
     # ---- decode (gptattn_decode): the last position of every sequence over the same qkv as a
     # key/value cache; HBM-bound, so its roofline is the measured copy bandwidth.  L2 flushed
     # before every call.  Also a large cache (B=64, T=4096 at this head layout) for the
@@ -505,6 +535,7 @@ def run_ours(args, w, rank, world, local_rank):
         "gpu_launches": launches,
         "decode": decode,
         "window": banded,
+        "deterministic": det,
         "clocks": clocks,
         "wall_s_timed": wall1 - wall0,
     }
