@@ -88,6 +88,14 @@ class Oracle:
         lib.oracle_bwd_window.restype = i
         lib.oracle_probs_window.argtypes = [dp, i, i, i, i, i, i, i, dp]
         lib.oracle_probs_window.restype = i
+        u64 = ctypes.c_uint64
+        lib.oracle_fwd_ex.argtypes = [dp, i, i, i, i, i, ctypes.c_double, u64, dp, dp]
+        lib.oracle_fwd_ex.restype = i
+        lib.oracle_bwd_ex.argtypes = [dp, dp, i, i, i, i, i, ctypes.c_double, u64, dp]
+        lib.oracle_bwd_ex.restype = i
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        lib.oracle_philox4x32_10.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i
         lib.oracle_set_num_threads.argtypes = [i]
@@ -101,14 +109,18 @@ class Oracle:
     def set_num_threads(self, n: int) -> None:
         self.lib.oracle_set_num_threads(int(n))
 
-    def forward(self, qkv, n_head: int, window=None):
+    def forward(self, qkv, n_head: int, window=None, dropout: float = 0.0, seed: int = 0):
         """Return (y[B,T,C], lse[B,n_head,T]) in float64.  window: local band width
-        (token t sees t-window < s <= t); None = causal (every past position)."""
+        (token t sees t-window < s <= t); None = causal (every past position).
+        dropout: probability of dropping an attention weight (Philox mask from seed)."""
         q = _f64(qkv)
         B, T, C = _shape(q, n_head)
         y = np.zeros((B, T, C), dtype=np.float64)
         lse = np.zeros((B, n_head, T), dtype=np.float64)
-        if window is None:
+        if dropout > 0.0:
+            w = max(T, 1) if window is None else int(window)
+            rc = self.lib.oracle_fwd_ex(_ptr(q), B, T, C, n_head, w, float(dropout), int(seed), _ptr(y), _ptr(lse))
+        elif window is None:
             rc = self.lib.oracle_fwd(_ptr(q), B, T, C, n_head, _ptr(y), _ptr(lse))
         else:
             rc = self.lib.oracle_fwd_window(_ptr(q), B, T, C, n_head, int(window), _ptr(y), _ptr(lse))
@@ -116,21 +128,32 @@ class Oracle:
             raise RuntimeError(f"oracle_fwd failed with code {rc}")
         return y, lse
 
-    def backward(self, qkv, dy, n_head: int, window=None):
-        """Return dqkv[B,T,3C] = d(sum(y*dy))/d(qkv) in float64 (window as in forward)."""
+    def backward(self, qkv, dy, n_head: int, window=None, dropout: float = 0.0, seed: int = 0):
+        """Return dqkv[B,T,3C] = d(sum(y*dy))/d(qkv) in float64 (window, dropout, seed as in forward)."""
         q = _f64(qkv)
         g = _f64(dy)
         B, T, C = _shape(q, n_head)
         if g.shape != (B, T, C):
             raise ValueError(f"dy must be {(B, T, C)}, got {g.shape}")
         dqkv = np.zeros((B, T, 3 * C), dtype=np.float64)
-        if window is None:
+        if dropout > 0.0:
+            w = max(T, 1) if window is None else int(window)
+            rc = self.lib.oracle_bwd_ex(_ptr(q), _ptr(g), B, T, C, n_head, w, float(dropout), int(seed), _ptr(dqkv))
+        elif window is None:
             rc = self.lib.oracle_bwd(_ptr(q), _ptr(g), B, T, C, n_head, _ptr(dqkv))
         else:
             rc = self.lib.oracle_bwd_window(_ptr(q), _ptr(g), B, T, C, n_head, int(window), _ptr(dqkv))
         if rc:
             raise RuntimeError(f"oracle_bwd failed with code {rc}")
         return dqkv
+
+    def philox(self, ctr, key):
+        """Philox4x32-10 of a 4-word counter under a 2-word key (four uint32 words)."""
+        c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in ctr])
+        k = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+        o = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(c, k, o)
+        return [int(x) for x in o]
 
     def probs(self, qkv, n_head: int, b: int, h: int, window=None):
         """Return the T x T attention weights of batch b, head h (window as in forward)."""
@@ -162,12 +185,16 @@ def set_num_threads(n: int) -> None:
     default().set_num_threads(n)
 
 
-def forward(qkv, n_head: int, window=None):
-    return default().forward(qkv, n_head, window)
+def forward(qkv, n_head: int, window=None, dropout: float = 0.0, seed: int = 0):
+    return default().forward(qkv, n_head, window, dropout, seed)
 
 
-def backward(qkv, dy, n_head: int, window=None):
-    return default().backward(qkv, dy, n_head, window)
+def backward(qkv, dy, n_head: int, window=None, dropout: float = 0.0, seed: int = 0):
+    return default().backward(qkv, dy, n_head, window, dropout, seed)
+
+
+def philox(ctr, key):
+    return default().philox(ctr, key)
 
 
 def probs(qkv, n_head: int, b: int, h: int, window=None):

@@ -33,6 +33,13 @@
  *    positions: token t sees s with t - window < s <= t (itself and the
  *    window-1 before it); window >= T is the dense causal case above, with the
  *    same arithmetic.
+ *  - "Let's build GPT" lecture page, chapter "scaling up the model! creating a
+ *    few variables. adding dropout": dropout on the attention weights.  Read
+ *    as inverted dropout after the softmax: weight P[t][s] is kept with
+ *    probability 1-p and then scaled by 1/(1-p), else zeroed; lse stays the
+ *    logsumexp of the undropped scores.  The keep decision is a counter-based
+ *    random number (Philox4x32-10, below), so the forward and the backward
+ *    see the same mask without storing it.
  *
  * Input packing (the projection output of a GPT-2 style block): qkv[B][T][3C]
  * row-major, q = columns [0,C), k = [C,2C), v = [2C,3C).  Output y[B][T][C]
@@ -56,6 +63,59 @@
 #include <omp.h>
 #endif
 
+/* ---------------------------------------------------------------------------
+ * Philox4x32-10, written from its published definition (J. Salmon, M. Moraes,
+ * R. Dror, D. Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011):
+ * ten rounds on a 128-bit counter (c0, c1, c2, c3) under a 64-bit key (k0, k1).
+ * A round multiplies c0 and c2 by the two round multipliers, keeps the 64-bit
+ * products' high and low words, and permutes them as
+ *     (hi(M1*c2) ^ c1 ^ k0,  lo(M1*c2),  hi(M0*c0) ^ c3 ^ k1,  lo(M0*c0));
+ * between rounds the key is advanced by the two Weyl constants.
+ * PARITY UNPINNED for the generator's exact bits: no known-answer vectors are
+ * available here; the pins check its statistics and every use of its output.
+ * ------------------------------------------------------------------------- */
+#define PHILOX_M0 0xD2511F53u
+#define PHILOX_M1 0xCD9E8D57u
+#define PHILOX_W0 0x9E3779B9u
+#define PHILOX_W1 0xBB67AE85u
+
+void oracle_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint32_t out[4]) {
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        const uint64_t p0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;
+        const uint64_t p1 = (uint64_t)PHILOX_M1 * (uint64_t)c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+        k0 += PHILOX_W0;
+        k1 += PHILOX_W1;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+/* Keep decision for attention weight (t, s) of batch-head pair bh: counter
+ * (s / 4, t, bh, 0), key = the 64-bit seed, word s % 4; kept iff that word is
+ * >= threshold, threshold = floor(p * 2^32). */
+static int dropout_keep(uint64_t seed, uint32_t threshold, int bh, int t, int s) {
+    const uint32_t ctr[4] = {(uint32_t)s >> 2, (uint32_t)t, (uint32_t)bh, 0u};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t r[4];
+    oracle_philox4x32_10(ctr, key, r);
+    return r[s & 3] >= threshold;
+}
+
+static uint32_t dropout_threshold(double p) {
+    const double x = floor(p * 4294967296.0);
+    return x >= 4294967295.0 ? 4294967295u : (uint32_t)x;
+}
+
 #define ORACLE_OK 0
 #define ORACLE_EINVAL 1
 #define ORACLE_ENOMEM 2
@@ -72,6 +132,18 @@ static inline double qkv_at(const double *qkv, int T, int C, int hs, int b, int 
                             int part, int h, int d) {
     size_t row = (size_t)b * (size_t)T + (size_t)t;
     return qkv[row * (size_t)(3 * C) + (size_t)part * (size_t)C + (size_t)h * (size_t)hs + (size_t)d];
+}
+
+/* Dropout on the attention weights: p = 0 means none. */
+typedef struct {
+    double p;
+    uint64_t seed;
+} Dropout;
+
+/* Factor applied to weight (t, s): 1/(1-p) if kept, 0 if dropped; exactly 1 without dropout. */
+static inline double drop_factor(const Dropout *dr, int bh, int t, int s) {
+    if (dr->p <= 0.0) return 1.0;
+    return dropout_keep(dr->seed, dropout_threshold(dr->p), bh, t, s) ? 1.0 / (1.0 - dr->p) : 0.0;
 }
 
 /* First key position visible to query t, and last query position that sees key s. */
@@ -109,15 +181,17 @@ static void head_probs(const double *qkv, int T, int C, int hs, int window, int 
     }
 }
 
-/* y[b,t,h*hs+d] = sum_s P[t][s] v_s[d] */
-static void head_output(const double *qkv, int T, int C, int hs, int window, int b, int h,
-                        const double *P, double *y) {
+/* y[b,t,h*hs+d] = sum_s P[t][s] f[t][s] v_s[d], f the dropout factor (1 without dropout) */
+static void head_output(const double *qkv, int T, int C, int hs, int window, const Dropout *dr, int n_head, int b,
+                        int h, const double *P, double *y) {
+    const int bh = b * n_head + h;
     for (int t = 0; t < T; ++t) {
         const double *Pt = P + (size_t)t * (size_t)T;
         double *yt = y + ((size_t)b * (size_t)T + (size_t)t) * (size_t)C + (size_t)h * (size_t)hs;
         for (int d = 0; d < hs; ++d) {
             double acc = 0.0;
-            for (int s = band_lo(t, window); s <= t; ++s) acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);
+            for (int s = band_lo(t, window); s <= t; ++s)
+                acc += Pt[s] * drop_factor(dr, bh, t, s) * qkv_at(qkv, T, C, hs, b, s, 2, h, d);
             yt[d] = acc;
         }
     }
@@ -139,12 +213,14 @@ void oracle_set_num_threads(int n) {
 #endif
 }
 
-/* Forward over a local window: y[B][T][C] and lse[B][n_head][T] (either may be
- * NULL).  window >= 1. */
-int oracle_fwd_window(const double *qkv, int B, int T, int C, int n_head, int window, double *y, double *lse) {
+/* Forward over a local window with dropout on the weights: y[B][T][C] and
+ * lse[B][n_head][T] (either may be NULL).  window >= 1, 0 <= p < 1. */
+int oracle_fwd_ex(const double *qkv, int B, int T, int C, int n_head, int window, double p, uint64_t seed, double *y,
+                  double *lse) {
     int rc = check_shape(B, T, C, n_head);
     if (rc) return rc;
-    if (window < 1) return ORACLE_EINVAL;
+    if (window < 1 || !(p >= 0.0 && p < 1.0)) return ORACLE_EINVAL;
+    const Dropout dr = {p, seed};
     if (B == 0 || T == 0) return ORACLE_OK;
     const int hs = C / n_head;
     const int pairs = B * n_head;
@@ -162,11 +238,17 @@ int oracle_fwd_window(const double *qkv, int B, int T, int C, int n_head, int wi
             const int b = p / n_head, h = p % n_head;
             double *lse_row = lse ? lse + ((size_t)b * (size_t)n_head + (size_t)h) * (size_t)T : NULL;
             head_probs(qkv, T, C, hs, window, b, h, P, lse_row);
-            if (y) head_output(qkv, T, C, hs, window, b, h, P, y);
+            if (y) head_output(qkv, T, C, hs, window, &dr, n_head, b, h, P, y);
         }
         free(P);
     }
     return err ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+/* Forward over a local window: y[B][T][C] and lse[B][n_head][T] (either may be
+ * NULL).  window >= 1. */
+int oracle_fwd_window(const double *qkv, int B, int T, int C, int n_head, int window, double *y, double *lse) {
+    return oracle_fwd_ex(qkv, B, T, C, n_head, window, 0.0, 0, y, lse);
 }
 
 /* Forward, causal (every past position visible). */
@@ -189,13 +271,16 @@ int oracle_probs(const double *qkv, int B, int T, int C, int n_head, int b, int 
     return oracle_probs_window(qkv, B, T, C, n_head, T > 0 ? T : 1, b, h, P);
 }
 
-/* Backward over a local window: dqkv[B][T][3C] = d(sum y o dy)/d(qkv), by the
- * chain rule through the weighted sum, the row softmax and the scaled dot
- * products.  window >= 1. */
-int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, int n_head, int window, double *dqkv) {
+/* Backward over a local window with dropout on the weights: dqkv[B][T][3C] =
+ * d(sum y o dy)/d(qkv) for the same dropout mask as oracle_fwd_ex, by the chain
+ * rule through the weighted sum (of the dropped weights P o f), the row softmax
+ * and the scaled dot products.  window >= 1, 0 <= p < 1. */
+int oracle_bwd_ex(const double *qkv, const double *dy, int B, int T, int C, int n_head, int window, double p,
+                  uint64_t seed, double *dqkv) {
     int rc = check_shape(B, T, C, n_head);
     if (rc) return rc;
-    if (window < 1) return ORACLE_EINVAL;
+    if (window < 1 || !(p >= 0.0 && p < 1.0)) return ORACLE_EINVAL;
+    const Dropout dr = {p, seed};
     if (B == 0 || T == 0) return ORACLE_OK;
     const int hs = C / n_head;
     const double scale = 1.0 / sqrt((double)hs);
@@ -220,8 +305,8 @@ int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, 
             double *dv = dq + 2 * C;
             const size_t ld_dy = (size_t)C, ld_dqkv = (size_t)(3 * C);
 
-            /* dP[t][s] = dy_t . v_s  (visible s only), then
-             * dS[t][s] = P[t][s] * (dP[t][s] - sum_r P[t][r] dP[t][r]) */
+            /* dP[t][s] = f[t][s] (dy_t . v_s)  (visible s only; dy_t . v_s is the gradient of
+             * the dropped weight), then dS[t][s] = P[t][s] * (dP[t][s] - sum_r P[t][r] dP[t][r]) */
             for (int t = 0; t < T; ++t) {
                 const double *Pt = P + (size_t)t * (size_t)T;
                 double *dSt = dS + (size_t)t * (size_t)T;
@@ -230,6 +315,7 @@ int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, 
                 for (int s = lo; s <= t; ++s) {
                     double acc = 0.0;
                     for (int d = 0; d < hs; ++d) acc += dyb[(size_t)t * ld_dy + d] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);
+                    acc *= drop_factor(&dr, b * n_head + h, t, s);
                     dSt[s] = acc;
                     rowdot += Pt[s] * acc;
                 }
@@ -237,12 +323,13 @@ int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, 
                 for (int s = 0; s < lo; ++s) dSt[s] = 0.0;
                 for (int s = t + 1; s < T; ++s) dSt[s] = 0.0;
             }
-            /* dV[s] = sum over the queries t that see s of P[t][s] dy_t */
+            /* dV[s] = sum over the queries t that see s of P[t][s] f[t][s] dy_t */
             for (int s = 0; s < T; ++s)
                 for (int d = 0; d < hs; ++d) {
                     double acc = 0.0;
                     for (int t = s; t <= band_hi(s, window, T); ++t)
-                        acc += P[(size_t)t * (size_t)T + s] * dyb[(size_t)t * ld_dy + d];
+                        acc += P[(size_t)t * (size_t)T + s] * drop_factor(&dr, b * n_head + h, t, s) *
+                               dyb[(size_t)t * ld_dy + d];
                     dv[(size_t)s * ld_dqkv + d] = acc;
                 }
             /* dQ[t] = scale * sum over the visible s of dS[t][s] k_s */
@@ -266,6 +353,11 @@ int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, 
         free(dS);
     }
     return err ? ORACLE_ENOMEM : ORACLE_OK;
+}
+
+/* Backward over a local window (no dropout). */
+int oracle_bwd_window(const double *qkv, const double *dy, int B, int T, int C, int n_head, int window, double *dqkv) {
+    return oracle_bwd_ex(qkv, dy, B, T, C, n_head, window, 0.0, 0, dqkv);
 }
 
 /* Backward, causal (every past position visible). */

@@ -11,7 +11,12 @@ Page cited throughout: "Let's build GPT: from scratch, in code, spelled out"
 (the lecture page with the chapter list and corrections).  The local-window
 pins (``pin_window_*``) follow the minGPT README page's reference notes on
 GPT-3 (alternating dense and locally banded sparse attention), read as: token
-t sees positions t-window < s <= t.
+t sees positions t-window < s <= t.  The dropout pins (``pin_dropout_*``) follow
+the lecture's chapter "scaling up the model! creating a few variables. adding
+dropout", read as inverted dropout on the attention weights with a Philox4x32-10
+keep mask (counter (s/4, t, b*n_head+h, 0), key = seed, word s%4, kept iff the
+word >= floor(p * 2^32)); the generator's own bits are not pinned (no
+known-answer vectors are available here), only its statistics.
 """
 from __future__ import annotations
 
@@ -413,6 +418,118 @@ def pin_window_finite_differences(orc):
     assert err < 1e-6, f"finite-difference mismatch {err:.3e}"
 
 
+# ---- dropout on the attention weights --------------------------------------------
+
+def _mask_probe(orc, p, seed, T=64, n_head=2):
+    """Zero queries (uniform weights) and v = the identity (hs = T): then
+    y[t][h*T + s] = f(t, s) / (t + 1) exposes the dropout factor f of every weight."""
+    hs = T
+    C = n_head * hs
+    qkv = np.zeros((1, T, 3 * C))
+    qkv[0, :, C:2 * C] = _rng(40).standard_normal((T, C))   # keys: irrelevant when q = 0
+    for h in range(n_head):
+        qkv[0, :, 2 * C + h * hs:2 * C + (h + 1) * hs] = np.eye(T)
+    y, _ = orc.forward(qkv, n_head, dropout=p, seed=seed)
+    f = np.zeros((n_head, T, T))
+    for h in range(n_head):
+        f[h] = y[0, :, h * hs:(h + 1) * hs] * (np.arange(T)[:, None] + 1)
+    return f
+
+
+def pin_dropout_mask_and_scale(orc):
+    """Inverted dropout: every visible weight is either 0 or scaled by exactly
+    1/(1-p); none above the diagonal; the keep rate is 1-p (binomial, 5 sigma);
+    the two heads get different masks."""
+    p = 0.3
+    f = _mask_probe(orc, p, seed=11)
+    T = f.shape[1]
+    tril = np.tril(np.ones((T, T), dtype=bool))
+    vals = f[:, tril]
+    kept = np.abs(vals - 1.0 / (1.0 - p)) < 1e-12
+    dropped = np.abs(vals) < 1e-15
+    assert np.all(kept | dropped)
+    assert np.all(np.abs(f[:, ~tril]) < 1e-15)
+    n = vals.size
+    rate = kept.mean()
+    assert abs(rate - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
+    assert not np.array_equal(kept.reshape(2, -1)[0], kept.reshape(2, -1)[1])
+
+
+def pin_dropout_counter_layout(orc):
+    """Weight (t, s) of batch-head pair bh is kept iff word s%4 of Philox4x32-10 at
+    counter (s/4, t, bh, 0) under key (seed low, seed high) is >= floor(p * 2^32):
+    the mapping the CUDA path must follow too."""
+    p, seed = 0.45, (7 << 32) | 12345
+    f = _mask_probe(orc, p, seed=seed, T=48, n_head=2)
+    thr = math.floor(p * 2.0 ** 32)
+    for h in range(2):
+        for t in range(48):
+            for s_ in range(t + 1):
+                r = orc.philox([s_ // 4, t, h, 0], [seed & 0xFFFFFFFF, seed >> 32])
+                assert (r[s_ % 4] >= thr) == (f[h, t, s_] > 0), (h, t, s_)
+
+
+def pin_dropout_lse_unchanged_and_unbiased(orc):
+    """lse is that of the undropped weights (bit-identical); averaged over many
+    seeds the output approaches the undropped output (inverted dropout is unbiased)."""
+    B, T, n_head, hs, p = 1, 12, 1, 4, 0.5
+    C = n_head * hs
+    qkv = _rng(41).standard_normal((B, T, 3 * C))
+    y0, l0 = orc.forward(qkv, n_head)
+    acc = np.zeros_like(y0)
+    N = 400
+    for k in range(N):
+        y, l = orc.forward(qkv, n_head, dropout=p, seed=1000 + k)
+        assert np.array_equal(l, l0)
+        acc += y
+    mean = acc / N
+    # per element the estimator's std is at most max|v| * sqrt(p/(1-p)) / sqrt(N)
+    bound = 5 * np.abs(qkv[:, :, 2 * C:]).max() * math.sqrt(p / (1 - p)) / math.sqrt(N)
+    assert np.abs(mean - y0).max() < bound
+
+
+def pin_dropout_finite_differences(orc):
+    """With the mask fixed by the seed, the backward is the gradient of sum(y * dy)."""
+    B, T, n_head, hs, p, seed = 1, 6, 2, 3, 0.4, 99
+    C = n_head * hs
+    r = _rng(42)
+    qkv = r.standard_normal((B, T, 3 * C))
+    G = r.standard_normal((B, T, C))
+    grad = orc.backward(qkv, G, n_head, dropout=p, seed=seed)
+    h = 1e-6
+    fd = np.zeros_like(qkv)
+    flat = qkv.reshape(-1)
+    for i in range(flat.size):
+        xp = flat.copy()
+        xm = flat.copy()
+        xp[i] += h
+        xm[i] -= h
+        yp, _ = orc.forward(xp.reshape(qkv.shape), n_head, dropout=p, seed=seed)
+        ym, _ = orc.forward(xm.reshape(qkv.shape), n_head, dropout=p, seed=seed)
+        fd.reshape(-1)[i] = ((yp * G).sum() - (ym * G).sum()) / (2 * h)
+    err = np.abs(fd - grad).max() / np.abs(grad).max()
+    assert err < 1e-6, f"finite-difference mismatch {err:.3e}"
+
+
+def pin_philox_statistics(orc):
+    """The generator's words look uniform: mean, every bit's frequency and a 16-bin
+    chi-square over 4096 counters (4 words each) within generous bounds."""
+    words = []
+    for i in range(4096):
+        words += orc.philox([i, 3 * i, 7, 0], [0x1234, 0x5678])
+    w = np.array(words, dtype=np.float64)
+    n = w.size
+    u = w / 2.0 ** 32
+    assert abs(u.mean() - 0.5) < 5 * math.sqrt(1 / 12 / n)
+    wi = np.array(words, dtype=np.uint64)
+    for bit in range(32):
+        freq = ((wi >> bit) & 1).mean()
+        assert abs(freq - 0.5) < 5 * math.sqrt(0.25 / n)
+    counts = np.bincount((u * 16).astype(int), minlength=16)
+    chi2 = ((counts - n / 16) ** 2 / (n / 16)).sum()
+    assert chi2 < 50  # 15 degrees of freedom: P(chi2 > 50) is about 1e-5
+
+
 ALL_PINS = [
     pin_single_token, pin_uniform_scores_prefix_mean, pin_tril_average_fixture,
     pin_rows_are_distributions, pin_weights_from_softmax_of_scaled_scores,
@@ -421,4 +538,6 @@ ALL_PINS = [
     pin_regression_fixture, pin_empty,
     pin_window_one, pin_window_covers_all, pin_window_uniform_scores, pin_window_locality,
     pin_window_library_special_case, pin_window_finite_differences,
+    pin_dropout_mask_and_scale, pin_dropout_counter_layout, pin_dropout_lse_unchanged_and_unbiased,
+    pin_dropout_finite_differences, pin_philox_statistics,
 ]

@@ -19,8 +19,8 @@ MUTANTS = [
     ("scores_transposed",
      "acc += qkv_at(qkv, T, C, hs, b, t, 0, h, d) * qkv_at(qkv, T, C, hs, b, s, 1, h, d);",
      "acc += qkv_at(qkv, T, C, hs, b, s, 0, h, d) * qkv_at(qkv, T, C, hs, b, t, 1, h, d);"),
-    ("output_sums_keys", "acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);",
-     "acc += Pt[s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);"),
+    ("output_sums_keys", "acc += Pt[s] * drop_factor(dr, bh, t, s) * qkv_at(qkv, T, C, hs, b, s, 2, h, d);",
+     "acc += Pt[s] * drop_factor(dr, bh, t, s) * qkv_at(qkv, T, C, hs, b, s, 1, h, d);"),
     ("future_leaks", "for (int s = t + 1; s < T; ++s) Pt[s] = 0.0;",
      "for (int s = t + 1; s < T; ++s) Pt[s] = (s == t + 1) ? 1e-3 : 0.0;"),
     ("softmax_jacobian_sign", "dSt[s] = Pt[s] * (dSt[s] - rowdot);", "dSt[s] = Pt[s] * (dSt[s] + rowdot);"),
@@ -28,12 +28,14 @@ MUTANTS = [
     ("dP_uses_keys",
      "acc += dyb[(size_t)t * ld_dy + d] * qkv_at(qkv, T, C, hs, b, s, 2, h, d);",
      "acc += dyb[(size_t)t * ld_dy + d] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);"),
-    ("dV_transposed_P", "acc += P[(size_t)t * (size_t)T + s] * dyb[(size_t)t * ld_dy + d];",
-     "acc += P[(size_t)s * (size_t)T + t] * dyb[(size_t)t * ld_dy + d];"),
+    ("dV_transposed_P", "acc += P[(size_t)t * (size_t)T + s] * drop_factor(&dr, b * n_head + h, t, s) *",
+     "acc += P[(size_t)s * (size_t)T + t] * drop_factor(&dr, b * n_head + h, t, s) *"),
     ("dQ_uses_queries",
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);",
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 0, h, d);"),
     ("dK_missing_scale", "dk[(size_t)s * ld_dqkv + d] = acc * scale;", "dk[(size_t)s * ld_dqkv + d] = acc;"),
+    ("dropout_scale_missing", "? 1.0 / (1.0 - dr->p) : 0.0;", "? 1.0 : 0.0;"),
+    ("dropout_mask_ignored_in_dP", "acc *= drop_factor(&dr, b * n_head + h, t, s);", "acc *= 1.0 / (1.0 - dr.p);"),
     ("band_one_key_too_many", "return t - window + 1 > 0 ? t - window + 1 : 0;", "return t - window > 0 ? t - window : 0;"),
     ("band_last_query_dropped", "return s + window - 1 < T - 1 ? s + window - 1 : T - 1;",
      "return s + window - 2 < T - 1 ? s + window - 2 : T - 1;"),
