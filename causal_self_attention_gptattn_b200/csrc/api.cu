@@ -18,6 +18,8 @@
 #include <vector>
 
 #include "gptattn.h"
+#include <cmath>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -258,13 +260,29 @@ gptattn_status check_window(int window, int T, int hs, gptattn_dtype dt, int *ke
     return GPTATTN_OK;
 }
 
+// Dropout probability -> kernel parameters (threshold floor(p * 2^32); a p so small
+// that the threshold is 0 drops nothing).  p must be in [0, 1); a bf16 dropout needs
+// the head-size-64 kernels.
+gptattn_status make_dropout(float p, unsigned long long seed, int hs, gptattn_dtype dt, DropoutParams *dp) {
+    if (!(p >= 0.f && p < 1.f)) return GPTATTN_ERR_INVALID_ARG;
+    const double x = floor((double)p * 4294967296.0);
+    dp->seed = seed;
+    dp->threshold = x >= 4294967295.0 ? 4294967295u : (uint32_t)x;
+    dp->scale = dp->threshold ? 1.f / (1.f - p) : 1.f;
+    if (dp->threshold && dt == GPTATTN_BF16 && hs != 64) return GPTATTN_ERR_UNSUPPORTED;
+    return GPTATTN_OK;
+}
+
 gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, int window,
-                        gptattn_dtype dt, gptattn_stream_t stream) {
+                        float dropout_p, unsigned long long seed, gptattn_dtype dt, gptattn_stream_t stream) {
     int hs = 0;
     gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
     if (st != GPTATTN_OK) return st;
     int kw = kCausalWindow;
     st = check_window(window, T, hs, dt, &kw);
+    if (st != GPTATTN_OK) return st;
+    DropoutParams dp{};
+    st = make_dropout(dropout_p, seed, hs, dt, &dp);
     if (st != GPTATTN_OK) return st;
     if (B == 0 || T == 0) return GPTATTN_OK;
     if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
@@ -274,7 +292,7 @@ gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int 
     if (dt == GPTATTN_F32) {
         return from_cuda(run_kernel(kKFwdF32, s, [&] {
             return launch_fwd_f32(hs, static_cast<const float *>(qkv), static_cast<float *>(y), lse, B, T, C, n_head, kw,
-                                  s);
+                                  dp, s);
         }));
     }
     int *status = nullptr;
@@ -284,7 +302,7 @@ gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int 
     if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&my, y, C, T, B)) return GPTATTN_ERR_CUDA;
     const DevCtx ctx{status, kDefaultBudgetNs};
     return from_cuda(
-        run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, kw, ctx, s); }));
+        run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, kw, dp, ctx, s); }));
 }
 }  // namespace
 
@@ -300,12 +318,15 @@ gptattn_status check_det(int B, int T, int n_head, int hs, gptattn_dtype dt) {
 
 gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv, void *workspace,
                         size_t workspace_bytes, int B, int T, int C, int n_head, int window, bool det,
-                        gptattn_dtype dt, gptattn_stream_t stream) {
+                        float dropout_p, unsigned long long seed, gptattn_dtype dt, gptattn_stream_t stream) {
     int hs = 0;
     gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
     if (st != GPTATTN_OK) return st;
     int kw = kCausalWindow;
     st = check_window(window, T, hs, dt, &kw);
+    if (st != GPTATTN_OK) return st;
+    DropoutParams dp{};
+    st = make_dropout(dropout_p, seed, hs, dt, &dp);
     if (st != GPTATTN_OK) return st;
     if (det && (st = check_det(B, T, n_head, hs, dt)) != GPTATTN_OK) return st;
     if (B == 0 || T == 0) return GPTATTN_OK;
@@ -327,10 +348,10 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
         cudaError_t e = run_kernel(kKBwdPreF32, s, [&] { return launch_bwd_f32_pre(hs, fy, fg, D, B, T, C, n_head, s); });
         if (e == cudaSuccess)
             e = run_kernel(kKBwdDqF32, s,
-                           [&] { return launch_bwd_f32_dq(hs, fq, fg, lse, D, fo, B, T, C, n_head, kw, s); });
+                           [&] { return launch_bwd_f32_dq(hs, fq, fg, lse, D, fo, B, T, C, n_head, kw, dp, s); });
         if (e == cudaSuccess)
             e = run_kernel(kKBwdDkvF32, s,
-                           [&] { return launch_bwd_f32_dkv(hs, fq, fg, lse, D, fo, B, T, C, n_head, kw, s); });
+                           [&] { return launch_bwd_f32_dkv(hs, fq, fg, lse, D, fo, B, T, C, n_head, kw, dp, s); });
         return from_cuda(e);
     }
 
@@ -352,7 +373,8 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
     });
     if (e == cudaSuccess)
         e = run_kernel(kKBwdMainBf16, s, [&] {
-            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, kw, n_slots, ctx, s);
+            return launch_bwd_main_bf16(hs, mq, mdy, mdqkv, mdq, lse2, D, B, T, C, n_head, T_pad, kw, n_slots, dp, ctx,
+                                        s);
         });
     if (e == cudaSuccess)
         e = run_kernel(kKBwdPostBf16, s, [&] {
@@ -384,12 +406,12 @@ const char *gptattn_last_error_string(void) { return t_last_error; }
 
 gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, gptattn_dtype dt,
                            gptattn_stream_t stream) {
-    return fwd_impl(qkv, y, lse, B, T, C, n_head, kCausalWindow, dt, stream);
+    return fwd_impl(qkv, y, lse, B, T, C, n_head, kCausalWindow, 0.f, 0, dt, stream);
 }
 
 gptattn_status gptattn_fwd_window(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head, int window,
                                   gptattn_dtype dt, gptattn_stream_t stream) {
-    return fwd_impl(qkv, y, lse, B, T, C, n_head, window, dt, stream);
+    return fwd_impl(qkv, y, lse, B, T, C, n_head, window, 0.f, 0, dt, stream);
 }
 
 gptattn_status gptattn_decode(const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C, int n_head,
@@ -419,14 +441,15 @@ size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtyp
 gptattn_status gptattn_bwd(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
                            void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, gptattn_dtype dt,
                            gptattn_stream_t stream) {
-    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, kCausalWindow, false, dt,
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, kCausalWindow, false, 0.f, 0, dt,
                     stream);
 }
 
 gptattn_status gptattn_bwd_window(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
                                   void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, int window,
                                   gptattn_dtype dt, gptattn_stream_t stream) {
-    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, false, dt, stream);
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, false, 0.f, 0, dt,
+                    stream);
 }
 
 size_t gptattn_bwd_det_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt) {
@@ -440,7 +463,57 @@ size_t gptattn_bwd_det_workspace_bytes(int B, int T, int C, int n_head, gptattn_
 gptattn_status gptattn_bwd_det(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
                                void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head, int window,
                                gptattn_dtype dt, gptattn_stream_t stream) {
-    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, true, dt, stream);
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, true, 0.f, 0, dt,
+                    stream);
+}
+
+// Options: a zero-initialised struct (or NULL) is the plain causal call.
+static gptattn_status read_opts(const gptattn_options *o, int *window, float *p, unsigned long long *seed, bool *det) {
+    *window = kCausalWindow;
+    *p = 0.f;
+    *seed = 0;
+    *det = false;
+    if (!o) return GPTATTN_OK;
+    if (o->window < 0) return GPTATTN_ERR_INVALID_ARG;
+    if (o->window > 0) *window = o->window;
+    *p = o->dropout_p;
+    *seed = o->dropout_seed;
+    *det = o->deterministic != 0;
+    return GPTATTN_OK;
+}
+
+gptattn_status gptattn_fwd_opts(const void *qkv, void *y, float *lse, int B, int T, int C, int n_head,
+                                const gptattn_options *opts, gptattn_dtype dt, gptattn_stream_t stream) {
+    int window;
+    float p;
+    unsigned long long seed;
+    bool det;
+    gptattn_status st = read_opts(opts, &window, &p, &seed, &det);
+    if (st != GPTATTN_OK) return st;
+    return fwd_impl(qkv, y, lse, B, T, C, n_head, window, p, seed, dt, stream);
+}
+
+size_t gptattn_bwd_opts_workspace_bytes(int B, int T, int C, int n_head, const gptattn_options *opts,
+                                        gptattn_dtype dt) {
+    int window;
+    float p;
+    unsigned long long seed;
+    bool det;
+    if (read_opts(opts, &window, &p, &seed, &det) != GPTATTN_OK) return (size_t)-1;
+    return det ? gptattn_bwd_det_workspace_bytes(B, T, C, n_head, dt) : gptattn_bwd_workspace_bytes(B, T, C, n_head, dt);
+}
+
+gptattn_status gptattn_bwd_opts(const void *qkv, const void *y, const float *lse, const void *dy, void *dqkv,
+                                void *workspace, size_t workspace_bytes, int B, int T, int C, int n_head,
+                                const gptattn_options *opts, gptattn_dtype dt, gptattn_stream_t stream) {
+    int window;
+    float p;
+    unsigned long long seed;
+    bool det;
+    gptattn_status st = read_opts(opts, &window, &p, &seed, &det);
+    if (st != GPTATTN_OK) return st;
+    return bwd_impl(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, window, det, p, seed, dt,
+                    stream);
 }
 
 gptattn_status gptattn_get_device_status(gptattn_stream_t stream) {

@@ -14,6 +14,9 @@
 // accumulator with TMA reduce-adds (whose order across CTAs varies run to run),
 // each (query tile i, key tile j) partial is stored in its own slot i(i+1)/2 + j
 // and the postprocess kernel sums the slots of a query tile in a fixed order.
+// Dropout (inverted dropout on the weights, Philox mask of philox.cuh): the
+// P^T stored for dV is the dropped, rescaled weight, and dS = P o (dP o f - D)
+// with f = 1/(1-p) for kept weights, 0 for dropped ones.
 //
 // Schedule: one persistent CTA per SM walks a static list of work items
 // (key tile j, batch b, head h), ordered longest first (small j first), in a
@@ -35,6 +38,8 @@
 // registers, so the tensor pipe computes tile i+1 while tile i is in softmax.
 // Every wait is bounded; roles never leave their loops early, so all named
 // barriers are reached the same number of times by every thread of a role.
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -111,11 +116,12 @@ __device__ __forceinline__ int item_index(int k, int cta, int grid) {
     return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
 }
 
+template <bool kDropout>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_h64_persistent(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
                        const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
                        const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C,
-                       int n_head, int T_pad, int n_t, int window, int n_slots, int *status,
+                       int n_head, int T_pad, int n_t, int window, int n_slots, DropoutParams dp, int *status,
                        unsigned long long budget_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -345,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) ok = warp_wait(bar(kBarQFull + st), (uint32_t)(gi / kQStages) & 1u, g);
                 if (ok) ok = warp_wait(bar(kBarSFull), ph, g);
                 float pf[64];  // P^T row segment, fp32
+                uint32_t keepb[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};  // dropout keep bits of the 64 columns
                 if (ok) {
                     tc_fence_after();
                     uint32_t sr[64];
@@ -381,8 +388,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (c >= cut) pf[c] = 0.f;
                     }
                     uint32_t pk[32];
+                    if constexpr (kDropout) {  // keep bits of this row's 64 columns; P^T dropped + rescaled
+                        const uint32_t skey = (uint32_t)(kt * kTile + row);
+                        keepb[0] = keepb[1] = 0u;
+#pragma unroll 4
+                        for (int c = 0; c < 64; ++c) {
+                            const uint32_t tq = (uint32_t)((kt + it) * kTile + 64 * half + c);
+                            const uint32_t bits = dropout_keep4(dp.seed, dp.threshold, (uint32_t)bh, tq, skey & ~3u);
+                            keepb[c >> 5] |= ((bits >> (skey & 3u)) & 1u) << (c & 31);
+                        }
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
+                        for (int c = 0; c < 32; ++c) {
+                            const float f0 = ((keepb[(2 * c) >> 5] >> ((2 * c) & 31)) & 1u) ? dp.scale : 0.f;
+                            const float f1 = ((keepb[(2 * c + 1) >> 5] >> ((2 * c + 1) & 31)) & 1u) ? dp.scale : 0.f;
+                            pk[c] = pack_bf16x2(pf[2 * c] * f0, pf[2 * c + 1] * f1);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]);
+                    }
                     if (gi > 0) ok = warp_wait(bar(kBarPEmpty), (uint32_t)(gi - 1) & 1u, g);
                     if (ok) {
                         tmem_st_x32(trow + kColP + 32 * half, pk);
@@ -406,29 +430,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_before();
                             mbar_arrive(bar(kBardPEmpty));
                         }
+                        // dS^T = P^T o (dP^T o f - D); f = 1 without dropout
+                        auto ds_chunk = [&](auto drop_tag) {
+                            constexpr bool kDrop = decltype(drop_tag)::value;
 #pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            const int q = 4 * part + qq;  // 16-byte chunk = 8 query columns
-                            uint32_t wv[4];
+                            for (int qq = 0; qq < 4; ++qq) {
+                                const int q = 4 * part + qq;  // 16-byte chunk = 8 query columns
+                                uint32_t wv[4];
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const float4 d = D4[2 * q + e];
-                                const int c = 8 * q + 4 * e;      // column within the half
-                                const int cr = 8 * qq + 4 * e;    // column within this dP chunk
-                                const uint64_t a01 = fadd2(f32x2_pack(__uint_as_float(dr[cr]), __uint_as_float(dr[cr + 1])),
-                                                           f32x2_pack(d.x, d.y));
-                                const uint64_t a23 = fadd2(f32x2_pack(__uint_as_float(dr[cr + 2]), __uint_as_float(dr[cr + 3])),
-                                                           f32x2_pack(d.z, d.w));
-                                const uint64_t s01 = fmul2(a01, f32x2_pack(pf[c], pf[c + 1]));
-                                const uint64_t s23 = fmul2(a23, f32x2_pack(pf[c + 2], pf[c + 3]));
-                                float s0, s1, s2, s3;
-                                f32x2_unpack(s01, s0, s1);
-                                f32x2_unpack(s23, s2, s3);
-                                wv[2 * e] = pack_bf16x2(s0, s1);
-                                wv[2 * e + 1] = pack_bf16x2(s2, s3);
+                                for (int e = 0; e < 2; ++e) {
+                                    const float4 d = D4[2 * q + e];
+                                    const int c = 8 * q + 4 * e;      // column within the half
+                                    const int cr = 8 * qq + 4 * e;    // column within this dP chunk
+                                    uint64_t g01 = f32x2_pack(__uint_as_float(dr[cr]), __uint_as_float(dr[cr + 1]));
+                                    uint64_t g23 = f32x2_pack(__uint_as_float(dr[cr + 2]), __uint_as_float(dr[cr + 3]));
+                                    if constexpr (kDrop) {
+                                        auto fac = [&](int cc) {
+                                            return ((keepb[cc >> 5] >> (cc & 31)) & 1u) ? dp.scale : 0.f;
+                                        };
+                                        g01 = fmul2(g01, f32x2_pack(fac(c), fac(c + 1)));
+                                        g23 = fmul2(g23, f32x2_pack(fac(c + 2), fac(c + 3)));
+                                    }
+                                    const uint64_t a01 = fadd2(g01, f32x2_pack(d.x, d.y));
+                                    const uint64_t a23 = fadd2(g23, f32x2_pack(d.z, d.w));
+                                    const uint64_t s01 = fmul2(a01, f32x2_pack(pf[c], pf[c + 1]));
+                                    const uint64_t s23 = fmul2(a23, f32x2_pack(pf[c + 2], pf[c + 3]));
+                                    float s0, s1, s2, s3;
+                                    f32x2_unpack(s01, s0, s1);
+                                    f32x2_unpack(s23, s2, s3);
+                                    wv[2 * e] = pack_bf16x2(s0, s1);
+                                    wv[2 * e + 1] = pack_bf16x2(s2, s3);
+                                }
+                                st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), wv[0], wv[1], wv[2],
+                                             wv[3]);
                             }
-                            st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), wv[0], wv[1], wv[2], wv[3]);
-                        }
+                        };
+                        ds_chunk(std::integral_constant<bool, kDropout>{});
                     }
                     fence_proxy_async_smem();
                     mbar_arrive(bar(kBardSFull));
@@ -529,8 +566,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                                int n_head, int T_pad, int window, int n_slots, DevCtx ctx, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_h64_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int n_head, int T_pad, int window, int n_slots, DropoutParams dp, DevCtx ctx,
+                                cudaStream_t s) {
+    auto kern = dp.threshold != 0u ? bwd_h64_persistent<true> : bwd_h64_persistent<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
@@ -540,8 +579,8 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
     const int n_t = ceil_div(T, kTile);
     const long long items = (long long)n_t * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    return launch_pdl(bwd_h64_persistent, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_dy, map_dqkv,
-                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, ctx.status, ctx.budget_ns);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_dy, map_dqkv,
+                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, dp, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

@@ -578,11 +578,11 @@ cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const flo
 cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
                                  const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
                                  const float *D, int B, int T, int C, int n_head, int T_pad, int window, int n_slots,
-                                 DevCtx ctx, cudaStream_t s) {
+                                 DropoutParams dp, DevCtx ctx, cudaStream_t s) {
     if (hs == 64)
         return launch_bwd_main_h64(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots,
-                                   ctx, s);
-    if (hs == 128 && window >= T && n_slots == 0)
+                                   dp, ctx, s);
+    if (hs == 128 && window >= T && n_slots == 0 && dp.threshold == 0u)
         return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
     return cudaErrorInvalidValue;
 }

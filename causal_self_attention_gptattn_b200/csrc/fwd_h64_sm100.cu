@@ -22,7 +22,13 @@
 // attention): query t sees keys t-window < s <= t; key tiles below a query
 // tile's band are skipped, and the band's lower edge is masked element-wise
 // like the diagonal.  window >= T is the causal case.
+// Dropout (lecture chapter "adding dropout", read as inverted dropout on the
+// weights): P goes into TMEM with dropped weights zeroed (Philox mask, see
+// philox.cuh); l and the rounded-weight sum stay those of the undropped weights,
+// and the epilogue scales y by 1/(1-p).
 // Every barrier wait is bounded; on a timeout all roles stop, drain and exit.
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -80,10 +86,11 @@ __device__ __forceinline__ int item_index(int k, int cta, int grid) {
     return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
 }
 
+template <bool kDropout>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_h64_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
-                   float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, int *status,
-                   unsigned long long budget_ns) {
+                   float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, DropoutParams dp,
+                   int *status, unsigned long long budget_ns) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -351,18 +358,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int a = 0; a < 4; ++a) sum2[a] = sumr2[a] = f32x2_pack(0.f, 0.f);
                 uint32_t pk[64];
+                // the exponentials; with dropout the stored weights are masked, the sums are not
+                auto exps = [&](auto drop_tag) {
+                    constexpr bool kDrop = decltype(drop_tag)::value;
+                    uint32_t keep4 = 0xFu;
+                    const uint32_t t_row = (uint32_t)(qt * kTile + row);
 #pragma unroll
-                for (int c = 0; c < 128; c += 2) {
-                    const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
-                    float x0, x1;
-                    f32x2_unpack(x, x0, x1);
-                    const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                    const uint32_t wv = pack_bf16x2(p0, p1);
-                    pk[c >> 1] = wv;
-                    const int a = (c >> 1) & 3;
-                    sum2[a] = fadd2(sum2[a], f32x2_pack(p0, p1));
-                    sumr2[a] = fadd2(sumr2[a], f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
-                }
+                    for (int c = 0; c < 128; c += 2) {
+                        if constexpr (kDrop) {
+                            if ((c & 3) == 0)
+                                keep4 = dropout_keep4(dp.seed, dp.threshold, (uint32_t)bh, t_row, (uint32_t)(j * kTile + c));
+                        }
+                        const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
+                        float x0, x1;
+                        f32x2_unpack(x, x0, x1);
+                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                        const uint32_t wv = pack_bf16x2(p0, p1);
+                        if constexpr (kDrop) {
+                            const uint32_t m = (((keep4 >> (c & 3)) & 1u) ? 0x0000FFFFu : 0u) |
+                                               (((keep4 >> ((c + 1) & 3)) & 1u) ? 0xFFFF0000u : 0u);
+                            pk[c >> 1] = wv & m;
+                        } else {
+                            pk[c >> 1] = wv;
+                        }
+                        const int a = (c >> 1) & 3;
+                        sum2[a] = fadd2(sum2[a], f32x2_pack(p0, p1));
+                        sumr2[a] = fadd2(sumr2[a], f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                    }
+                };
+                exps(std::integral_constant<bool, kDropout>{});
                 float s0, s1, r0, r1;
                 f32x2_unpack(fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3])), s0, s1);
                 f32x2_unpack(fadd2(fadd2(sumr2[0], sumr2[1]), fadd2(sumr2[2], sumr2[3])), r0, r1);
@@ -401,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_x32(tO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                 tc_fence_before();
                 mbar_arrive(bar(kBarOFree + t));
-                const float inv_l = 1.f / l_r;
+                const float inv_l = (kDropout ? dp.scale : 1.f) / l_r;  // 1/(1-p) with dropout
                 const uint32_t rbase = stg + (uint32_t)row * 128u;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -440,8 +464,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace
 
 cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
-                           int n_head, int window, DevCtx ctx, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_h64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+                           int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
+    auto kern = dp.threshold != 0u ? fwd_h64_kernel<true> : fwd_h64_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
@@ -450,8 +475,8 @@ cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y,
     const int n_qt = ceil_div(T, kTile);
     const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    return launch_pdl(fwd_h64_kernel, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_y, lse, B, T, C,
-                      n_head, n_qt, window, ctx.status, ctx.budget_ns);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_y, lse, B, T, C,
+                      n_head, n_qt, window, dp, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace gptattn

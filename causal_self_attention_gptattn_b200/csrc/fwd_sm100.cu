@@ -462,9 +462,10 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
 }  // namespace
 
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T,
-                            int C, int n_head, int window, DevCtx ctx, cudaStream_t s) {
-    if (hs == 64) return launch_fwd_h64(map_qkv, map_y, lse, B, T, C, n_head, window, ctx, s);
-    if (hs == 128 && window >= T) return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, ctx, s);
+                            int C, int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
+    if (hs == 64) return launch_fwd_h64(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s);
+    if (hs == 128 && window >= T && dp.threshold == 0u)
+        return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, ctx, s);
     return cudaErrorInvalidValue;
 }
 

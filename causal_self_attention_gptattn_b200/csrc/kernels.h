@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "philox.cuh"
+
 namespace gptattn {
 
 // Per-launch device context: where a kernel records a timeout, and how long
@@ -51,11 +53,12 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // window: query t sees keys t-window < s <= t (kCausalWindow or any value >= T: causal);
 // the head-size-128 kernels support the causal case only.
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse,
-                            int B, int T, int C, int n_head, int window, DevCtx ctx, cudaStream_t s);
+                            int B, int T, int C, int n_head, int window, DropoutParams dp, DevCtx ctx,
+                            cudaStream_t s);
 
 // Head-size-64 forward with separate P buffers (same arguments as above).
 cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
-                           int n_head, int window, DevCtx ctx, cudaStream_t s);
+                           int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s);
 
 // D[bh][t] = sum_d y*dy, lse2[bh][t] = lse*log2(e) (rows t >= T: 0 and +inf),
 // dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].
@@ -67,12 +70,13 @@ cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const flo
 cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_dy,
                                  const CUtensorMap &map_dqkv, const CUtensorMap &map_dq, const float *lse2,
                                  const float *D, int B, int T, int C, int n_head, int T_pad, int window, int n_slots,
-                                 DevCtx ctx, cudaStream_t s);
+                                 DropoutParams dp, DevCtx ctx, cudaStream_t s);
 
 // Persistent head-size-64 variant of the above (same arguments).
 cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                                int n_head, int T_pad, int window, int n_slots, DevCtx ctx, cudaStream_t s);
+                                int n_head, int T_pad, int window, int n_slots, DropoutParams dp, DevCtx ctx,
+                                cudaStream_t s);
 
 // dqkv[b][t][h*hs+d] = bf16(dqacc[(b*n_head+h)*T_pad + t][d] / sqrt(hs)).
 cudaError_t launch_bwd_post_bf16(int hs, const float *dqacc, void *dqkv, int B, int T, int C, int n_head,
@@ -86,13 +90,15 @@ cudaError_t launch_bwd_post_det_bf16(int hs, const float *part, void *dqkv, int 
 
 // ---- fp32 CUDA-core path --------------------------------------------------
 cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,
-                           cudaStream_t s);
+                           DropoutParams dp, cudaStream_t s);
 cudaError_t launch_bwd_f32_pre(int hs, const float *y, const float *dy, float *D, int B, int T, int C,
                                int n_head, cudaStream_t s);
 cudaError_t launch_bwd_f32_dq(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
-                              float *dqkv, int B, int T, int C, int n_head, int window, cudaStream_t s);
+                              float *dqkv, int B, int T, int C, int n_head, int window, DropoutParams dp,
+                              cudaStream_t s);
 cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
-                               float *dqkv, int B, int T, int C, int n_head, int window, cudaStream_t s);
+                               float *dqkv, int B, int T, int C, int n_head, int window, DropoutParams dp,
+                               cudaStream_t s);
 
 // ---- decode: last position over a key/value cache (cluster of 8 CTAs per (b, h))
 cudaError_t launch_decode(int hs, bool bf16, const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C,

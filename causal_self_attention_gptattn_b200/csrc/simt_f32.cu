@@ -11,9 +11,18 @@
 // rows are staged through shared memory in tiles of kRows.  Deterministic: no
 // atomics.  Accurate expf/logf (no approximate intrinsics).
 #include "kernels.h"
+#include "philox.cuh"
 
 namespace gptattn {
 namespace {
+
+// Dropout factor of the weight of query t for key s: 1 without dropout, else
+// 1/(1-p) if the Philox mask keeps it and 0 if not.
+__device__ __forceinline__ float drop_factor(const DropoutParams &dp, int bh, int t, int s) {
+    if (dp.threshold == 0u) return 1.f;
+    const uint32_t bits = dropout_keep4(dp.seed, dp.threshold, (uint32_t)bh, (uint32_t)t, (uint32_t)(s & ~3));
+    return ((bits >> (s & 3)) & 1u) ? dp.scale : 0.f;
+}
 
 constexpr int kRows = 64;  // threads per block = rows per staged tile
 
@@ -25,10 +34,12 @@ __device__ __forceinline__ float dot_row(const float *a, const float *b) {
     return acc;
 }
 
-// y[b,t,h*HS+d] and lse[b,h,t] for query rows of one (b, h).
+// y[b,t,h*HS+d] and lse[b,h,t] for query rows of one (b, h); the weights are
+// dropped (and rescaled) in the weighted sum only, lse is the undropped one.
 template <int HS>
 __global__ void __launch_bounds__(kRows) fwd_f32_kernel(const float *__restrict__ qkv, float *__restrict__ y,
-                                                        float *__restrict__ lse, int T, int C, int n_head, int window) {
+                                                        float *__restrict__ lse, int T, int C, int n_head, int window,
+                                                        DropoutParams dp) {
     extern __shared__ float sm[];
     float *sk = sm;              // [kRows][HS]
     float *sv = sm + kRows * HS;  // [kRows][HS]
@@ -68,8 +79,9 @@ __global__ void __launch_bounds__(kRows) fwd_f32_kernel(const float *__restrict_
                 const float corr = expf(m - m_new);
                 const float p = expf(sc - m_new);
                 l = l * corr + p;
+                const float pd = p * drop_factor(dp, bh, t, s0 + r);
 #pragma unroll
-                for (int d = 0; d < HS; ++d) acc[d] = fmaf(acc[d], corr, p * sv[r * HS + d]);
+                for (int d = 0; d < HS; ++d) acc[d] = fmaf(acc[d], corr, pd * sv[r * HS + d]);
                 m = m_new;
             }
         }
@@ -107,7 +119,7 @@ template <int HS>
 __global__ void __launch_bounds__(kRows) bwd_f32_dq_kernel(const float *__restrict__ qkv, const float *__restrict__ dy,
                                                            const float *__restrict__ lse, const float *__restrict__ D,
                                                            float *__restrict__ dqkv, int T, int C, int n_head,
-                                                           int window) {
+                                                           int window, DropoutParams dp) {
     extern __shared__ float sm[];
     float *sk = sm;
     float *sv = sm + kRows * HS;
@@ -149,7 +161,7 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dq_kernel(const float *__restri
             const int smax = min(kRows, t - s0 + 1);
             for (int r = max(0, lo_t - s0); r < smax; ++r) {
                 const float p = expf(dot_row<HS>(q, sk + r * HS) - lse_t);
-                const float ds = p * (dot_row<HS>(g, sv + r * HS) - D_t);
+                const float ds = p * (dot_row<HS>(g, sv + r * HS) * drop_factor(dp, bh, t, s0 + r) - D_t);
 #pragma unroll
                 for (int d = 0; d < HS; ++d) acc[d] = fmaf(ds, sk[r * HS + d], acc[d]);
             }
@@ -167,7 +179,7 @@ template <int HS>
 __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restrict__ qkv, const float *__restrict__ dy,
                                                             const float *__restrict__ lse, const float *__restrict__ D,
                                                             float *__restrict__ dqkv, int T, int C, int n_head,
-                                                            int window) {
+                                                            int window, DropoutParams dp) {
     extern __shared__ float sm[];
     float *sq = sm;                   // [kRows][HS] queries (pre-scaled)
     float *sg = sm + kRows * HS;      // [kRows][HS] dy rows
@@ -214,10 +226,12 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restr
             const int rmax = (int)min((long long)min(kRows, T - t0), (long long)s + window - t0);  // t < s + window
             for (int r = rmin; r < rmax; ++r) {
                 const float p = expf(dot_row<HS>(sq + r * HS, k) - sl[r]);
-                const float ds = p * (dot_row<HS>(sg + r * HS, v) - sD[r]);
+                const float f = drop_factor(dp, bh, t0 + r, s);
+                const float ds = p * (dot_row<HS>(sg + r * HS, v) * f - sD[r]);
+                const float pd = p * f;
 #pragma unroll
                 for (int d = 0; d < HS; ++d) {
-                    dv[d] = fmaf(p, sg[r * HS + d], dv[d]);
+                    dv[d] = fmaf(pd, sg[r * HS + d], dv[d]);
                     dk[d] = fmaf(ds, sq[r * HS + d], dk[d]);  // sq already carries one factor of scale
                 }
             }
@@ -235,30 +249,30 @@ __global__ void __launch_bounds__(kRows) bwd_f32_dkv_kernel(const float *__restr
 
 template <int HS>
 cudaError_t launch_fwd_t(const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,
-                         cudaStream_t s) {
+                         DropoutParams dp, cudaStream_t s) {
     const size_t smem = 2 * kRows * HS * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fwd_f32_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, y, lse, T, C, n_head, window);
+    fwd_f32_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, y, lse, T, C, n_head, window, dp);
     return cudaGetLastError();
 }
 template <int HS>
 cudaError_t launch_dq_t(const float *qkv, const float *dy, const float *lse, const float *D, float *dqkv, int B, int T,
-                        int C, int n_head, int window, cudaStream_t s) {
+                        int C, int n_head, int window, DropoutParams dp, cudaStream_t s) {
     const size_t smem = 2 * kRows * HS * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_f32_dq_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    bwd_f32_dq_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, dy, lse, D, dqkv, T, C, n_head, window);
+    bwd_f32_dq_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, dy, lse, D, dqkv, T, C, n_head, window, dp);
     return cudaGetLastError();
 }
 template <int HS>
 cudaError_t launch_dkv_t(const float *qkv, const float *dy, const float *lse, const float *D, float *dqkv, int B, int T,
-                         int C, int n_head, int window, cudaStream_t s) {
+                         int C, int n_head, int window, DropoutParams dp, cudaStream_t s) {
     const size_t smem = (2 * kRows * HS + 2 * kRows) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(bwd_f32_dkv_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     bwd_f32_dkv_kernel<HS><<<dim3(ceil_div(T, kRows), B * n_head), kRows, smem, s>>>(qkv, dy, lse, D, dqkv, T, C,
-                                                                                     n_head, window);
+                                                                                     n_head, window, dp);
     return cudaGetLastError();
 }
 
@@ -274,8 +288,8 @@ cudaError_t launch_dkv_t(const float *qkv, const float *dy, const float *lse, co
 }  // namespace
 
 cudaError_t launch_fwd_f32(int hs, const float *qkv, float *y, float *lse, int B, int T, int C, int n_head, int window,
-                           cudaStream_t s) {
-#define CALL(H) launch_fwd_t<H>(qkv, y, lse, B, T, C, n_head, window, s)
+                           DropoutParams dp, cudaStream_t s) {
+#define CALL(H) launch_fwd_t<H>(qkv, y, lse, B, T, C, n_head, window, dp, s)
     GPTATTN_HS_DISPATCH(hs, CALL)
 #undef CALL
 }
@@ -292,15 +306,16 @@ cudaError_t launch_bwd_f32_pre(int hs, const float *y, const float *dy, float *D
 }
 
 cudaError_t launch_bwd_f32_dq(int hs, const float *qkv, const float *dy, const float *lse, const float *D, float *dqkv,
-                              int B, int T, int C, int n_head, int window, cudaStream_t s) {
-#define CALL(H) launch_dq_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, window, s)
+                              int B, int T, int C, int n_head, int window, DropoutParams dp, cudaStream_t s) {
+#define CALL(H) launch_dq_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, window, dp, s)
     GPTATTN_HS_DISPATCH(hs, CALL)
 #undef CALL
 }
 
 cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const float *lse, const float *D,
-                               float *dqkv, int B, int T, int C, int n_head, int window, cudaStream_t s) {
-#define CALL(H) launch_dkv_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, window, s)
+                               float *dqkv, int B, int T, int C, int n_head, int window, DropoutParams dp,
+                               cudaStream_t s) {
+#define CALL(H) launch_dkv_t<H>(qkv, dy, lse, D, dqkv, B, T, C, n_head, window, dp, s)
     GPTATTN_HS_DISPATCH(hs, CALL)
 #undef CALL
 }

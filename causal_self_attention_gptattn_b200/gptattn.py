@@ -29,11 +29,17 @@ GPTATTN_BF16 = 1
 # Every symbol include/gptattn.h declares.
 EXPORTED = (
     "gptattn_fwd", "gptattn_fwd_window", "gptattn_bwd_window", "gptattn_bwd_det_workspace_bytes", "gptattn_bwd_det",
-    "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
+    "gptattn_fwd_opts", "gptattn_bwd_opts_workspace_bytes", "gptattn_bwd_opts", "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
     "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
     "gptattn_last_error_string",
 )
+
+
+class Options(ctypes.Structure):
+    """gptattn_options: window (0 = causal), dropout_p, dropout_seed, deterministic."""
+    _fields_ = [("window", ctypes.c_int), ("dropout_p", ctypes.c_float), ("dropout_seed", ctypes.c_ulonglong),
+                ("deterministic", ctypes.c_int)]
 
 
 class LibraryNotBuilt(RuntimeError):
@@ -81,6 +87,13 @@ def lib():
             L.gptattn_bwd_det_workspace_bytes.restype = sz
             L.gptattn_bwd_det.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, st]
             L.gptattn_bwd_det.restype = i
+            op = ctypes.POINTER(Options)
+            L.gptattn_fwd_opts.argtypes = [vp, vp, vp, i, i, i, i, op, i, st]
+            L.gptattn_fwd_opts.restype = i
+            L.gptattn_bwd_opts_workspace_bytes.argtypes = [i, i, i, i, op, i]
+            L.gptattn_bwd_opts_workspace_bytes.restype = sz
+            L.gptattn_bwd_opts.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, op, i, st]
+            L.gptattn_bwd_opts.restype = i
             L.gptattn_decode.argtypes = [vp, vp, vp, i, i, i, i, i, i, st]
             L.gptattn_decode.restype = i
             L.gptattn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
@@ -149,6 +162,24 @@ def gptattn_bwd_det(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, 
                     stream=None) -> int:
     return lib().gptattn_bwd_det(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), _ptr(workspace),
                                  workspace_bytes, B, T, C, n_head, window, dt, _stream(stream))
+
+
+def _opts(opts):
+    return None if opts is None else ctypes.byref(opts)
+
+
+def gptattn_fwd_opts(qkv, y, lse, B, T, C, n_head, opts, dt, stream=None) -> int:
+    return lib().gptattn_fwd_opts(_ptr(qkv), _ptr(y), _ptr(lse), B, T, C, n_head, _opts(opts), dt, _stream(stream))
+
+
+def gptattn_bwd_opts_workspace_bytes(B, T, C, n_head, opts, dt) -> int:
+    return lib().gptattn_bwd_opts_workspace_bytes(B, T, C, n_head, _opts(opts), dt)
+
+
+def gptattn_bwd_opts(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C, n_head, opts, dt,
+                     stream=None) -> int:
+    return lib().gptattn_bwd_opts(_ptr(qkv), _ptr(y), _ptr(lse), _ptr(dy), _ptr(dqkv), _ptr(workspace),
+                                  workspace_bytes, B, T, C, n_head, _opts(opts), dt, _stream(stream))
 
 
 def gptattn_decode(qkv, y, lse, B, T, T_cap, C, n_head, dt, stream=None) -> int:

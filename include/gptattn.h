@@ -121,6 +121,40 @@ GPTATTN_API gptattn_status gptattn_bwd_det(const void *qkv, const void *y, const
                                int B, int T, int C, int n_head, int window,
                                gptattn_dtype dt, gptattn_stream_t stream);
 
+/* Options for the general entry points below.  A zero-initialised struct (or
+ * a NULL pointer) is the plain causal call of gptattn_fwd / gptattn_bwd.
+ *   window        0: causal; > 0: local window as in gptattn_fwd_window; < 0: invalid.
+ *   dropout_p     probability of dropping an attention weight, 0 <= p < 1 (else
+ *                 GPTATTN_ERR_INVALID_ARG).  Inverted dropout on the weights after
+ *                 the softmax (the lecture page's chapter "scaling up the model! ...
+ *                 adding dropout"): a kept weight is scaled by 1/(1-p); lse stays
+ *                 the logsumexp of the undropped scores.  Weight (t, s) of batch b,
+ *                 head h is kept iff word s%4 of Philox4x32-10 (Salmon et al.,
+ *                 SC 2011) at counter (s/4, t, b*n_head+h, 0) under key
+ *                 (seed & 0xffffffff, seed >> 32) is >= floor(p * 2^32); p < 2^-32
+ *                 drops nothing.  The backward must get the forward's seed and p.
+ *                 bf16 dropout needs head size 64.
+ *   dropout_seed  the 64-bit Philox key.
+ *   deterministic backward only: bit-identical results as gptattn_bwd_det (and
+ *                 its workspace size). */
+typedef struct gptattn_options {
+    int window;
+    float dropout_p;
+    unsigned long long dropout_seed;
+    int deterministic;
+} gptattn_options;
+
+GPTATTN_API gptattn_status gptattn_fwd_opts(const void *qkv, void *y, float *lse,
+                                int B, int T, int C, int n_head, const gptattn_options *opts,
+                                gptattn_dtype dt, gptattn_stream_t stream);
+/* Workspace for gptattn_bwd_opts with these options ((size_t)-1 if unsupported/invalid). */
+GPTATTN_API size_t gptattn_bwd_opts_workspace_bytes(int B, int T, int C, int n_head, const gptattn_options *opts,
+                                                    gptattn_dtype dt);
+GPTATTN_API gptattn_status gptattn_bwd_opts(const void *qkv, const void *y, const float *lse, const void *dy,
+                                void *dqkv, void *workspace, size_t workspace_bytes,
+                                int B, int T, int C, int n_head, const gptattn_options *opts,
+                                gptattn_dtype dt, gptattn_stream_t stream);
+
 /* Decode: attention of the last position over a key/value cache (no
  * counterpart on the pages beyond the operation itself: it is row T-1 of
  * gptattn_fwd, the only row the pages' generate loop reads, computed without

@@ -34,9 +34,10 @@ class Guarded:
         return bool((lo == self.fill).all().item() and (hi == self.fill).all().item())
 
 
-def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream=None, window=None):
+def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream=None, window=None, opts=None):
     """Forward + backward through the C ABI (the local-window entry points when
-    window is given).  Returns float64 numpy (y, lse, dqkv)."""
+    window is given, the options entry points when opts is given).  Returns
+    float64 numpy (y, lse, dqkv)."""
     dev = torch.device("cuda", 0)
     dtype = qkv_cpu.dtype
     dt = ga.GPTATTN_BF16 if dtype == torch.bfloat16 else ga.GPTATTN_F32
@@ -47,10 +48,15 @@ def run_fwd_bwd(qkv_cpu: torch.Tensor, dy_cpu: torch.Tensor, n_head: int, stream
     y = Guarded(B * T * C, dtype, dev)
     lse = Guarded(B * n_head * T, torch.float32, dev)
     dqkv = Guarded(B * T * 3 * C, dtype, dev)
-    nbytes = ga.gptattn_bwd_workspace_bytes(B, T, C, n_head, dt)
+    nbytes = (ga.gptattn_bwd_workspace_bytes(B, T, C, n_head, dt) if opts is None
+              else ga.gptattn_bwd_opts_workspace_bytes(B, T, C, n_head, opts, dt))
     ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
     s = stream if stream is not None else torch.cuda.current_stream(dev)
-    if window is None:
+    if opts is not None:
+        ga.check(ga.gptattn_fwd_opts(qkv, y.view, lse.view, B, T, C, n_head, opts, dt, s), "gptattn_fwd_opts")
+        ga.check(ga.gptattn_bwd_opts(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, opts, dt, s),
+                 "gptattn_bwd_opts")
+    elif window is None:
         ga.check(ga.gptattn_fwd(qkv, y.view, lse.view, B, T, C, n_head, dt, s), "gptattn_fwd")
         ga.check(ga.gptattn_bwd(qkv, y.view, lse.view, dy, dqkv.view, ws, nbytes, B, T, C, n_head, dt, s),
                  "gptattn_bwd")

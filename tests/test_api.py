@@ -154,3 +154,19 @@ def test_deterministic_backward_workspace_and_validation():
     assert ga.gptattn_bwd_det(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, B, T, C, nh, 0, bf,
                               None) == ga.GPTATTN_ERR_INVALID_ARG
     assert ga.gptattn_bwd_det(None, None, None, None, None, None, 0, 0, T, C, nh, 1, bf, None) == ga.GPTATTN_OK
+
+
+def test_options_validation():
+    bf, f32 = ga.GPTATTN_BF16, ga.GPTATTN_F32
+    O = ga.Options
+    args = (2, 8, 128, 2)
+    assert ga.gptattn_fwd_opts(FAKE, FAKE, FAKE, *args, O(window=-1), bf, None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd_opts(FAKE, FAKE, FAKE, *args, O(dropout_p=1.0), bf, None) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd_opts(FAKE, FAKE, FAKE, *args, O(dropout_p=-0.1), f32, None) == ga.GPTATTN_ERR_INVALID_ARG
+    # bf16 dropout needs head size 64
+    assert ga.gptattn_fwd_opts(FAKE, FAKE, FAKE, 2, 8, 256, 2, O(dropout_p=0.1), bf, None) == ga.GPTATTN_ERR_UNSUPPORTED
+    assert ga.gptattn_fwd_opts(None, None, None, 0, 8, 128, 2, None, bf, None) == ga.GPTATTN_OK
+    assert ga.gptattn_bwd_opts_workspace_bytes(*args, None, bf) == ga.gptattn_bwd_workspace_bytes(*args, bf)
+    assert ga.gptattn_bwd_opts_workspace_bytes(*args, O(deterministic=1), bf) == \
+        ga.gptattn_bwd_det_workspace_bytes(*args, bf)
+    assert ga.gptattn_bwd_opts_workspace_bytes(*args, O(window=-2), bf) == (1 << 64) - 1
