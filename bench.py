@@ -439,6 +439,35 @@ def run_ours(args, w, rank, world, local_rank):
                "workspace_bytes": nb_det}
         del ws_det
 
+    # ---- attention dropout p = 0.1 (gptattn_fwd_opts + gptattn_bwd_opts): the same step with
+    # the Philox keep mask generated in the forward and again in the backward; FLOPs counted as
+    # for the plain step (the mask adds no matrix work).
+    drop = None
+    if not args.profile_run and (dt == ga.GPTATTN_F32 or w.hs == 64):
+        o = ga.Options(dropout_p=0.1, dropout_seed=1234)
+        nb_o = ga.gptattn_bwd_opts_workspace_bytes(B, T, C, nh, o, dt)
+
+        def step_drop():
+            ga.check(ga.gptattn_fwd_opts(qkv, y, lse, B, T, C, nh, o, dt, s), "gptattn_fwd_opts")
+            ga.check(ga.gptattn_bwd_opts(qkv, y, lse, dy, dqkv, ws, nb_o, B, T, C, nh, o, dt, s), "gptattn_bwd_opts")
+
+        for _ in range(5):
+            flush.zero_()
+            step_drop()
+        torch.cuda.synchronize()
+        Ko = max(1, min(K, 200))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ko)]
+        for a, b_ in evs:
+            flush.zero_()
+            a.record(s)
+            step_drop()
+            b_.record(s)
+        torch.cuda.synchronize()
+        to = sum(a.elapsed_time(b_) for a, b_ in evs)
+        ga.check(ga.gptattn_get_device_status(s), "device status after the dropout steps")
+        drop = {"dropout_p": 0.1, "steps": Ko, "ms_per_step": to / Ko, "value": flops * Ko / (to / 1e3) / 1e12,
+                "unit": "TFLOP/s", "flop_count": "as the plain step"}
+
     # ---- decode (gptattn_decode): the last position of every sequence over the same qkv as a
     # key/value cache; HBM-bound, so its roofline is the measured copy bandwidth.  L2 flushed
     # before every call.  Also a large cache (B=64, T=4096 at this head layout) for the
@@ -536,6 +565,7 @@ def run_ours(args, w, rank, world, local_rank):
         "decode": decode,
         "window": banded,
         "deterministic": det,
+        "dropout": drop,
         "clocks": clocks,
         "wall_s_timed": wall1 - wall0,
     }
