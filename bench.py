@@ -49,6 +49,8 @@ def parse_args():
     p.add_argument("--skip-cpu-baseline", action="store_true")
     p.add_argument("--profile-run", action="store_true",
                    help="warm-up and timed steps only (no clock sampling, e2e or CPU leg): for ncu captures")
+    p.add_argument("--block-run", action="store_true",
+                   help="only the attention sub-block call, warm-up + steps times: for ncu captures of its kernels")
     return p.parse_args()
 
 
@@ -204,6 +206,28 @@ def run_reference(args, w, rank):
 
 
 # --------------------------------------------------------------------------- GPU arm
+def make_block_call(ga, w, dev, s):
+    """Device buffers of the pre-LN attention sub-block at the workload's B, T, C (seeded
+    inputs) and a closure that enqueues one gptattn_attn_block_fwd call on stream s."""
+    import torch
+
+    from causal_self_attention_gptattn_b200.workloads import block_inputs
+    B, T, C, nh = w.B, w.T, w.C, w.n_head
+    xb_c, pb_c = block_inputs(B, T, C, seed=2000 + w.index)
+    bufs = {"x": xb_c.to(dev), **{k: v.to(dev) for k, v in pb_c.items()},
+            "qkv": torch.empty(B, T, 3 * C, dtype=torch.bfloat16, device=dev),
+            "y": torch.empty(B, T, C, dtype=torch.bfloat16, device=dev),
+            "lse": torch.empty(B, nh, T, dtype=torch.float32, device=dev),
+            "out": torch.empty(B, T, C, dtype=torch.bfloat16, device=dev)}
+
+    def call():
+        b = bufs
+        ga.check(ga.gptattn_attn_block_fwd(b["x"], b["ln_w"], b["ln_b"], b["w_attn"], b["b_attn"], b["w_proj"],
+                                           b["b_proj"], b["qkv"], b["y"], b["lse"], b["out"], B, T, C, nh,
+                                           ga.GPTATTN_BF16, s), "gptattn_attn_block_fwd")
+    return call, bufs
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
 
@@ -232,6 +256,18 @@ def run_ours(args, w, rank, world, local_rank):
     ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MiB > 126 MB L2
     s = torch.cuda.current_stream(dev)
+    if args.block_run:
+        block_call, _ = make_block_call(ga, w, dev, s)
+        for _ in range(args.warmup + args.steps):
+            flush.zero_()
+            block_call()
+        torch.cuda.synchronize()
+        ga.check(ga.gptattn_get_device_status(s), "device status after the sub-block calls")
+        if dist is not None:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"block_run": "ok", "calls": args.warmup + args.steps}), flush=True)
+        return
 
     def step(q=qkv, g=dy):
         ga.check(ga.gptattn_fwd(q, y, lse, B, T, C, nh, dt, s), "gptattn_fwd")
@@ -513,6 +549,59 @@ def run_ours(args, w, rank, world, local_rank):
                   "large_cache": {"B": BL, "T": TL, "us_per_call": ms_l * 1e3, "kv_bytes": kv_l,
                                   "achieved_gbs": kv_l / ms_l / 1e6, "frac_of_hbm": kv_l / ms_l / 1e6 / hbm}}
 
+    # ---- the attention sub-block (gptattn_attn_block_fwd): LayerNorm -> c_attn -> causal
+    # attention -> c_proj + residual at this workload's B, T, C; bf16 only.  Whole-call time
+    # with CUDA events (L2 flushed before each call), then per-kernel times from the library's
+    # event records (launch order: layernorm, c_attn GEMM, attention forward, c_proj GEMM).
+    attn_block = None
+    if not args.profile_run and dt == ga.GPTATTN_BF16:
+        peaks_b, src_b = load_peaks()
+        tc_peak = float(peaks_b.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        hbm_b = float(peaks_b.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        block_call, block_bufs = make_block_call(ga, w, dev, s)
+
+        for _ in range(5):
+            flush.zero_()
+            block_call()
+        torch.cuda.synchronize()
+        Kb = max(1, min(K, 100))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Kb)]
+        for a, b_ in evs:
+            flush.zero_()
+            a.record(s)
+            block_call()
+            b_.record(s)
+        torch.cuda.synchronize()
+        ms_b = sum(a.elapsed_time(b_) for a, b_ in evs) / Kb
+        ga.gptattn_profile_enable(4 * Kb + 16)
+        for _ in range(Kb):
+            flush.zero_()
+            block_call()
+        torch.cuda.synchronize()
+        recs = ga.gptattn_profile_read(4 * Kb + 16)
+        ga.gptattn_profile_enable(0)
+        ga.check(ga.gptattn_get_device_status(s), "device status after the sub-block calls")
+        parts = {"layernorm": [], "c_attn": [], "attention": [], "c_proj": []}
+        for i in range(0, len(recs) - 3, 4):
+            for key, (_, ms) in zip(parts, recs[i:i + 4]):
+                parts[key].append(ms)
+        pm = {k: (statistics.mean(v) if v else None) for k, v in parts.items()}
+        M = B * T
+        fl = {"c_attn": 2.0 * M * C * 3 * C, "attention": w.flops_fwd(), "c_proj": 2.0 * M * C * C}
+        ln_bytes = 2 * M * C * 2 + 4 * C
+        attn_block = {
+            "workload": f"{w.name}: pre-LN attention sub-block forward, x [{B},{T},{C}] bf16",
+            "ms_per_call": ms_b, "flops_per_call": sum(fl.values()),
+            "value": sum(fl.values()) / (ms_b / 1e3) / 1e12, "unit": "TFLOP/s",
+            "kernels_ms": pm,
+            "gemm_tflops": {k: (fl[k] / (pm[k] / 1e3) / 1e12 if pm[k] else None) for k in ("c_attn", "c_proj")},
+            "gemm_frac_of_bf16_peak": {k: (fl[k] / (pm[k] / 1e3) / 1e12 / tc_peak if pm[k] else None)
+                                       for k in ("c_attn", "c_proj")},
+            "layernorm_gbs": (ln_bytes / (pm["layernorm"] / 1e3) / 1e9 if pm["layernorm"] else None),
+            "layernorm_frac_of_hbm": (ln_bytes / (pm["layernorm"] / 1e3) / 1e9 / hbm_b if pm["layernorm"] else None),
+            "peak_source": f"{src_b} bf16 burst / copy bandwidth", "calls": Kb}
+        del block_bufs
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -563,6 +652,7 @@ def run_ours(args, w, rank, world, local_rank):
                 "overlap": "copies in / compute / copies out on three streams, device buffers double-buffered"},
         "gpu_launches": launches,
         "decode": decode,
+        "attn_block": attn_block,
         "window": banded,
         "deterministic": det,
         "dropout": drop,

@@ -112,6 +112,20 @@ bool map_f32_acc(CUtensorMap *m, const void *ptr, int hs, long long rows) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 row-major matrix [outer][inner] viewed as 2-D (inner, outer); box (64,
+// box_outer); 128-byte swizzle; out-of-range rows read as zero and are not written.
+bool map_bf16_2d(CUtensorMap *m, const void *ptr, long long inner, long long outer, int box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)inner * 2u};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------
 // Validation (pure host; nothing is enqueued on failure)
 // ---------------------------------------------------------------------------
@@ -385,6 +399,41 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
 }
 }  // namespace
 
+namespace {
+// Linear map checks: sizes, alignment (16 bytes: TMA bases and vector loads).
+gptattn_status check_linear(const void *a, const void *w, const void *bias, const void *resid, const void *out, int M,
+                            int N, int K) {
+    if (M < 0 || N <= 0 || K <= 0) return GPTATTN_ERR_INVALID_ARG;
+    if (N % 64 != 0 || K % 64 != 0) return GPTATTN_ERR_UNSUPPORTED;
+    if (M == 0) return GPTATTN_OK;
+    if (!a || !w || !out) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return GPTATTN_ERR_INVALID_ARG;
+    if ((bias && !aligned16(bias)) || (resid && !aligned16(resid))) return GPTATTN_ERR_INVALID_ARG;
+    return GPTATTN_OK;
+}
+
+gptattn_status linear_impl(const void *a, const void *w, const void *bias, const void *resid, void *out, int M, int N,
+                           int K, cudaStream_t s) {
+    int *status = nullptr;
+    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    CUtensorMap ma, mw, mc;
+    if (!map_bf16_2d(&ma, a, K, M, 128) || !map_bf16_2d(&mw, w, K, N, 256) || !map_bf16_2d(&mc, out, N, M, 128))
+        return GPTATTN_ERR_CUDA;
+    const DevCtx ctx{status, kDefaultBudgetNs};
+    return from_cuda(
+        run_kernel(kKGemm, s, [&] { return launch_gemm_bf16(ma, mw, mc, bias, resid, M, N, K, ctx, s); }));
+}
+
+gptattn_status check_layernorm(const void *x, const void *w, const void *b, const void *out, int M, int C) {
+    if (M < 0 || C <= 0) return GPTATTN_ERR_INVALID_ARG;
+    if (C % 8 != 0 || C > 4096) return GPTATTN_ERR_UNSUPPORTED;
+    if (M == 0) return GPTATTN_OK;
+    if (!x || !w || !b || !out) return GPTATTN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(b) || !aligned16(out)) return GPTATTN_ERR_INVALID_ARG;
+    return GPTATTN_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char *gptattn_status_string(gptattn_status s) {
@@ -516,6 +565,48 @@ gptattn_status gptattn_bwd_opts(const void *qkv, const void *y, const float *lse
                     stream);
 }
 
+gptattn_status gptattn_layernorm(const void *x, const void *w, const void *b, void *out, int M, int C,
+                                 gptattn_dtype dt, gptattn_stream_t stream) {
+    if (dt != GPTATTN_BF16) return GPTATTN_ERR_UNSUPPORTED;
+    gptattn_status st = check_layernorm(x, w, b, out, M, C);
+    if (st != GPTATTN_OK || M == 0) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return from_cuda(run_kernel(kKLayerNorm, s, [&] { return launch_layernorm_bf16(x, w, b, out, M, C, s); }));
+}
+
+gptattn_status gptattn_linear(const void *a, const void *w, const void *bias, const void *resid, void *out, int M,
+                              int N, int K, gptattn_dtype dt, gptattn_stream_t stream) {
+    if (dt != GPTATTN_BF16) return GPTATTN_ERR_UNSUPPORTED;
+    gptattn_status st = check_linear(a, w, bias, resid, out, M, N, K);
+    if (st != GPTATTN_OK || M == 0) return st;
+    return linear_impl(a, w, bias, resid, out, M, N, K, reinterpret_cast<cudaStream_t>(stream));
+}
+
+gptattn_status gptattn_attn_block_fwd(const void *x, const void *ln_w, const void *ln_b, const void *w_attn,
+                                      const void *b_attn, const void *w_proj, const void *b_proj, void *qkv, void *y,
+                                      float *lse, void *out, int B, int T, int C, int n_head, gptattn_dtype dt,
+                                      gptattn_stream_t stream) {
+    if (dt != GPTATTN_BF16) return GPTATTN_ERR_UNSUPPORTED;
+    int hs = 0;
+    gptattn_status st = check_shape(B, T, C, n_head, dt, &hs);
+    if (st != GPTATTN_OK) return st;
+    if ((long long)B * T > 0x7fffffffLL) return GPTATTN_ERR_UNSUPPORTED;
+    const int M = B * T;
+    st = check_layernorm(x, ln_w, ln_b, y, M, C);
+    if (st == GPTATTN_OK) st = check_linear(y, w_attn, b_attn, nullptr, qkv, M, 3 * C, C);
+    if (st == GPTATTN_OK) st = check_linear(y, w_proj, b_proj, x, out, M, C, C);
+    if (st != GPTATTN_OK) return st;
+    if (M == 0) return GPTATTN_OK;
+    if (!lse || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // y holds LN(x) until the attention overwrites it with the heads' outputs.
+    st = from_cuda(run_kernel(kKLayerNorm, s, [&] { return launch_layernorm_bf16(x, ln_w, ln_b, y, M, C, s); }));
+    if (st == GPTATTN_OK) st = linear_impl(y, w_attn, b_attn, nullptr, qkv, M, 3 * C, C, s);
+    if (st == GPTATTN_OK) st = fwd_impl(qkv, y, lse, B, T, C, n_head, kCausalWindow, 0.f, 0, dt, stream);
+    if (st == GPTATTN_OK) st = linear_impl(y, w_proj, b_proj, x, out, M, C, C, s);
+    return st;
+}
+
 gptattn_status gptattn_get_device_status(gptattn_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return GPTATTN_ERR_CUDA;
@@ -573,7 +664,8 @@ int gptattn_profile_read(int *kernel_ids, float *ms, int capacity) {
 const char *gptattn_kernel_name(int kernel_id) {
     static const char *names[kKNumKernels] = {
         "fwd_bf16_sm100", "bwd_pre_bf16", "bwd_bf16_sm100", "bwd_post_bf16", "fwd_f32_simt",
-        "bwd_pre_f32",    "bwd_dq_f32",   "bwd_dkv_f32",    "selftest_timeout", "decode"};
+        "bwd_pre_f32",    "bwd_dq_f32",   "bwd_dkv_f32",    "selftest_timeout", "decode",
+        "layernorm_bf16", "gemm_bf16_sm100"};
     if (kernel_id < 0 || kernel_id >= kKNumKernels) return "unknown";
     return names[kernel_id];
 }

@@ -104,6 +104,16 @@ cudaError_t launch_bwd_f32_dkv(int hs, const float *qkv, const float *dy, const 
 cudaError_t launch_decode(int hs, bool bf16, const void *qkv, void *y, float *lse, int B, int T, int T_cap, int C,
                           int n_head, cudaStream_t s);
 
+// ---- the attention sub-block's neighbours (bf16): LayerNorm and the two linear maps
+// out[M][N] = a[M][K] w[N][K]^T + bias[N] (+ resid[M][N]); bias and resid may be null.
+// map_a: 2-D (K, M) view of a, box (64, 128); map_w: 2-D (K, N) view of w, box (64, 256);
+// map_c: 2-D (N, M) view of out, box (64, 128); all 128-byte swizzle.  N % 64 == K % 64 == 0.
+cudaError_t launch_gemm_bf16(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_c,
+                             const void *bias, const void *resid, int M, int N, int K, DevCtx ctx, cudaStream_t s);
+// out[M][C] = (x - mean) / sqrt(var + 1e-5) * w + b per row (C % 8 == 0, C <= 4096).
+cudaError_t launch_layernorm_bf16(const void *x, const void *w, const void *b, void *out, int M, int C,
+                                  cudaStream_t s);
+
 // ---- bounded-wait self-test -----------------------------------------------
 cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s);
 
@@ -119,7 +129,9 @@ enum KernelId {
     kKBwdDkvF32 = 7,
     kKSelftest = 8,
     kKDecode = 9,
-    kKNumKernels = 10
+    kKLayerNorm = 10,
+    kKGemm = 11,
+    kKNumKernels = 12
 };
 
 }  // namespace gptattn

@@ -32,7 +32,7 @@ EXPORTED = (
     "gptattn_fwd_opts", "gptattn_bwd_opts_workspace_bytes", "gptattn_bwd_opts", "gptattn_decode", "gptattn_bwd_workspace_bytes", "gptattn_bwd", "gptattn_get_device_status",
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
     "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
-    "gptattn_last_error_string",
+    "gptattn_last_error_string", "gptattn_layernorm", "gptattn_linear", "gptattn_attn_block_fwd",
 )
 
 
@@ -96,6 +96,12 @@ def lib():
             L.gptattn_bwd_opts.restype = i
             L.gptattn_decode.argtypes = [vp, vp, vp, i, i, i, i, i, i, st]
             L.gptattn_decode.restype = i
+            L.gptattn_layernorm.argtypes = [vp, vp, vp, vp, i, i, i, st]
+            L.gptattn_layernorm.restype = i
+            L.gptattn_linear.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, st]
+            L.gptattn_linear.restype = i
+            L.gptattn_attn_block_fwd.argtypes = [vp] * 11 + [i, i, i, i, i, st]
+            L.gptattn_attn_block_fwd.restype = i
             L.gptattn_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
             L.gptattn_bwd_workspace_bytes.restype = sz
             L.gptattn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, st]
@@ -184,6 +190,21 @@ def gptattn_bwd_opts(qkv, y, lse, dy, dqkv, workspace, workspace_bytes, B, T, C,
 
 def gptattn_decode(qkv, y, lse, B, T, T_cap, C, n_head, dt, stream=None) -> int:
     return lib().gptattn_decode(_ptr(qkv), _ptr(y), _ptr(lse), B, T, T_cap, C, n_head, dt, _stream(stream))
+
+
+def gptattn_layernorm(x, w, b, out, M, C, dt, stream=None) -> int:
+    return lib().gptattn_layernorm(_ptr(x), _ptr(w), _ptr(b), _ptr(out), M, C, dt, _stream(stream))
+
+
+def gptattn_linear(a, w, bias, resid, out, M, N, K, dt, stream=None) -> int:
+    return lib().gptattn_linear(_ptr(a), _ptr(w), _ptr(bias), _ptr(resid), _ptr(out), M, N, K, dt, _stream(stream))
+
+
+def gptattn_attn_block_fwd(x, ln_w, ln_b, w_attn, b_attn, w_proj, b_proj, qkv, y, lse, out, B, T, C, n_head, dt,
+                           stream=None) -> int:
+    return lib().gptattn_attn_block_fwd(_ptr(x), _ptr(ln_w), _ptr(ln_b), _ptr(w_attn), _ptr(b_attn), _ptr(w_proj),
+                                        _ptr(b_proj), _ptr(qkv), _ptr(y), _ptr(lse), _ptr(out), B, T, C, n_head, dt,
+                                        _stream(stream))
 
 
 def gptattn_bwd_workspace_bytes(B, T, C, n_head, dt) -> int:

@@ -106,3 +106,19 @@ def workload_inputs(w: Workload, B: int | None = None, T: int | None = None):
     return make_inputs(B if B is not None else w.B, T if T is not None else w.T, w.n_head, w.hs,
                        dtype=w.torch_dtype, seed=1000 + w.index, recipe=w.recipe,
                        qkv_scale=w.qkv_scale)
+
+
+def block_inputs(B: int, T: int, C: int, seed: int = 0):
+    """Seeded inputs of the pre-LN attention sub-block, bf16 on the CPU:
+    x[B,T,C] ~ N(0,1); LayerNorm gain 1 + 0.1 N(0,1) and bias 0.1 N(0,1);
+    c_attn weight [3C][C] and c_proj weight [C][C] ~ N(0,1)/sqrt(C) (so the
+    projected queries and keys are O(1) and the softmax is not flat); both
+    biases 0.1 N(0,1).  Draw order: x, ln_w, ln_b, w_attn, b_attn, w_proj, b_proj."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    rn = lambda *shape: torch.randn(*shape, generator=g, dtype=torch.float32)
+    x = rn(B, T, C)
+    p = {"ln_w": 1.0 + 0.1 * rn(C), "ln_b": 0.1 * rn(C),
+         "w_attn": rn(3 * C, C) / C ** 0.5, "b_attn": 0.1 * rn(3 * C),
+         "w_proj": rn(C, C) / C ** 0.5, "b_proj": 0.1 * rn(C)}
+    return x.to(torch.bfloat16).contiguous(), {k: v.to(torch.bfloat16).contiguous() for k, v in p.items()}

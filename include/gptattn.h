@@ -227,6 +227,46 @@ GPTATTN_API const char *gptattn_last_error_string(void);
 /* Library version, major * 10000 + minor * 100 + patch. */
 GPTATTN_API int gptattn_version(void);
 
+/* ---- The attention sub-block of a pre-LN GPT block (bf16 only) ------------
+ * minGPT README page ("卡帕西(氏)MinGPT"), GPT-2 notes: the layer norm sits at
+ * the input of each sub-block; lecture page ("Let's build GPT: from scratch, in
+ * code, spelled out"), chapters "multi-headed self-attention", "residual
+ * connections" and "layernorm (and its relationship to our previous
+ * batchnorm)".  Linear weights use nn.Linear's layout, [out_features]
+ * [in_features] row-major.  All buffers are device memory owned by the caller,
+ * 16-byte aligned; nothing is allocated.  dt must be GPTATTN_BF16 (else
+ * GPTATTN_ERR_UNSUPPORTED).
+ *
+ * gptattn_layernorm: out[m][:] = (x[m][:] - mean) / sqrt(var + 1e-5) * w + b for
+ *   each of the M rows of x[M][C] (population variance over the C features,
+ *   fp32 statistics); w, b are [C].  C % 8 == 0 and C <= 4096
+ *   (GPTATTN_ERR_UNSUPPORTED otherwise); M == 0 is a valid empty call.
+ *
+ * gptattn_linear: out[M][N] = a[M][K] w[N][K]^T + bias[N] (+ resid[M][N]), fp32
+ *   accumulation, one rounding to bf16.  bias and resid may be NULL (no term).
+ *   resid may equal out (in-place residual add); a and w must not overlap out.
+ *   N % 64 == 0 and K % 64 == 0 (GPTATTN_ERR_UNSUPPORTED otherwise).
+ *
+ * gptattn_attn_block_fwd: for x[B][T][C],
+ *     qkv = LN(x) w_attn^T + b_attn          (w_attn [3C][C], b_attn [3C])
+ *     y, lse = gptattn_fwd(qkv)              (causal, as above)
+ *     out = x + y w_proj^T + b_proj          (w_proj [C][C], b_proj [C])
+ *   qkv [B][T][3C], y [B][T][C], lse [B][n_head][T] (float32) and out
+ *   [B][T][C] are all written (qkv, y, lse are what a backward needs); y also
+ *   holds LN(x) between the first two steps, so no scratch is needed.  out may
+ *   equal x.  Shape rules are gptattn_fwd's (head size 64 or 128) plus the two
+ *   functions above; B*T < 2^31. */
+GPTATTN_API gptattn_status gptattn_layernorm(const void *x, const void *w, const void *b, void *out, int M, int C,
+                                             gptattn_dtype dt, gptattn_stream_t stream);
+GPTATTN_API gptattn_status gptattn_linear(const void *a, const void *w, const void *bias, const void *resid,
+                                          void *out, int M, int N, int K, gptattn_dtype dt,
+                                          gptattn_stream_t stream);
+GPTATTN_API gptattn_status gptattn_attn_block_fwd(const void *x, const void *ln_w, const void *ln_b,
+                                                  const void *w_attn, const void *b_attn, const void *w_proj,
+                                                  const void *b_proj, void *qkv, void *y, float *lse, void *out,
+                                                  int B, int T, int C, int n_head, gptattn_dtype dt,
+                                                  gptattn_stream_t stream);
+
 /* ---- Instrumentation (no counterpart on the pages; used by the benchmark) --
  * gptattn_profile_enable(n) with n > 0 makes later calls on the current device
  * record a pair of CUDA events around each kernel they launch, keeping up to n

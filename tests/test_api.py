@@ -170,3 +170,33 @@ def test_options_validation():
     assert ga.gptattn_bwd_opts_workspace_bytes(*args, O(deterministic=1), bf) == \
         ga.gptattn_bwd_det_workspace_bytes(*args, bf)
     assert ga.gptattn_bwd_opts_workspace_bytes(*args, O(window=-2), bf) == (1 << 64) - 1
+
+
+def test_block_validation():
+    BF, F32 = ga.GPTATTN_BF16, ga.GPTATTN_F32
+    OK, INV, UNS = 0, ga.GPTATTN_ERR_INVALID_ARG, ga.GPTATTN_ERR_UNSUPPORTED
+    # layernorm: C % 8, C <= 4096, bf16 only, pointers
+    assert ga.gptattn_layernorm(FAKE, FAKE, FAKE, FAKE, 4, 12, BF) == UNS
+    assert ga.gptattn_layernorm(FAKE, FAKE, FAKE, FAKE, 4, 4104, BF) == UNS
+    assert ga.gptattn_layernorm(FAKE, FAKE, FAKE, FAKE, 4, 768, F32) == UNS
+    assert ga.gptattn_layernorm(None, FAKE, FAKE, FAKE, 4, 768, BF) == INV
+    assert ga.gptattn_layernorm(FAKE + 2, FAKE, FAKE, FAKE, 4, 768, BF) == INV
+    assert ga.gptattn_layernorm(FAKE, FAKE, FAKE, FAKE, -1, 768, BF) == INV
+    assert ga.gptattn_layernorm(None, None, None, None, 0, 768, BF) == OK
+    # linear: N % 64, K % 64, pointers; bias and resid optional but aligned
+    assert ga.gptattn_linear(FAKE, FAKE, FAKE, None, FAKE, 8, 96, 64, BF) == UNS
+    assert ga.gptattn_linear(FAKE, FAKE, FAKE, None, FAKE, 8, 64, 32, BF) == UNS
+    assert ga.gptattn_linear(FAKE, FAKE, FAKE, None, FAKE, 8, 64, 64, F32) == UNS
+    assert ga.gptattn_linear(None, FAKE, FAKE, None, FAKE, 8, 64, 64, BF) == INV
+    assert ga.gptattn_linear(FAKE, FAKE, FAKE + 8, None, FAKE, 8, 64, 64, BF) == INV
+    assert ga.gptattn_linear(FAKE, FAKE, None, FAKE + 4, FAKE, 8, 64, 64, BF) == INV
+    assert ga.gptattn_linear(FAKE, FAKE, None, None, FAKE, 8, 0, 64, BF) == INV
+    assert ga.gptattn_linear(None, None, None, None, None, 0, 64, 64, BF) == OK
+    # block: attention shape rules + the two above
+    args = [FAKE] * 11
+    assert ga.gptattn_attn_block_fwd(*args, 2, 16, 96, 3, BF) == UNS      # head size 32
+    assert ga.gptattn_attn_block_fwd(*args, 2, 16, 768, 12, F32) == UNS
+    assert ga.gptattn_attn_block_fwd(*args[:9], None, FAKE, 2, 16, 768, 12, BF) == INV   # lse
+    assert ga.gptattn_attn_block_fwd(*args[:5], FAKE + 2, *args[6:], 2, 16, 768, 12, BF) == INV   # w_proj
+    assert ga.gptattn_attn_block_fwd(*([None] * 11), 0, 16, 768, 12, BF) == OK
+    assert ga.gptattn_attn_block_fwd(*([None] * 11), 2, 0, 768, 12, BF) == OK
