@@ -416,12 +416,13 @@ gptattn_status linear_impl(const void *a, const void *w, const void *bias, const
                            int K, cudaStream_t s) {
     int *status = nullptr;
     if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    const int tile_n = gemm_tile_n(M, N);
     CUtensorMap ma, mw, mc;
-    if (!map_bf16_2d(&ma, a, K, M, 128) || !map_bf16_2d(&mw, w, K, N, 256) || !map_bf16_2d(&mc, out, N, M, 128))
+    if (!map_bf16_2d(&ma, a, K, M, 128) || !map_bf16_2d(&mw, w, K, N, tile_n) || !map_bf16_2d(&mc, out, N, M, 128))
         return GPTATTN_ERR_CUDA;
     const DevCtx ctx{status, kDefaultBudgetNs};
     return from_cuda(
-        run_kernel(kKGemm, s, [&] { return launch_gemm_bf16(ma, mw, mc, bias, resid, M, N, K, ctx, s); }));
+        run_kernel(kKGemm, s, [&] { return launch_gemm_bf16(ma, mw, mc, bias, resid, M, N, K, tile_n, ctx, s); }));
 }
 
 gptattn_status check_layernorm(const void *x, const void *w, const void *b, const void *out, int M, int C) {

@@ -15,8 +15,9 @@
 // 4-stage TMA ring (128-byte swizzle), two TMEM accumulators so the epilogue of
 // one tile overlaps the MMAs of the next.  Warps: 0 TMA producer, 1 TMEM owner
 // + MMA issuer, 2..5 epilogue (one output row per thread): TMEM -> + bias
-// (+ residual row, read from global memory) -> bf16 -> swizzled staging ->
-// TMA store, 64 columns at a time through two staging tiles.  Every wait is
+// (+ residual, read one chunk ahead and passed through the staging tile) ->
+// bf16 -> swizzled staging -> TMA store, 64 columns at a time through two
+// staging tiles.  Every wait is
 // bounded.
 #include <type_traits>
 
@@ -27,31 +28,47 @@ namespace gptattn {
 namespace {
 
 constexpr int kGThreads = 192;
-constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kGStages = 4;
-constexpr uint32_t kABytes = kBM * kBK * 2;  // 16 KB
-constexpr uint32_t kBBytes = kBN * kBK * 2;  // 32 KB
+constexpr int kBM = 128, kBK = 64;
+constexpr uint32_t kABytes = kBM * kBK * 2;   // 16 KB
 constexpr uint32_t kStgBytes = kBM * 64 * 2;  // one 128 x 64 bf16 chunk
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kGStages * kABytes;
-constexpr uint32_t kOffStg = kOffB + kGStages * kBBytes;
-constexpr uint32_t kOffGBar = kOffStg + 2 * kStgBytes;
-constexpr int kGBarFull = 0, kGBarEmpty = kGBarFull + kGStages, kGBarAccFull = kGBarEmpty + kGStages,
-              kGBarAccEmpty = kGBarAccFull + 2, kGBarDone = kGBarAccEmpty + 2, kGNumBars = kGBarDone + 1;
-constexpr uint32_t kGSmemBytes = kOffGBar + 128 + 1024;
-static_assert(kGNumBars * 8 + 16 <= 128, "barrier area");
-static_assert(kGSmemBytes <= 232448, "shared memory per CTA");
+
+// Tile width along N and ring depth: 128 x 256 tiles with 4 stages, or 128 x 128 tiles
+// with 6 stages (same shared memory) when the wide tiles would leave fewer than three
+// per CTA.
+template <int BN, int STAGES>
+struct GemmShape {
+    static constexpr int kBN = BN, kGStages = STAGES;
+    static constexpr uint32_t kBBytes = BN * kBK * 2;
+    static constexpr uint32_t kOffA = 0;
+    static constexpr uint32_t kOffB = kOffA + STAGES * kABytes;
+    static constexpr uint32_t kOffStg = kOffB + STAGES * kBBytes;
+    static constexpr uint32_t kOffGBar = kOffStg + 2 * kStgBytes;
+    static constexpr int kGBarFull = 0, kGBarEmpty = kGBarFull + STAGES, kGBarAccFull = kGBarEmpty + STAGES,
+                         kGBarAccEmpty = kGBarAccFull + 2, kGBarDone = kGBarAccEmpty + 2, kGNumBars = kGBarDone + 1;
+    static constexpr uint32_t kGSmemBytes = kOffGBar + 256 + 1024;
+    static constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
+    static_assert(kGNumBars * 8 + 16 <= 256, "barrier area");
+    static_assert(kGSmemBytes <= 232448, "shared memory per CTA");
+    static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation");
+};
+using GemmWide = GemmShape<256, 4>;
+using GemmNarrow = GemmShape<128, 6>;
 
 __device__ __forceinline__ bool warp_wait_g(uint32_t bar, uint32_t parity, const WaitGuard &g) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, g));
 }
 
-template <bool kResidual>
+template <bool kResidual, class Shape>
 __global__ void __launch_bounds__(kGThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
                 const __grid_constant__ CUtensorMap map_c, const __nv_bfloat16 *__restrict__ bias,
                 const __nv_bfloat16 *__restrict__ resid, int M, int N, int K, int *status,
                 unsigned long long budget_ns) {
+    constexpr int kBN = Shape::kBN, kGStages = Shape::kGStages;
+    constexpr uint32_t kBBytes = Shape::kBBytes, kOffA = Shape::kOffA, kOffB = Shape::kOffB, kOffStg = Shape::kOffStg,
+                       kOffGBar = Shape::kOffGBar, kTmemCols = Shape::kTmemCols;
+    constexpr int kGBarFull = Shape::kGBarFull, kGBarEmpty = Shape::kGBarEmpty, kGBarAccFull = Shape::kGBarAccFull,
+                  kGBarAccEmpty = Shape::kGBarAccEmpty, kGBarDone = Shape::kGBarDone, kGNumBars = Shape::kGNumBars;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -79,7 +96,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -156,20 +173,42 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const bool leader = (warp == 2 && lane == 0);
         bool ok = true;
         int tc = 0, cc = 0;
+        // Residual chunks are read one chunk ahead and cooperatively: lane l of the warp holds
+        // 16 bytes of row sp*32 + 4i + l/8 (i = 0..7), columns 8*(l%8) .. +7 of the chunk, so
+        // each load instruction covers four whole 128-byte row segments.
+        const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+        auto chunks_of = [&](int tt) {
+            const int rem = N - (tt % tiles_n) * kBN;
+            return rem < kBN ? rem / 64 : kBN / 64;
+        };
+        auto load_resid = [&](int tt, int c, uint4(&dst)[8]) {
+            const bool valid = tt < n_tiles;
+            const int n0r = (tt % tiles_n) * kBN + c * 64;
+            const int r0 = (tt / tiles_n) * kBM + sp * 32 + (lane >> 3);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = r0 + 4 * i;
+                dst[i] = (valid && r < M)
+                             ? *reinterpret_cast<const uint4 *>(resid + (size_t)r * N + n0r + 8 * (lane & 7))
+                             : zero4;
+            }
+        };
+        uint4 rnext[8];
+        if constexpr (kResidual) load_resid(blockIdx.x, 0, rnext);
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tc) {
             const int tm = t / tiles_n, tn = t % tiles_n;
             const int acc = tc & 1;
-            const int grow = tm * kBM + row;
             if (ok) ok = warp_wait_g(bar(kGBarAccFull + acc), (uint32_t)(tc >> 1) & 1u, g);
             if (ok) tc_fence_after();
             for (int ch = 0; ch < kBN / 64; ++ch, ++cc) {
                 const int n0 = tn * kBN + ch * 64;
                 if (n0 >= N) break;  // uniform over the 128 threads (N % 64 == 0)
-                uint4 r8[8];
+                uint4 rcur[8];
                 if constexpr (kResidual) {
-                    const uint4 *rp = reinterpret_cast<const uint4 *>(resid + (size_t)grow * N + n0);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) r8[q] = grow < M ? rp[q] : make_uint4(0u, 0u, 0u, 0u);
+                    for (int i = 0; i < 8; ++i) rcur[i] = rnext[i];
+                    const bool last = ch + 1 >= chunks_of(t);
+                    load_resid(last ? t + (int)gridDim.x : t, last ? 0 : ch + 1, rnext);
                 }
                 uint32_t v[64];
                 if (ok) {
@@ -186,6 +225,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 const uint32_t stg = sbase + kOffStg + (uint32_t)(cc & 1) * kStgBytes;
                 if (ok) {
                     const uint32_t rbase = stg + (uint32_t)row * 128u;
+                    if constexpr (kResidual) {  // the warp's 32 residual rows into its rows of the staging tile
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const uint32_t rr = (uint32_t)(sp * 32 + 4 * i + (lane >> 3));
+                            st_shared_v4(stg + rr * 128u + ((((uint32_t)lane & 7u) ^ (rr & 7u)) << 4), rcur[i].x,
+                                         rcur[i].y, rcur[i].z, rcur[i].w);
+                        }
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {  // 8 columns per 16-byte chunk
                         const uint4 bq = bias ? *reinterpret_cast<const uint4 *>(bias + n0 + 8 * q)
@@ -193,10 +241,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
                         const uint32_t bw[4] = {bq.x, bq.y, bq.z, bq.w};
                         uint32_t rw[4] = {0u, 0u, 0u, 0u};
                         if constexpr (kResidual) {
-                            rw[0] = r8[q].x;
-                            rw[1] = r8[q].y;
-                            rw[2] = r8[q].z;
-                            rw[3] = r8[q].w;
+                            const uint4 r4 = ld_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4));
+                            rw[0] = r4.x;
+                            rw[1] = r4.y;
+                            rw[2] = r4.z;
+                            rw[3] = r4.w;
                         }
                         uint32_t o[4];
 #pragma unroll
@@ -226,7 +275,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -290,20 +339,43 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16 *__r
 
 }  // namespace
 
-cudaError_t launch_gemm_bf16(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_c,
-                             const void *bias, const void *resid, int M, int N, int K, DevCtx ctx, cudaStream_t s) {
-    auto kern = resid ? gemm_kernel<true> : gemm_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGSmemBytes);
+namespace {
+int sm_count(int *sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? 0 : -1;
+}
+
+template <class Shape>
+cudaError_t launch_gemm_shape(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_c,
+                              const void *bias, const void *resid, int M, int N, int K, int sms, DevCtx ctx,
+                              cudaStream_t s) {
+    auto kern = resid ? gemm_kernel<true, Shape> : gemm_kernel<false, Shape>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape::kGSmemBytes);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    const long long tiles = (long long)((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+    const long long tiles = (long long)((M + kBM - 1) / kBM) * ((N + Shape::kBN - 1) / Shape::kBN);
     const int grid = (int)(tiles < sms ? tiles : sms);
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(kGThreads), kGSmemBytes, s, map_a, map_w, map_c,
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kGThreads), Shape::kGSmemBytes, s, map_a, map_w, map_c,
                       static_cast<const __nv_bfloat16 *>(bias), static_cast<const __nv_bfloat16 *>(resid), M, N, K,
                       ctx.status, ctx.budget_ns);
+}
+}  // namespace
+
+int gemm_tile_n(int M, int N) {
+    int sms = 148;
+    if (sm_count(&sms) != 0 || sms <= 0) sms = 148;
+    const long long wide = (long long)((M + kBM - 1) / kBM) * ((N + 255) / 256);
+    return wide < 3LL * sms ? 128 : 256;
+}
+
+cudaError_t launch_gemm_bf16(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_c,
+                             const void *bias, const void *resid, int M, int N, int K, int tile_n, DevCtx ctx,
+                             cudaStream_t s) {
+    int sms = 0;
+    if (sm_count(&sms) != 0) return cudaErrorInvalidDevice;
+    if (tile_n == 256) return launch_gemm_shape<GemmWide>(map_a, map_w, map_c, bias, resid, M, N, K, sms, ctx, s);
+    if (tile_n == 128) return launch_gemm_shape<GemmNarrow>(map_a, map_w, map_c, bias, resid, M, N, K, sms, ctx, s);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_layernorm_bf16(const void *x, const void *w, const void *b, void *out, int M, int C,

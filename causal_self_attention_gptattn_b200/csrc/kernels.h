@@ -106,10 +106,13 @@ cudaError_t launch_decode(int hs, bool bf16, const void *qkv, void *y, float *ls
 
 // ---- the attention sub-block's neighbours (bf16): LayerNorm and the two linear maps
 // out[M][N] = a[M][K] w[N][K]^T + bias[N] (+ resid[M][N]); bias and resid may be null.
-// map_a: 2-D (K, M) view of a, box (64, 128); map_w: 2-D (K, N) view of w, box (64, 256);
+// map_a: 2-D (K, M) view of a, box (64, 128); map_w: 2-D (K, N) view of w, box (64, tile_n);
 // map_c: 2-D (N, M) view of out, box (64, 128); all 128-byte swizzle.  N % 64 == K % 64 == 0.
+// tile_n (128 or 256) is the output tile width gemm_tile_n() picks for the shape.
+int gemm_tile_n(int M, int N);
 cudaError_t launch_gemm_bf16(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_c,
-                             const void *bias, const void *resid, int M, int N, int K, DevCtx ctx, cudaStream_t s);
+                             const void *bias, const void *resid, int M, int N, int K, int tile_n, DevCtx ctx,
+                             cudaStream_t s);
 // out[M][C] = (x - mean) / sqrt(var + 1e-5) * w + b per row (C % 8 == 0, C <= 4096).
 cudaError_t launch_layernorm_bf16(const void *x, const void *w, const void *b, void *out, int M, int C,
                                   cudaStream_t s);

@@ -62,7 +62,8 @@ def test_layernorm_parity(M, C):
     (300, 768, 768, True, True),      # c_proj with the residual
     (128, 64, 64, False, False),      # one tile, one chunk
     (1, 192, 128, True, True),        # a single row
-    (517, 320, 1024, False, True),    # N not a multiple of the 256-wide tile
+    (517, 320, 1024, False, True),    # N not a multiple of the tile width
+    (20000, 768, 256, True, True),    # enough tiles for the 128 x 256 shape (the smaller ones use 128 x 128)
 ])
 def test_linear_parity(M, N, K, with_bias, with_resid):
     r = np.random.default_rng(M * 7 + N + K)
