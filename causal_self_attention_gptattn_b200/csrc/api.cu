@@ -299,8 +299,8 @@ gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int 
     st = make_dropout(dropout_p, seed, hs, dt, &dp);
     if (st != GPTATTN_OK) return st;
     if (B == 0 || T == 0) return GPTATTN_OK;
-    if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
-    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    if (!qkv || !y) return GPTATTN_ERR_INVALID_ARG;  // lse may be null: inference, not written
+    if (!aligned16(qkv) || !aligned16(y) || (lse && !aligned16(lse))) return GPTATTN_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
     if (dt == GPTATTN_F32) {
@@ -472,8 +472,8 @@ gptattn_status gptattn_decode(const void *qkv, void *y, float *lse, int B, int T
     if (T_cap < T) return GPTATTN_ERR_INVALID_ARG;
     if ((long long)B * n_head > 65535LL) return GPTATTN_ERR_UNSUPPORTED;  // grid.y
     if (B == 0 || T == 0) return GPTATTN_OK;
-    if (!qkv || !y || !lse) return GPTATTN_ERR_INVALID_ARG;
-    if (!aligned16(qkv) || !aligned16(y) || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    if (!qkv || !y) return GPTATTN_ERR_INVALID_ARG;  // lse may be null: inference, not written
+    if (!aligned16(qkv) || !aligned16(y) || (lse && !aligned16(lse))) return GPTATTN_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return from_cuda(run_kernel(kKDecode, s, [&] {
         return launch_decode(hs, dt == GPTATTN_BF16, qkv, y, lse, B, T, T_cap, C, n_head, s);
@@ -598,7 +598,7 @@ gptattn_status gptattn_attn_block_fwd(const void *x, const void *ln_w, const voi
     if (st == GPTATTN_OK) st = check_linear(y, w_proj, b_proj, x, out, M, C, C);
     if (st != GPTATTN_OK) return st;
     if (M == 0) return GPTATTN_OK;
-    if (!lse || !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;
+    if (lse && !aligned16(lse)) return GPTATTN_ERR_INVALID_ARG;  // null: not written
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // y holds LN(x) until the attention overwrites it with the heads' outputs.
     st = from_cuda(run_kernel(kKLayerNorm, s, [&] { return launch_layernorm_bf16(x, ln_w, ln_b, y, M, C, s); }));

@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kDecThreads, 8) decode_kernel(const Elem *__re
             *dst = __float2bfloat16_rn(yv);
         else
             *dst = yv;
-        if (threadIdx.x == 0) lse[(size_t)b * n_head + h] = (mm + __log2f(ll)) * 0.6931471805599453f;
+        if (threadIdx.x == 0 && lse) lse[(size_t)b * n_head + h] = (mm + __log2f(ll)) * 0.6931471805599453f;
     }
     cluster_sync();  // peers keep their shared memory until rank 0 has read it
 }

@@ -438,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 fence_proxy_async_smem();
                 const int tq = qt * kTile + row;
-                if (tq < T) lse[(size_t)bh * (size_t)T + (size_t)tq] = (mrow + __log2f(l)) * 0.6931471805599453f;
+                if (tq < T && lse) lse[(size_t)bh * (size_t)T + (size_t)tq] = (mrow + __log2f(l)) * 0.6931471805599453f;
             }
             named_bar_sync(1 + t, 128);
             if (leader) {

@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kRows) fwd_f32_kernel(const float *__restrict_
         float *yr = y + ((size_t)b * T + t) * (size_t)C + (size_t)h * HS;
 #pragma unroll
         for (int d = 0; d < HS; ++d) yr[d] = acc[d] * inv;
-        lse[(size_t)bh * T + t] = m + logf(l);
+        if (lse) lse[(size_t)bh * T + t] = m + logf(l);
     }
 }
 

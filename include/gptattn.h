@@ -17,7 +17,9 @@
  *                      columns [h*hs, (h+1)*hs) of each part (hs = C/n_head).
  *                      This is the output of a GPT-2 block's c_attn projection.
  *     y    [B][T][C]   heads concatenated back in the same column order.
- *     lse  [B][n_head][T]  float32 always.
+ *     lse  [B][n_head][T]  float32 always.  The forward entry points (and
+ *          gptattn_decode, gptattn_attn_block_fwd) accept lse == NULL for
+ *          inference, when no backward follows: it is then not written.
  *     dy   [B][T][C], dqkv [B][T][3C]: same layouts as y and qkv.
  *
  * Element types: GPTATTN_BF16 -> qkv, y, dy, dqkv are bfloat16 (tensor-core

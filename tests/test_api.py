@@ -69,11 +69,12 @@ def test_null_and_misaligned_pointers_rejected():
     args = (2, 8, 128, 2, ga.GPTATTN_BF16, None)
     assert ga.gptattn_fwd(None, FAKE, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
     assert ga.gptattn_fwd(FAKE, None, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
-    assert ga.gptattn_fwd(FAKE, FAKE, None, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_fwd(FAKE, FAKE, FAKE + 4, *args) == ga.GPTATTN_ERR_INVALID_ARG  # lse misaligned (NULL is allowed)
     assert ga.gptattn_fwd(FAKE + 8, FAKE, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
     assert ga.gptattn_fwd(FAKE, FAKE + 2, FAKE, *args) == ga.GPTATTN_ERR_INVALID_ARG
     ws = ga.gptattn_bwd_workspace_bytes(2, 8, 128, 2, ga.GPTATTN_BF16)
     assert ga.gptattn_bwd(FAKE, FAKE, FAKE, None, FAKE, FAKE, ws, *args) == ga.GPTATTN_ERR_INVALID_ARG
+    assert ga.gptattn_bwd(FAKE, FAKE, None, FAKE, FAKE, FAKE, ws, *args) == ga.GPTATTN_ERR_INVALID_ARG  # bwd needs lse
     assert ga.gptattn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, ws, *args) == ga.GPTATTN_ERR_INVALID_ARG
 
 
@@ -196,7 +197,7 @@ def test_block_validation():
     args = [FAKE] * 11
     assert ga.gptattn_attn_block_fwd(*args, 2, 16, 96, 3, BF) == UNS      # head size 32
     assert ga.gptattn_attn_block_fwd(*args, 2, 16, 768, 12, F32) == UNS
-    assert ga.gptattn_attn_block_fwd(*args[:9], None, FAKE, 2, 16, 768, 12, BF) == INV   # lse
+    assert ga.gptattn_attn_block_fwd(*args[:9], FAKE + 4, FAKE, 2, 16, 768, 12, BF) == INV   # lse misaligned
     assert ga.gptattn_attn_block_fwd(*args[:5], FAKE + 2, *args[6:], 2, 16, 768, 12, BF) == INV   # w_proj
     assert ga.gptattn_attn_block_fwd(*([None] * 11), 0, 16, 768, 12, BF) == OK
     assert ga.gptattn_attn_block_fwd(*([None] * 11), 2, 0, 768, 12, BF) == OK
