@@ -29,8 +29,9 @@
 //                 Q_i, dO_i, lse_i, D_i through a 3-stage ring
 //   warp 1        TMEM owner + MMA issuer
 //   warps 2..9    softmax: TMEM sub-partition warp%4 (32 key rows), column
-//                 half (warp-2)/4 (64 query columns): P^T, dS^T, dK/dV epilogue
-//   warps 10..13  dQ drain: TMEM -> smem (fp32, swizzled) -> TMA reduce-add
+//                 half (warp-2)/4 (64 query columns): P^T, dS^T
+//   warps 10..13  dQ drain: TMEM -> smem (fp32, swizzled) -> TMA reduce-add;
+//                 and per item the dK/dV epilogue (TMEM -> bf16 -> TMA store)
 // TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T [256,320) (bf16 pairs)
 //                     dV [320,384)  dK [384,448)  dQ [448,512)
 // MMA order per item: S_0 dP_0 | S_1 dV_0 dK_0 dQ_0 dP_1 | S_2 dV_1 ...
@@ -167,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(kBardQFull), 1);
         mbar_init(bar(kBardQEmpty), kDrainThreads);
         mbar_init(bar(kBarKdV), 1);
-        mbar_init(bar(kBarAccFree), kSoftmaxThreads);
+        mbar_init(bar(kBarAccFree), kDrainThreads);
         mbar_init(bar(kBarDone), 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0;; ++k, ++n) {
             const int w = item_index(k, blockIdx.x, gridDim.x);
             if (w >= n_items) break;
-            const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
+            const int kt = w / BH, bh = w % BH;
             const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
             for (int it = 0; it < niter; ++it, ++gi) {
                 const int st = gi % kQStages;
@@ -471,40 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(bar(kBardSFull));
                 }
             }
-            // ---------------------------------------------------- dK / dV epilogue of this item
-            // staging: the dS buffer (free once the item's last dQ retired): dV -> slab 0, dK -> slab 1
-            if (ok) ok = warp_wait(bar(kBarKdV), (uint32_t)n & 1u, g);
-            if (ok) {
-                tc_fence_after();
-                const uint32_t col = half == 0 ? kColdV : kColdK;
-                const float mul = half == 0 ? 1.f : 0.125f;
-                uint32_t o[64];
-                tmem_ld_x32(trow + col, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-                tmem_ld_x32(trow + col + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
-                tc_fence_before();
-                mbar_arrive(bar(kBarAccFree));
-                const uint32_t rbase = sdS + (uint32_t)half * kSlabBytes + (uint32_t)row * 128u;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    uint32_t wv[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        wv[e] = pack_bf16x2(__uint_as_float(o[8 * q + 2 * e]) * mul,
-                                            __uint_as_float(o[8 * q + 2 * e + 1]) * mul);
-                    st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), wv[0], wv[1], wv[2], wv[3]);
-                }
-                fence_proxy_async_smem();
-            }
-            named_bar_sync(1, kSoftmaxThreads);
-            if (warp == 2 && lane == 0 && ok && !*abort_flag) {
-                tma_store_3d(&map_dqkv, sdS, 2 * C + h * HS, kt * kTile, b);
-                tma_store_3d(&map_dqkv, sdS + kSlabBytes, C + h * HS, kt * kTile, b);
-                bulk_commit_group();
-                bulk_wait_group_read_0();  // staging may be overwritten by the next item's dS
-            }
-            named_bar_sync(1, kSoftmaxThreads);
         }
-        if (warp == 2 && lane == 0) bulk_wait_group_0();
     } else {
         // ================================================================ dQ drain warps
         const int sp = warp & 3;
@@ -513,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool leader = (warp == 10 && lane == 0);
         bool ok = true;
         int gi = 0;
-        for (int k = 0;; ++k) {
+        for (int k = 0, n = 0;; ++k, ++n) {
             const int w = item_index(k, blockIdx.x, gridDim.x);
             if (w >= n_items) break;
             const int kt = w / BH, bh = w % BH;
@@ -548,6 +516,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_store_2d(&map_dq, sdQ, 32 * hh, (bh * n_slots + qt * (qt + 1) / 2 + kt) * kTile);
                         bulk_commit_group();
                     }
+                }
+            }
+            // ------------------------------------------------ dK / dV epilogue of this item
+            // (here rather than on the softmax warps, which go straight on to the next item):
+            // TMEM -> bf16 (dK scaled) -> the staging slab -> TMA store, dV then dK
+            if (ok) ok = warp_wait(bar(kBarKdV), (uint32_t)n & 1u, g);
+            const int b = bh / n_head, h = bh % n_head;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
+                uint32_t pv[32];
+                if (ok) {
+                    tc_fence_after();
+                    const float mul = which == 0 ? 1.f : 0.125f;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part) {
+                        uint32_t o[32];
+                        tmem_ld_x32(trow + (which == 0 ? kColdV : kColdK) + 32 * part, o);
+#pragma unroll
+                        for (int c = 0; c < 16; ++c)
+                            pv[16 * part + c] =
+                                pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
+                    }
+                    if (which == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(kBarAccFree));  // the next item's dV / dK may overwrite the accumulators
+                    }
+                }
+                if (leader) bulk_wait_group_read_0();
+                named_bar_sync(2, kDrainThreads);
+                if (ok) {
+                    const uint32_t rbase = sdQ + (uint32_t)row * 128u;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), pv[4 * q], pv[4 * q + 1],
+                                     pv[4 * q + 2], pv[4 * q + 3]);
+                    fence_proxy_async_smem();
+                }
+                named_bar_sync(2, kDrainThreads);
+                if (leader && ok && !*abort_flag) {
+                    tma_store_3d(&map_dqkv, sdQ, (which == 0 ? 2 * C : C) + h * HS, kt * kTile, b);
+                    bulk_commit_group();
                 }
             }
         }
