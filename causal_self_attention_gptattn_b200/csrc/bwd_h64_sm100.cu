@@ -34,7 +34,7 @@
 //                 and per item the dK/dV epilogue (TMEM -> bf16 -> TMA store)
 // TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T [256,320) (bf16 pairs)
 //                     dV [320,384)  dK [384,448)  dQ [448,512)
-// MMA order per item: S_0 dP_0 | S_1 dV_0 dK_0 dQ_0 dP_1 | S_2 dV_1 ...
+// MMA order per item: S_0 dP_0 | S_1 dV_0 dP_1 dK_0 dQ_0 | S_2 dV_1 dP_2 ...
 // S^T and dP^T are released as soon as the softmax warps hold them in
 // registers, so the tensor pipe computes tile i+1 while tile i is in softmax.
 // Every wait is bounded; roles never leave their loops early, so all named
@@ -294,6 +294,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, at(b, kk * 2048u), idAcc, kk > 0 ? 1u : acc);
                     }
                     umma_commit(bar(kBarPEmpty));
+                    // dP^T of the next query tile, ahead of this tile's dK and dQ (which wait for
+                    // this tile's dS), so the softmax warps find it ready when they reach it
+                    if (more) {
+                        if (!(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
+                        tc_fence_after();
+                        issue_dP(kvs, st1);
+                    }
                     // dK += dS^T Q ; dQ = dS K
                     if (!(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
                     tc_fence_after();
@@ -316,11 +323,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_commit(bar(kBardQFull));
                     umma_commit(bar(kBardSEmpty));
                     umma_commit(bar(kBarQEmpty + st));
-                    if (more) {  // dP^T of the next query tile
-                        if (!(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
-                        tc_fence_after();
-                        issue_dP(kvs, st1);
-                    }
                 }
                 if (!ok) break;
                 umma_commit(bar(kBarKdV));
