@@ -107,6 +107,29 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
+// 2^x for a pair of x <= ~1 on the FMA pipe, to take part of the exponentials off the
+// multi-function unit: Cody-Waite style reduction x = j + f with j an integer (rounded by
+// adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it on that interval by
+// weighted least squares (relative error below 7.6e-5); j added to the exponent field.
+// x is clamped at -125, so results below 2^-125 come out as about 2^-125 instead of 0.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float &y0, float &y1) {
+    const uint64_t x = f32x2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = fadd2(x, f32x2_pack(12582912.f, 12582912.f));           // 1.5 * 2^23 + j
+    const uint64_t xi = fadd2(t, f32x2_pack(-12582912.f, -12582912.f));         // j
+    const uint64_t f = ffma2(xi, f32x2_pack(-1.f, -1.f), x);                    // x - j
+    uint64_t p = ffma2(f32x2_pack(0.05517605319619179f, 0.05517605319619179f), f,
+                       f32x2_pack(0.24261149764060974f, 0.24261149764060974f));
+    p = ffma2(p, f, f32x2_pack(0.6932601928710938f, 0.6932601928710938f));
+    p = ffma2(p, f, f32x2_pack(0.9999280571937561f, 0.9999280571937561f));
+    float p0, p1, t0, t1;
+    f32x2_unpack(p, p0, p1);
+    f32x2_unpack(t, t0, t1);
+    // the low mantissa bits of t hold j; shifted into the exponent field (the constant's own
+    // bits shift out of the word)
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // Last query tile that key tile kt's band reaches.
 __device__ __forceinline__ int band_hi_tile(int kt, int window, int n_t) {
     const long long t = (long long)kt * kTile + kTile - 2 + window;  // largest key + window - 1
@@ -374,10 +397,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float x0, x1, x2, x3;
                         f32x2_unpack(x01, x0, x1);
                         f32x2_unpack(x23, x2, x3);
-                        pf[c] = ex2_approx(x0);
-                        pf[c + 1] = ex2_approx(x1);
-                        pf[c + 2] = ex2_approx(x2);
-                        pf[c + 3] = ex2_approx(x3);
+                        if ((c4 & 3) == 3) {  // a quarter of the exponentials on the FMA pipe
+                            exp2_poly_x2(x0, x1, pf[c], pf[c + 1]);
+                            exp2_poly_x2(x2, x3, pf[c + 2], pf[c + 3]);
+                        } else {
+                            pf[c] = ex2_approx(x0);
+                            pf[c + 1] = ex2_approx(x1);
+                            pf[c + 2] = ex2_approx(x2);
+                            pf[c + 3] = ex2_approx(x3);
+                        }
                     }
                     if (it == 0) {  // diagonal tile: query column q sees key `row` only if row <= q
 #pragma unroll
