@@ -335,6 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             umma_ss(tmem + kColdK, at(ddS, (kk >> 2) * kSlabBytes + (kk & 3) * 32u), at(b, kk * 2048u),
                                     idAcc, kk > 0 ? 1u : acc);
                     }
+                    // dK was the last reader of Q_i and dO_i (dQ reads dS and K): release their stage
+                    umma_commit(bar(kBarQEmpty + st));
                     if (gi > 0 && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
                     tc_fence_after();
                     {
@@ -345,7 +347,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     umma_commit(bar(kBardQFull));
                     umma_commit(bar(kBardSEmpty));
-                    umma_commit(bar(kBarQEmpty + st));
                 }
                 if (!ok) break;
                 umma_commit(bar(kBarKdV));
