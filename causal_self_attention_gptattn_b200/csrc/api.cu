@@ -46,6 +46,12 @@ gptattn_status from_cuda(cudaError_t e) {
     return GPTATTN_ERR_CUDA;
 }
 
+// A failure that is not a CUDA error code (tensor-map encoding): record why.
+gptattn_status fail_cuda(const char *why) {
+    t_last_error = why;
+    return GPTATTN_ERR_CUDA;
+}
+
 // Device address of g_device_status for the current device (looked up once
 // per device, with that device current).
 cudaError_t status_ptr(int **out) {
@@ -311,9 +317,10 @@ gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int 
     }
     int *status = nullptr;
     cudaError_t e = status_ptr(&status);
-    if (e != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     CUtensorMap mq, my;
-    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&my, y, C, T, B)) return GPTATTN_ERR_CUDA;
+    if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&my, y, C, T, B))
+        return fail_cuda("tensor map encoding failed");
     const DevCtx ctx{status, kDefaultBudgetNs};
     return from_cuda(
         run_kernel(kKFwdBf16, s, [&] { return launch_fwd_bf16(hs, mq, my, lse, B, T, C, n_head, kw, dp, ctx, s); }));
@@ -370,7 +377,7 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
     }
 
     int *status = nullptr;
-    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t es = status_ptr(&status)) return from_cuda(es);
     const int T_pad = padded_T(T);
     float *D = reinterpret_cast<float *>(ws + w.D);
     float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
@@ -379,7 +386,7 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
     if (!map_bf16_rows(&mq, qkv, 3 * C, T, B) || !map_bf16_rows(&mdy, dy, C, T, B) ||
         !map_bf16_rows(&mdqkv, dqkv, 3 * C, T, B) ||
         !map_f32_acc(&mdq, dqacc, hs, det ? (long long)B * n_head * det_slots(T) * kTile : (long long)B * n_head * T_pad))
-        return GPTATTN_ERR_CUDA;
+        return fail_cuda("tensor map encoding failed");
     const int n_slots = det ? (int)det_slots(T) : 0;
     const DevCtx ctx{status, kDefaultBudgetNs};
     cudaError_t e = run_kernel(kKBwdPreBf16, s, [&] {
@@ -415,11 +422,11 @@ gptattn_status check_linear(const void *a, const void *w, const void *bias, cons
 gptattn_status linear_impl(const void *a, const void *w, const void *bias, const void *resid, void *out, int M, int N,
                            int K, cudaStream_t s) {
     int *status = nullptr;
-    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t es = status_ptr(&status)) return from_cuda(es);
     const int tile_n = gemm_tile_n(M, N);
     CUtensorMap ma, mw, mc;
     if (!map_bf16_2d(&ma, a, K, M, 128) || !map_bf16_2d(&mw, w, K, N, tile_n) || !map_bf16_2d(&mc, out, N, M, 128))
-        return GPTATTN_ERR_CUDA;
+        return fail_cuda("tensor map encoding failed");
     const DevCtx ctx{status, kDefaultBudgetNs};
     return from_cuda(
         run_kernel(kKGemm, s, [&] { return launch_gemm_bf16(ma, mw, mc, bias, resid, M, N, K, tile_n, ctx, s); }));
@@ -610,13 +617,13 @@ gptattn_status gptattn_attn_block_fwd(const void *x, const void *ln_w, const voi
 
 gptattn_status gptattn_get_device_status(gptattn_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t e = cudaStreamSynchronize(s)) return from_cuda(e);
     int *p = nullptr;
-    if (status_ptr(&p) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t es = status_ptr(&p)) return from_cuda(es);
     int v = 0;
-    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost)) return from_cuda(e);
     const int zero = 0;
-    if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t e = cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice)) return from_cuda(e);
     return v == 0 ? GPTATTN_OK : static_cast<gptattn_status>(v);
 }
 
@@ -628,7 +635,7 @@ gptattn_status gptattn_profile_enable(int max_records) {
     const size_t want = 2u * (size_t)max_records;
     while (g_prof.pool.size() + 2u * g_prof.records.size() < want) {
         cudaEvent_t e = nullptr;
-        if (cudaEventCreate(&e) != cudaSuccess) return GPTATTN_ERR_CUDA;
+        if (cudaError_t ce = cudaEventCreate(&e)) return from_cuda(ce);
         g_prof.pool.push_back(e);
     }
     if (max_records == 0) {
@@ -676,7 +683,7 @@ unsigned long long gptattn_launch_count(void) { return g_launches.load(); }
 gptattn_status gptattn_selftest_wait_timeout(unsigned long long budget_ns, gptattn_stream_t stream) {
     if (budget_ns < 1000ull || budget_ns > 2000000000ull) return GPTATTN_ERR_INVALID_ARG;
     int *status = nullptr;
-    if (status_ptr(&status) != cudaSuccess) return GPTATTN_ERR_CUDA;
+    if (cudaError_t es = status_ptr(&status)) return from_cuda(es);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const DevCtx ctx{status, budget_ns};
     return from_cuda(run_kernel(kKSelftest, s, [&] { return launch_selftest_timeout(ctx, s); }));

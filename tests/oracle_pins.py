@@ -248,6 +248,26 @@ def pin_finite_differences(orc):
         assert err < 1e-6, f"finite-difference mismatch {err:.3e}"
 
 
+def pin_row_identity(orc):
+    """The backward's row term: rowsum(dY o y) equals rowsum(P o dP) with dP = dY V^T, because
+    y = P V (the lecture's weighted aggregation); y from the forward, P from the weights
+    routine, element sums in fp64."""
+    B, T, n_head, hs = 2, 23, 3, 6
+    C = n_head * hs
+    r = _rng(41)
+    qkv = r.standard_normal((B, T, 3 * C)) * 1.3
+    dy = r.standard_normal((B, T, C))
+    y, _ = orc.forward(qkv, n_head)
+    _, _, v = _split(qkv, n_head)
+    for b in range(B):
+        for h in range(n_head):
+            P = orc.probs(qkv, n_head, b, h)
+            dyh = dy[b, :, h * hs:(h + 1) * hs]
+            lhs = (dyh * y[b, :, h * hs:(h + 1) * hs]).sum(axis=1)
+            rhs = (P * (dyh @ v[b, h].T)).sum(axis=1)
+            assert np.allclose(lhs, rhs, rtol=0, atol=1e-12)
+
+
 def pin_library_special_case(orc):
     """A different implementation of the same function: PyTorch's
     scaled_dot_product_attention(is_causal=True) and autograd, in fp64 on
@@ -531,6 +551,7 @@ def pin_philox_statistics(orc):
 
 
 ALL_PINS = [
+    pin_row_identity,
     pin_single_token, pin_uniform_scores_prefix_mean, pin_tril_average_fixture,
     pin_rows_are_distributions, pin_weights_from_softmax_of_scaled_scores,
     pin_worked_two_heads, pin_causality, pin_batch_independence, pin_head_permutation,

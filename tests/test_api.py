@@ -201,3 +201,17 @@ def test_block_validation():
     assert ga.gptattn_attn_block_fwd(*args[:5], FAKE + 2, *args[6:], 2, 16, 768, 12, BF) == INV   # w_proj
     assert ga.gptattn_attn_block_fwd(*([None] * 11), 0, 16, 768, 12, BF) == OK
     assert ga.gptattn_attn_block_fwd(*([None] * 11), 2, 0, 768, 12, BF) == OK
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="needs a machine without a usable CUDA device")
+def test_cuda_failure_maps_to_status_and_message():
+    """Fault injection from the environment: with no usable device, every call that passes validation
+    fails in the CUDA runtime, returns GPTATTN_ERR_CUDA and leaves the runtime's message readable."""
+    assert ga.gptattn_fwd(FAKE, FAKE, FAKE, 2, 8, 128, 2, ga.GPTATTN_BF16, None) == ga.GPTATTN_ERR_CUDA
+    assert ga.gptattn_last_error_string() not in ("", "no error")
+    assert ga.gptattn_fwd(FAKE, FAKE, FAKE, 2, 8, 64, 4, ga.GPTATTN_F32, None) == ga.GPTATTN_ERR_CUDA
+    ws = ga.gptattn_bwd_workspace_bytes(2, 8, 128, 2, ga.GPTATTN_BF16)
+    assert ga.gptattn_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws, 2, 8, 128, 2, ga.GPTATTN_BF16, None) == \
+        ga.GPTATTN_ERR_CUDA
+    assert ga.gptattn_linear(FAKE, FAKE, None, None, FAKE, 8, 64, 64, ga.GPTATTN_BF16, None) == ga.GPTATTN_ERR_CUDA
+    assert ga.gptattn_get_device_status(None) == ga.GPTATTN_ERR_CUDA
