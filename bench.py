@@ -228,6 +228,43 @@ def make_block_call(ga, w, dev, s):
     return call, bufs
 
 
+# --------------------------------------------------------------------------- ranks
+# One process per GPU under torchrun.  Each rank runs the unchanged single-GPU op on a batch
+# of its own (independent problems: weak scaling, no collective on the data path); the only
+# collectives are the barriers around the timed region and the max of the ranks' times.
+def rank_seed(w, rank: int) -> int:
+    """Seed of a rank's synthetic batch: every rank draws different inputs."""
+    return 1000 + w.index + 7919 * rank
+
+
+def init_ranks(world: int, backend: str = "nccl", device=None):
+    """Process group for world > 1 (NCCL on GPUs; the CPU tests use gloo), short timeout; None at world 1."""
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    kw = {"device_id": device} if backend == "nccl" and device is not None else {}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    return dist
+
+
+def max_over_ranks(dist, x: float, device="cpu") -> float:
+    """The largest of the ranks' values (the job's time is the slowest rank's)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(world: int, steps: int, flops_per_step: float, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank ran `steps` steps of `flops_per_step` FLOPs, and the job
+    took as long as its slowest rank."""
+    return world * steps * flops_per_step / (max_total_ms / 1e3) / 1e12
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
 
@@ -236,17 +273,12 @@ def run_ours(args, w, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    dist = init_ranks(world, "nccl", dev)
 
     dt = ga.GPTATTN_BF16 if w.dtype == "bf16" else ga.GPTATTN_F32
     B, T, C, nh = w.B, w.T, w.C, w.n_head
-    qkv_c, dy_c = make_inputs(B, T, nh, w.hs, dtype=w.torch_dtype, seed=1000 + w.index + 7919 * rank,
-                              recipe=w.recipe, qkv_scale=w.qkv_scale)
+    qkv_c, dy_c = make_inputs(B, T, nh, w.hs, dtype=w.torch_dtype, seed=rank_seed(w, rank), recipe=w.recipe,
+                              qkv_scale=w.qkv_scale)
     qkv = qkv_c.to(dev)
     dy = dy_c.to(dev)
     y = torch.empty(B, T, C, dtype=w.torch_dtype, device=dev)
@@ -277,12 +309,8 @@ def run_ours(args, w, rank, world, local_rank):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x: float) -> float:
+        return max_over_ranks(dist, x, dev)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -335,9 +363,9 @@ def run_ours(args, w, rank, world, local_rank):
     ga.gptattn_profile_enable(0)
 
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms))
+    total_ms = slowest(sum(step_ms))
     flops = w.flops_fwd_bwd()
-    value = world * K * flops / (total_ms / 1e3) / 1e12
+    value = aggregate_tflops(world, K, flops, total_ms)
 
     # per-kernel durations recorded by the library inside the timed loop
     per_kernel = {}
@@ -405,8 +433,8 @@ def run_ours(args, w, rank, world, local_rank):
         e2e_run(Ke, e_start, e_end)
         e2e_ms = e_start.elapsed_time(e_end)
     barrier()
-    e2e_ms = max_over_ranks(e2e_ms)
-    e2e_value = world * Ke * flops / (e2e_ms / 1e3) / 1e12 if Ke else None
+    e2e_ms = slowest(e2e_ms)
+    e2e_value = aggregate_tflops(world, Ke, flops, e2e_ms) if Ke else None
     h2d = qkv_h.numel() * qkv_h.element_size() + dy_h.numel() * dy_h.element_size()
     d2h = y_h.numel() * y_h.element_size() + dqkv_h.numel() * dqkv_h.element_size()
 
