@@ -27,7 +27,9 @@
  * CUDA-core path).  lse and the workspace are float32 in both cases.
  *
  * Supported head sizes: bf16 hs in {64, 128}; f32 hs in {16, 32, 64, 128}.
- * Scale is fixed at 1/sqrt(hs); masking is always causal; no dropout.
+ * Scale is fixed at 1/sqrt(hs).  gptattn_fwd / gptattn_bwd are causal without
+ * dropout; the _window, _det and _opts entry points below add a local window,
+ * a deterministic backward and dropout on the attention weights.
  *
  * Ownership and synchronisation: every pointer is a caller-owned DEVICE
  * pointer on the current CUDA device, 16-byte aligned.  The library never
