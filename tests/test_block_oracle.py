@@ -42,6 +42,7 @@ def _load_mutant(tmp_path, name, text):
     return mod
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")  # broken copies may average empty slices
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_block_mutant_is_caught(orc, tmp_path, name, old, new):
     assert SRC.count(old) == 1, f"mutation anchor for {name} not unique"
