@@ -5,7 +5,6 @@ import importlib.util
 import numpy as np
 import pytest
 
-import oracle
 import oracle.block as block
 from block_pins import BLOCK_PINS
 

@@ -2,7 +2,6 @@
 each one trips at least one pin -- evidence that the pins constrain every
 step: the scale, the mask, the softmax shift, operand order and the backward
 terms."""
-import os
 
 import pytest
 

@@ -5,7 +5,6 @@ import pytest
 import torch
 
 import oracle
-from causal_self_attention_gptattn_b200 import gptattn as ga
 from causal_self_attention_gptattn_b200.workloads import WORKLOADS, make_inputs, workload_inputs
 from gpu_helpers import compare, run_fwd_bwd, select_heads
 
