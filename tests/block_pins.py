@@ -148,6 +148,18 @@ def pin_block_library_special_case(blk, orc):
     assert np.abs(out - ref.numpy()).max() < 1e-12
 
 
+def pin_block_regression_fixture(blk, orc):
+    """Regression fixture written by tests/golden/make_golden.py from this oracle:
+    catches any later change to the block oracle's arithmetic."""
+    import json
+    import os
+    fx = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "block_small_seeded.json")))
+    p = {k: np.array(fx[k]) for k in ("ln_w", "ln_b", "w_attn", "b_attn", "w_proj", "b_proj")}
+    out, qkv, y, lse = blk.attn_block_forward(np.array(fx["x"]), n_head=fx["n_head"], attention=orc.forward, **p)
+    for got, key in ((out, "out"), (qkv, "qkv"), (y, "y"), (lse, "lse")):
+        assert np.allclose(got, fx[key], rtol=0, atol=1e-12), key
+
+
 def pin_block_empty(blk, orc):
     """T = 0: nothing to compute, shapes preserved."""
     C = 8
@@ -166,4 +178,5 @@ BLOCK_PINS = [
     pin_block_prefix_average,
     pin_block_library_special_case,
     pin_block_empty,
+    pin_block_regression_fixture,
 ]
