@@ -13,10 +13,10 @@ each step follows.
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (closed forms, invariants, finite differences, a library special case and the
-worked fixtures under ``tests/golden/``), except the exact bits of the dropout
-generator (Philox4x32-10): PARITY UNPINNED for those bits (no known-answer
-vectors are available here); its statistics and every use of the mask are
-pinned.
+worked fixtures under ``tests/golden/``); the dropout generator (Philox4x32-10)
+is pinned by its published known-answer vectors
+(``tests/golden/philox4x32_10_kat.json``), its statistics and every use of the
+mask.
 """
 from __future__ import annotations
 

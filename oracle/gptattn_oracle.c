@@ -71,8 +71,9 @@
  * products' high and low words, and permutes them as
  *     (hi(M1*c2) ^ c1 ^ k0,  lo(M1*c2),  hi(M0*c0) ^ c3 ^ k1,  lo(M0*c0));
  * between rounds the key is advanced by the two Weyl constants.
- * PARITY UNPINNED for the generator's exact bits: no known-answer vectors are
- * available here; the pins check its statistics and every use of its output.
+ * Pinned by the generator's published known-answer vectors (the Random123
+ * library's list for philox4x32 with 10 rounds), besides its statistics and
+ * every use of its output.
  * ------------------------------------------------------------------------- */
 #define PHILOX_M0 0xD2511F53u
 #define PHILOX_M1 0xCD9E8D57u

@@ -15,8 +15,8 @@ t sees positions t-window < s <= t.  The dropout pins (``pin_dropout_*``) follow
 the lecture's chapter "scaling up the model! creating a few variables. adding
 dropout", read as inverted dropout on the attention weights with a Philox4x32-10
 keep mask (counter (s/4, t, b*n_head+h, 0), key = seed, word s%4, kept iff the
-word >= floor(p * 2^32)); the generator's own bits are not pinned (no
-known-answer vectors are available here), only its statistics.
+word >= floor(p * 2^32)); the generator's own bits are pinned by the published
+known-answer vectors of Philox4x32-10 (``tests/golden/philox4x32_10_kat.json``).
 """
 from __future__ import annotations
 
@@ -550,6 +550,22 @@ def pin_philox_statistics(orc):
     assert chi2 < 50  # 15 degrees of freedom: P(chi2 > 50) is about 1e-5
 
 
+def pin_philox_known_answers(orc):
+    """Philox4x32-10 reproduces the generator's published known-answer vectors
+    (the Random123 library's list for philox4x32 with 10 rounds, which accompanies
+    Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011): the
+    round count, both multipliers, the word permutation and the key schedule are
+    all fixed by these three outputs."""
+    fx = json.load(open(os.path.join(GOLDEN, "philox4x32_10_kat.json")))
+    assert fx["rounds"] == 10 and len(fx["vectors"]) == 3
+    for v in fx["vectors"]:
+        ctr = [int(w, 16) for w in v["ctr"]]
+        key = [int(w, 16) for w in v["key"]]
+        want = [int(w, 16) for w in v["out"]]
+        got = [int(w) for w in orc.philox(ctr, key)]
+        assert got == want, f"philox({v['ctr']}, {v['key']}) = {[f'{w:08x}' for w in got]}, want {v['out']}"
+
+
 ALL_PINS = [
     pin_row_identity,
     pin_single_token, pin_uniform_scores_prefix_mean, pin_tril_average_fixture,
@@ -560,5 +576,5 @@ ALL_PINS = [
     pin_window_one, pin_window_covers_all, pin_window_uniform_scores, pin_window_locality,
     pin_window_library_special_case, pin_window_finite_differences,
     pin_dropout_mask_and_scale, pin_dropout_counter_layout, pin_dropout_lse_unchanged_and_unbiased,
-    pin_dropout_finite_differences, pin_philox_statistics,
+    pin_dropout_finite_differences, pin_philox_statistics, pin_philox_known_answers,
 ]

@@ -41,6 +41,12 @@ MUTANTS = [
     ("dK_transposed_dS",
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);",
      "acc += dS[(size_t)s * (size_t)T + t] * qkv_at(qkv, T, C, hs, b, t, 0, h, d);"),
+    # the dropout generator: mistakes that keep its output uniform, so only the
+    # published known-answer vectors can catch them
+    ("philox_nine_rounds", "for (int round = 0; round < 10; ++round)", "for (int round = 0; round < 9; ++round)"),
+    ("philox_multipliers_swapped", "const uint64_t p0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;",
+     "const uint64_t p0 = (uint64_t)PHILOX_M1 * (uint64_t)c0;"),
+    ("philox_key_schedule_swapped", "k0 += PHILOX_W0;", "k0 += PHILOX_W1;"),
 ]
 
 
