@@ -9,9 +9,12 @@
 // this entry point takes its scratch from one fixed array compiled into the
 // library instead.
 //
-// The array lives in global memory of every GPU that loads the library and is
-// held until the process exits.  Its host-side name is only a stand-in for the
-// symbol: the device address is looked up once per device with
+// The array is a module global in device memory.  With CUDA's default lazy
+// module loading a device gets it when the first call on that device looks its
+// address up (which loads this file's module, so that first call does extra
+// work); with eager loading, when the library's device code is loaded.  Either
+// way the device holds it until the process exits.  Its host-side name is only a
+// stand-in for the symbol: the device address is looked up once per device with
 // cudaGetSymbolAddress (with that device current) on the first call made on
 // that device, and cached.  Every call shares the array and the previous
 // call's contents stay in it; the backward's first kernel rewrites every part

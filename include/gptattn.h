@@ -178,7 +178,9 @@ GPTATTN_API gptattn_status gptattn_decode(const void *qkv, void *y, float *lse,
                               gptattn_dtype dt, gptattn_stream_t stream);
 
 /* Bytes of device scratch gptattn_bwd needs for this shape (0 for an empty
- * shape; (size_t)-1 for an invalid one).  Pure host function. */
+ * shape; (size_t)-1 for an invalid one).  Pure host function.  No counterpart
+ * on the pages: the scratch (per-row softmax statistics and an fp32 dQ
+ * accumulator) belongs to this library's backward design, not to the method. */
 GPTATTN_API size_t gptattn_bwd_workspace_bytes(int B, int T, int C, int n_head, gptattn_dtype dt);
 
 /* Backward.  Given the forward's qkv, y and lse and the incoming gradient dy,
@@ -199,14 +201,18 @@ GPTATTN_API gptattn_status gptattn_bwd(const void *qkv, const void *y, const flo
  * on their path, since it can synchronise the device.  This entry point takes
  * the same arguments as gptattn_bwd minus the workspace: the scratch comes
  * from one array of GPTATTN_NOALLOC_SCRATCH_BYTES (64 MiB) compiled into the
- * library, which every GPU that loads the library holds until the process
+ * library.  The array is a module global of the library's device code: with
+ * CUDA's default lazy module loading a device gets it when this entry point's
+ * first call on that device loads the module (so that first call does extra
+ * work), with eager loading (CUDA_MODULE_LOADING=EAGER) when the library's
+ * device code is loaded; either way the device holds it until the process
  * exits.  The caller still owns and passes every input and output.
  * Returns GPTATTN_ERR_WORKSPACE, enqueueing nothing, when the shape needs more
  * scratch than that (gptattn_bwd_workspace_bytes(...) > 64 MiB).  It allocates
  * nothing: no cudaMalloc, cudaFree or allocating library routine.
  * The first call on each device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the previous call's
+ * device current), loading the module if needed, and caches it; make that
+ * first call before any stream capture.  All calls share the one array and it keeps the previous call's
  * contents (the backward re-initialises what it needs); calls whose work
  * overlaps on the GPU -- on two streams or from two host threads -- race on it
  * and produce wrong results, so serialise them. */
@@ -218,17 +224,19 @@ GPTATTN_API gptattn_status gptattn_bwd_noalloc(const void *qkv, const void *y, c
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: GPTATTN_OK, GPTATTN_ERR_TIMEOUT if a kernel gave up on
  * a wait since the last call, or GPTATTN_ERR_CUDA if the stream reports an
- * error. */
+ * error.  No counterpart on the pages: error reporting of this library. */
 GPTATTN_API gptattn_status gptattn_get_device_status(gptattn_stream_t stream);
 
-/* Static human-readable name of a status code. */
+/* Static human-readable name of a status code (no counterpart on the pages). */
 GPTATTN_API const char *gptattn_status_string(gptattn_status s);
 
 /* Text of the last CUDA error that made a call on this host thread return
- * GPTATTN_ERR_CUDA ("no error" if none yet).  Static string. */
+ * GPTATTN_ERR_CUDA ("no error" if none yet).  Static string.  No counterpart
+ * on the pages. */
 GPTATTN_API const char *gptattn_last_error_string(void);
 
-/* Library version, major * 10000 + minor * 100 + patch. */
+/* Library version, major * 10000 + minor * 100 + patch (no counterpart on the
+ * pages). */
 GPTATTN_API int gptattn_version(void);
 
 /* ---- The attention sub-block of a pre-LN GPT block (bf16 only) ------------
