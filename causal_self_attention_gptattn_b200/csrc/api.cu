@@ -254,7 +254,25 @@ __global__ void selftest_timeout_kernel(int *status, unsigned long long budget_n
     __syncthreads();
 }
 
+// The FMA-pipe exponential of the backward kernel, evaluated on caller data:
+// y[i] = exp2_poly_x2 of x[i] (pairs of elements per thread).
+__global__ void selftest_exp2_kernel(const float *__restrict__ x, float *__restrict__ y, int n) {
+    const long long i = 2ll * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+    float y0, y1;
+    exp2_poly_x2(x0, x1, y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_exp2(const float *x, float *y, int n, cudaStream_t s) {
+    const long long pairs = ((long long)n + 1) / 2;
+    selftest_exp2_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(x, y, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s) {
     selftest_timeout_kernel<<<1, 32, 0, s>>>(ctx.status, ctx.budget_ns);
@@ -687,6 +705,15 @@ gptattn_status gptattn_selftest_wait_timeout(unsigned long long budget_ns, gptat
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const DevCtx ctx{status, budget_ns};
     return from_cuda(run_kernel(kKSelftest, s, [&] { return launch_selftest_timeout(ctx, s); }));
+}
+
+gptattn_status gptattn_selftest_exp2(const float *x, float *y, int n, gptattn_stream_t stream) {
+    if (n < 0) return GPTATTN_ERR_INVALID_ARG;
+    if (n == 0) return GPTATTN_OK;
+    if (!x || !y || (reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u))
+        return GPTATTN_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return from_cuda(run_kernel(kKSelftest, s, [&] { return launch_selftest_exp2(x, y, n, s); }));
 }
 
 }  // extern "C"

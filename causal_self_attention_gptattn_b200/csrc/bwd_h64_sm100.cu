@@ -24,13 +24,14 @@
 // reversed on odd rounds), which evens out the causal triangle's work across
 // CTAs.  Per item the CTA loops over query tiles i >= j.
 //
-// Warp roles (14 warps):
+// Warp roles (16 warps, four warpgroups; setmaxnreg moves registers from the
+// first warpgroup to the last):
 //   warp 0        TMA producer: K_j, V_j (double-buffered across items), and
 //                 Q_i, dO_i, lse_i, D_i through a 3-stage ring
-//   warp 1        TMEM owner + MMA issuer
-//   warps 2..9    softmax: TMEM sub-partition warp%4 (32 key rows), column
-//                 half (warp-2)/4 (64 query columns): P^T, dS^T
-//   warps 10..13  dQ drain: TMEM -> smem (fp32, swizzled) -> TMA reduce-add;
+//   warp 1        TMEM owner + MMA issuer (warps 2, 3 idle)
+//   warps 4..11   softmax: TMEM sub-partition warp%4 (32 key rows), column
+//                 half warp/4 - 1 (64 query columns): P^T, dS^T
+//   warps 12..15  dQ drain: TMEM -> smem (fp32, swizzled) -> TMA reduce-add;
 //                 and per item the dK/dV epilogue (TMEM -> bf16 -> TMA store)
 // TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T [256,320) (bf16 pairs)
 //                     dV [320,384)  dK [384,448)  dQ [448,512)
@@ -47,7 +48,12 @@
 namespace gptattn {
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 512;
+// register budgets per thread of the four warpgroups (sum = 4 x kLaunchRegs, what the
+// CTA is launched with)
+constexpr int kLaunchRegs = 128;
+constexpr uint32_t kRegsCtl = 96, kRegsSoftmax = 144, kRegsDrain = 128;
+static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsDrain == 4 * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr int HS = 64;
@@ -107,29 +113,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
-// 2^x for a pair of x <= ~1 on the FMA pipe, to take part of the exponentials off the
-// multi-function unit: Cody-Waite style reduction x = j + f with j an integer (rounded by
-// adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it on that interval by
-// weighted least squares (relative error below 7.6e-5); j added to the exponent field.
-// x is clamped at -125, so results below 2^-125 come out as about 2^-125 instead of 0.
-__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float &y0, float &y1) {
-    const uint64_t x = f32x2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = fadd2(x, f32x2_pack(12582912.f, 12582912.f));           // 1.5 * 2^23 + j
-    const uint64_t xi = fadd2(t, f32x2_pack(-12582912.f, -12582912.f));         // j
-    const uint64_t f = ffma2(xi, f32x2_pack(-1.f, -1.f), x);                    // x - j
-    uint64_t p = ffma2(f32x2_pack(0.05517605319619179f, 0.05517605319619179f), f,
-                       f32x2_pack(0.24261149764060974f, 0.24261149764060974f));
-    p = ffma2(p, f, f32x2_pack(0.6932601928710938f, 0.6932601928710938f));
-    p = ffma2(p, f, f32x2_pack(0.9999280571937561f, 0.9999280571937561f));
-    float p0, p1, t0, t1;
-    f32x2_unpack(p, p0, p1);
-    f32x2_unpack(t, t0, t1);
-    // the low mantissa bits of t hold j; shifted into the exponent field (the constant's own
-    // bits shift out of the word)
-    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // Last query tile that key tile kt's band reaches.
 __device__ __forceinline__ int band_hi_tile(int kt, int window, int n_t) {
     const long long t = (long long)kt * kTile + kTile - 2 + window;  // largest key + window - 1
@@ -154,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
     const int BH = B * n_head;
     const int n_items = n_t * BH;
 
@@ -207,160 +191,164 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_launch_dependents();
     griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
-    if (warp == 0) {
-        // ================================================================ producer
-        if (lane == 0) {
-            tma_prefetch_map(&map_qkv);
-            tma_prefetch_map(&map_dy);
-            bool ok = true;
-            int n = 0;   // items started
-            int gq = 0;  // query tiles issued (ring position)
-            for (int k = 0; ok; ++k, ++n) {
-                const int w = item_index(k, blockIdx.x, gridDim.x);
-                if (w >= n_items) break;
-                const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
-                const int kvs = n & 1;
-                if (n >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + kvs), (uint32_t)((n >> 1) & 1) ^ 1u, g)))
-                    break;
-                mbar_arrive_expect_tx(bar(kBarKVFull + kvs), 2 * kTileBytes);
-                tma_load_3d(sK(kvs), &map_qkv, bar(kBarKVFull + kvs), C + h * HS, kt * kTile, b);
-                tma_load_3d(sV(kvs), &map_qkv, bar(kBarKVFull + kvs), 2 * C + h * HS, kt * kTile, b);
-                const int qt_end = band_hi_tile(kt, window, n_t);
-                for (int qt = kt; qt <= qt_end; ++qt, ++gq) {
-                    const int st = gq % kQStages;
-                    const uint32_t ph = (uint32_t)(gq / kQStages) & 1u;
-                    if (gq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + st), ph ^ 1u, g))) break;
-                    const uint32_t fb = bar(kBarQFull + st);
-                    mbar_arrive_expect_tx(fb, 2 * kTileBytes + 1024);
-                    tma_load_3d(sQ(st), &map_qkv, fb, h * HS, qt * kTile, b);
-                    tma_load_3d(sdO(st), &map_dy, fb, h * HS, qt * kTile, b);
-                    const size_t rowoff = (size_t)bh * (size_t)T_pad + (size_t)qt * kTile;
-                    bulk_load(sbase + kOffLse + st * 512, lse2 + rowoff, 512, fb);
-                    bulk_load(sbase + kOffD + st * 512, Dvec + rowoff, 512, fb);
+    if (wg == 0) {
+        regs_dec<kRegsCtl>();
+        if (warp == 0) {
+            // ================================================================ producer
+            if (lane == 0) {
+                tma_prefetch_map(&map_qkv);
+                tma_prefetch_map(&map_dy);
+                bool ok = true;
+                int n = 0;   // items started
+                int gq = 0;  // query tiles issued (ring position)
+                for (int k = 0; ok; ++k, ++n) {
+                    const int w = item_index(k, blockIdx.x, gridDim.x);
+                    if (w >= n_items) break;
+                    const int kt = w / BH, bh = w % BH, b = bh / n_head, h = bh % n_head;
+                    const int kvs = n & 1;
+                    if (n >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + kvs), (uint32_t)((n >> 1) & 1) ^ 1u, g)))
+                        break;
+                    mbar_arrive_expect_tx(bar(kBarKVFull + kvs), 2 * kTileBytes);
+                    tma_load_3d(sK(kvs), &map_qkv, bar(kBarKVFull + kvs), C + h * HS, kt * kTile, b);
+                    tma_load_3d(sV(kvs), &map_qkv, bar(kBarKVFull + kvs), 2 * C + h * HS, kt * kTile, b);
+                    const int qt_end = band_hi_tile(kt, window, n_t);
+                    for (int qt = kt; qt <= qt_end; ++qt, ++gq) {
+                        const int st = gq % kQStages;
+                        const uint32_t ph = (uint32_t)(gq / kQStages) & 1u;
+                        if (gq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + st), ph ^ 1u, g))) break;
+                        const uint32_t fb = bar(kBarQFull + st);
+                        mbar_arrive_expect_tx(fb, 2 * kTileBytes + 1024);
+                        tma_load_3d(sQ(st), &map_qkv, fb, h * HS, qt * kTile, b);
+                        tma_load_3d(sdO(st), &map_dy, fb, h * HS, qt * kTile, b);
+                        const size_t rowoff = (size_t)bh * (size_t)T_pad + (size_t)qt * kTile;
+                        bulk_load(sbase + kOffLse + st * 512, lse2 + rowoff, 512, fb);
+                        bulk_load(sbase + kOffD + st * 512, Dvec + rowoff, 512, fb);
+                    }
+                }
+                if (!ok || *abort_flag) {
+                    // let the last copies of each buffer land before shared memory is released
+                    for (int k = (n > kKVStages ? n - kKVStages : 0); k < n; ++k)
+                        drain_wait(bar(kBarKVFull + (k & 1)), (uint32_t)(k >> 1) & 1u, budget_ns);
+                    for (int k = (gq > kQStages ? gq - kQStages : 0); k < gq; ++k)
+                        drain_wait(bar(kBarQFull + k % kQStages), (uint32_t)(k / kQStages) & 1u, budget_ns);
                 }
             }
-            if (!ok || *abort_flag) {
-                // let the last copies of each buffer land before shared memory is released
-                for (int k = (n > kKVStages ? n - kKVStages : 0); k < n; ++k)
-                    drain_wait(bar(kBarKVFull + (k & 1)), (uint32_t)(k >> 1) & 1u, budget_ns);
-                for (int k = (gq > kQStages ? gq - kQStages : 0); k < gq; ++k)
-                    drain_wait(bar(kBarQFull + k % kQStages), (uint32_t)(k / kQStages) & 1u, budget_ns);
-            }
-        }
-    } else if (warp == 1) {
-        // ================================================================ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idSS = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idAcc = idesc_bf16_f32(128, HS, false, true);
-            constexpr uint32_t idQ = idesc_bf16_f32(128, HS, true, true);
-            // Descriptors of every buffer, built once.  K-major views: rows of 128 B,
-            // 8-row groups 1024 B apart.  N/M-major views: 8-row groups 1024 B apart,
-            // 64-element column blocks one slab apart.  A k-step moves the start address.
-            const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024), dV0 = sdesc_sw128(sV(0), 16, 1024);
-            const uint64_t dQ0 = sdesc_sw128(sQ(0), 16, 1024), ddO0 = sdesc_sw128(sdO(0), 16, 1024);
-            const uint64_t ddOmn0 = sdesc_sw128(sdO(0), kSlabBytes, 1024), dQmn0 = sdesc_sw128(sQ(0), kSlabBytes, 1024);
-            const uint64_t dKmn0 = sdesc_sw128(sK(0), kSlabBytes, 1024);
-            const uint64_t ddS = sdesc_sw128(sdS, 16, 1024), ddSmn = sdesc_sw128(sdS, kSlabBytes, 1024);
-            auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
-            bool ok = true, any = false;
-            int n = 0, gi = 0;
-            auto issue_S = [&](int kvs, int st) {
-                const uint64_t a = at(dK0, kvs * kTileBytes), b = at(dQ0, st * kTileBytes);
-#pragma unroll
-                for (int kk = 0; kk < HS / 16; ++kk)
-                    umma_ss(tmem + kColS, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
-                umma_commit(bar(kBarSFull));
-            };
-            auto issue_dP = [&](int kvs, int st) {
-                const uint64_t a = at(dV0, kvs * kTileBytes), b = at(ddO0, st * kTileBytes);
-#pragma unroll
-                for (int kk = 0; kk < HS / 16; ++kk)
-                    umma_ss(tmem + kColdP, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
-                umma_commit(bar(kBardPFull));
-            };
-            for (int k = 0; ok; ++k, ++n) {
-                const int w = item_index(k, blockIdx.x, gridDim.x);
-                if (w >= n_items) break;
-                const int kt = w / BH;
-                const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
-                const int kvs = n & 1;
-                if (!(ok = mbar_wait(bar(kBarKVFull + kvs), (uint32_t)(n >> 1) & 1u, g))) break;
-                // first S and dP of this item
-                if (!(ok = mbar_wait(bar(kBarQFull + gi % kQStages), (uint32_t)(gi / kQStages) & 1u, g))) break;
-                if (gi > 0 && !(ok = mbar_wait(bar(kBarSEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
-                tc_fence_after();
-                issue_S(kvs, gi % kQStages);
-                any = true;
-                if (gi > 0 && !(ok = mbar_wait(bar(kBardPEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
-                tc_fence_after();
-                issue_dP(kvs, gi % kQStages);
-                for (int it = 0; it < niter; ++it, ++gi) {
-                    const int st = gi % kQStages;
-                    const int st1 = (gi + 1) % kQStages;
-                    const bool more = it + 1 < niter;
-                    const uint32_t ph = (uint32_t)gi & 1u;
-                    if (more) {  // S^T of the next query tile
-                        if (!(ok = mbar_wait(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u, g))) break;
-                        if (!(ok = mbar_wait(bar(kBarSEmpty), ph, g))) break;
+        } else if (warp == 1) {
+            // ================================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idSS = idesc_bf16_f32(128, 128, false, false);
+                constexpr uint32_t idAcc = idesc_bf16_f32(128, HS, false, true);
+                constexpr uint32_t idQ = idesc_bf16_f32(128, HS, true, true);
+                // Descriptors of every buffer, built once.  K-major views: rows of 128 B,
+                // 8-row groups 1024 B apart.  N/M-major views: 8-row groups 1024 B apart,
+                // 64-element column blocks one slab apart.  A k-step moves the start address.
+                const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024), dV0 = sdesc_sw128(sV(0), 16, 1024);
+                const uint64_t dQ0 = sdesc_sw128(sQ(0), 16, 1024), ddO0 = sdesc_sw128(sdO(0), 16, 1024);
+                const uint64_t ddOmn0 = sdesc_sw128(sdO(0), kSlabBytes, 1024), dQmn0 = sdesc_sw128(sQ(0), kSlabBytes, 1024);
+                const uint64_t dKmn0 = sdesc_sw128(sK(0), kSlabBytes, 1024);
+                const uint64_t ddS = sdesc_sw128(sdS, 16, 1024), ddSmn = sdesc_sw128(sdS, kSlabBytes, 1024);
+                auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+                bool ok = true, any = false;
+                int n = 0, gi = 0;
+                auto issue_S = [&](int kvs, int st) {
+                    const uint64_t a = at(dK0, kvs * kTileBytes), b = at(dQ0, st * kTileBytes);
+    #pragma unroll
+                    for (int kk = 0; kk < HS / 16; ++kk)
+                        umma_ss(tmem + kColS, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar(kBarSFull));
+                };
+                auto issue_dP = [&](int kvs, int st) {
+                    const uint64_t a = at(dV0, kvs * kTileBytes), b = at(ddO0, st * kTileBytes);
+    #pragma unroll
+                    for (int kk = 0; kk < HS / 16; ++kk)
+                        umma_ss(tmem + kColdP, at(a, kk * 32u), at(b, kk * 32u), idSS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar(kBardPFull));
+                };
+                for (int k = 0; ok; ++k, ++n) {
+                    const int w = item_index(k, blockIdx.x, gridDim.x);
+                    if (w >= n_items) break;
+                    const int kt = w / BH;
+                    const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
+                    const int kvs = n & 1;
+                    if (!(ok = mbar_wait(bar(kBarKVFull + kvs), (uint32_t)(n >> 1) & 1u, g))) break;
+                    // first S and dP of this item
+                    if (!(ok = mbar_wait(bar(kBarQFull + gi % kQStages), (uint32_t)(gi / kQStages) & 1u, g))) break;
+                    if (gi > 0 && !(ok = mbar_wait(bar(kBarSEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                    tc_fence_after();
+                    issue_S(kvs, gi % kQStages);
+                    any = true;
+                    if (gi > 0 && !(ok = mbar_wait(bar(kBardPEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                    tc_fence_after();
+                    issue_dP(kvs, gi % kQStages);
+                    for (int it = 0; it < niter; ++it, ++gi) {
+                        const int st = gi % kQStages;
+                        const int st1 = (gi + 1) % kQStages;
+                        const bool more = it + 1 < niter;
+                        const uint32_t ph = (uint32_t)gi & 1u;
+                        if (more) {  // S^T of the next query tile
+                            if (!(ok = mbar_wait(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u, g))) break;
+                            if (!(ok = mbar_wait(bar(kBarSEmpty), ph, g))) break;
+                            tc_fence_after();
+                            issue_S(kvs, st1);
+                        }
+                        // dV += P^T dO
+                        if (!(ok = mbar_wait(bar(kBarPFull), ph, g))) break;
+                        if (it == 0 && n > 0 && !(ok = mbar_wait(bar(kBarAccFree), (uint32_t)(n - 1) & 1u, g))) break;
                         tc_fence_after();
-                        issue_S(kvs, st1);
-                    }
-                    // dV += P^T dO
-                    if (!(ok = mbar_wait(bar(kBarPFull), ph, g))) break;
-                    if (it == 0 && n > 0 && !(ok = mbar_wait(bar(kBarAccFree), (uint32_t)(n - 1) & 1u, g))) break;
-                    tc_fence_after();
-                    {
-                        const uint64_t b = at(ddOmn0, st * kTileBytes);
-                        const uint32_t acc = it > 0 ? 1u : 0u;
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, at(b, kk * 2048u), idAcc, kk > 0 ? 1u : acc);
-                    }
-                    umma_commit(bar(kBarPEmpty));
-                    // dP^T of the next query tile, ahead of this tile's dK and dQ (which wait for
-                    // this tile's dS), so the softmax warps find it ready when they reach it
-                    if (more) {
-                        if (!(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
+                        {
+                            const uint64_t b = at(ddOmn0, st * kTileBytes);
+                            const uint32_t acc = it > 0 ? 1u : 0u;
+    #pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, at(b, kk * 2048u), idAcc, kk > 0 ? 1u : acc);
+                        }
+                        umma_commit(bar(kBarPEmpty));
+                        // dP^T of the next query tile, ahead of this tile's dK and dQ (which wait for
+                        // this tile's dS), so the softmax warps find it ready when they reach it
+                        if (more) {
+                            if (!(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
+                            tc_fence_after();
+                            issue_dP(kvs, st1);
+                        }
+                        // dK += dS^T Q ; dQ = dS K
+                        if (!(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
                         tc_fence_after();
-                        issue_dP(kvs, st1);
+                        {
+                            const uint64_t b = at(dQmn0, st * kTileBytes);
+                            const uint32_t acc = it > 0 ? 1u : 0u;
+    #pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                umma_ss(tmem + kColdK, at(ddS, (kk >> 2) * kSlabBytes + (kk & 3) * 32u), at(b, kk * 2048u),
+                                        idAcc, kk > 0 ? 1u : acc);
+                        }
+                        // dK was the last reader of Q_i and dO_i (dQ reads dS and K): release their stage
+                        umma_commit(bar(kBarQEmpty + st));
+                        if (gi > 0 && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                        tc_fence_after();
+                        {
+                            const uint64_t b = at(dKmn0, kvs * kTileBytes);
+    #pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                umma_ss(tmem + kColdQ, at(ddSmn, kk * 2048u), at(b, kk * 2048u), idQ, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar(kBardQFull));
+                        umma_commit(bar(kBardSEmpty));
                     }
-                    // dK += dS^T Q ; dQ = dS K
-                    if (!(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
-                    tc_fence_after();
-                    {
-                        const uint64_t b = at(dQmn0, st * kTileBytes);
-                        const uint32_t acc = it > 0 ? 1u : 0u;
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_ss(tmem + kColdK, at(ddS, (kk >> 2) * kSlabBytes + (kk & 3) * 32u), at(b, kk * 2048u),
-                                    idAcc, kk > 0 ? 1u : acc);
-                    }
-                    // dK was the last reader of Q_i and dO_i (dQ reads dS and K): release their stage
-                    umma_commit(bar(kBarQEmpty + st));
-                    if (gi > 0 && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
-                    tc_fence_after();
-                    {
-                        const uint64_t b = at(dKmn0, kvs * kTileBytes);
-#pragma unroll
-                        for (int kk = 0; kk < 8; ++kk)
-                            umma_ss(tmem + kColdQ, at(ddSmn, kk * 2048u), at(b, kk * 2048u), idQ, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar(kBardQFull));
-                    umma_commit(bar(kBardSEmpty));
+                    if (!ok) break;
+                    umma_commit(bar(kBarKdV));
+                    umma_commit(bar(kBarKVEmpty + kvs));
                 }
-                if (!ok) break;
-                umma_commit(bar(kBarKdV));
-                umma_commit(bar(kBarKVEmpty + kvs));
-            }
-            if (any) {
-                umma_commit(bar(kBarDone));
-                drain_wait(bar(kBarDone), 0, budget_ns);
+                if (any) {
+                    umma_commit(bar(kBarDone));
+                    drain_wait(bar(kBarDone), 0, budget_ns);
+                }
             }
         }
-    } else if (warp < 10) {
+    } else if (wg < 3) {
+        regs_inc<kRegsSoftmax>();
         // ================================================================ softmax warps
         const int sp = warp & 3;                 // TMEM sub-partition: key rows 32*sp .. 32*sp+31
-        const int half = (warp - 2) >> 2;        // query columns 64*half .. 64*half+63
+        const int half = wg - 1;                 // query columns 64*half .. 64*half+63
         const int row = sp * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
         const float scale_log2 = 0.125f * 1.4426950408889634f;
@@ -506,12 +494,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ================================================================ dQ drain warps
+        regs_inc<kRegsDrain>();
         const int sp = warp & 3;
         const int row = sp * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
-        const bool leader = (warp == 10 && lane == 0);
+        const bool leader = (warp == 12 && lane == 0);
         bool ok = true;
         int gi = 0;
+        // 32 words as row `row` of the staging slab (128-byte swizzled); the slab's previous
+        // copy-out must have read it first
+        auto stage = [&](const uint32_t *v) {
+            if (leader) bulk_wait_group_read_0();
+            named_bar_sync(2, kDrainThreads);
+            if (ok) {
+                const uint32_t rbase = sdQ + (uint32_t)row * 128u;
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), v[4 * q], v[4 * q + 1],
+                                 v[4 * q + 2], v[4 * q + 3]);
+                fence_proxy_async_smem();
+            }
+            named_bar_sync(2, kDrainThreads);
+        };
         for (int k = 0, n = 0;; ++k, ++n) {
             const int w = item_index(k, blockIdx.x, gridDim.x);
             if (w >= n_items) break;
@@ -529,17 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {  // two 32-column halves through one 16 KB staging slab
-                    if (leader) bulk_wait_group_read_0();
-                    named_bar_sync(2, kDrainThreads);
-                    if (ok) {
-                        const uint32_t rbase = sdQ + (uint32_t)row * 128u;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), v[32 * hh + 4 * q],
-                                         v[32 * hh + 4 * q + 1], v[32 * hh + 4 * q + 2], v[32 * hh + 4 * q + 3]);
-                        fence_proxy_async_smem();
-                    }
-                    named_bar_sync(2, kDrainThreads);
+                    stage(&v[32 * hh]);
                     if (leader && ok && !*abort_flag) {
                         if (n_slots == 0)  // add into the (b, h, query tile) rows of the accumulator
                             tma_reduce_add_2d(&map_dq, sdQ, 32 * hh, bh * T_pad + qt * kTile);
@@ -574,17 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(bar(kBarAccFree));  // the next item's dV / dK may overwrite the accumulators
                     }
                 }
-                if (leader) bulk_wait_group_read_0();
-                named_bar_sync(2, kDrainThreads);
-                if (ok) {
-                    const uint32_t rbase = sdQ + (uint32_t)row * 128u;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), pv[4 * q], pv[4 * q + 1],
-                                     pv[4 * q + 2], pv[4 * q + 3]);
-                    fence_proxy_async_smem();
-                }
-                named_bar_sync(2, kDrainThreads);
+                stage(pv);
                 if (leader && ok && !*abort_flag) {
                     tma_store_3d(&map_dqkv, sdQ, (which == 0 ? 2 * C : C) + h * HS, kt * kTile, b);
                     bulk_commit_group();
@@ -612,6 +596,12 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
+    // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs per
+    // thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

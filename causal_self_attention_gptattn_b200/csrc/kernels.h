@@ -119,6 +119,8 @@ cudaError_t launch_layernorm_bf16(const void *x, const void *w, const void *b, v
 
 // ---- bounded-wait self-test -----------------------------------------------
 cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s);
+// ---- the backward's FMA-pipe exponential on caller data ---------------------
+cudaError_t launch_selftest_exp2(const float *x, float *y, int n, cudaStream_t s);
 
 // Kernel identifiers for the instrumentation records.
 enum KernelId {

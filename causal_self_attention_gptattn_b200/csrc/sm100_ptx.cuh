@@ -153,6 +153,25 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 __device__ __forceinline__ void bulk_wait_group_read_0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_group_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_group_0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups are pending, writes included.
+__device__ __forceinline__ void bulk_wait_group_1() { asm volatile("cp.async.bulk.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_2() { asm volatile("cp.async.bulk.wait_group 2;" ::: "memory"); }
+// Order this thread's global-memory accesses across the generic and async proxies
+// (bulk copies, TMA reductions) in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// gpu-scope acquire load / acquire-release add on a global counter
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t *p, uint32_t x) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(x) : "memory");
+    return old;
+}
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -252,6 +271,40 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// TMEM loads without their wait, for software pipelining: issue the next load,
+// work on the previous one, then tmem_ld_wait() on the new destination.  The
+// wait names the destination registers as in-out operands, so no use of them
+// can be scheduled before it.
+__device__ __forceinline__ void tmem_ld_x32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr) : "memory");
+}
+__device__ __forceinline__ void tmem_ld_x16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr) : "memory");
+}
+// Wait for every outstanding TMEM load of this thread; a (32 + 16)-register
+// destination set is threaded through the wait.
+__device__ __forceinline__ void tmem_ld_wait_48(uint32_t (&a)[32], uint32_t (&b)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31]),
+                   "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]), "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15])
+                 :: "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait_32(uint32_t (&a)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]), "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]), "+r"(a[29]), "+r"(a[30]), "+r"(a[31])
+                 :: "memory");
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
 // TMEM address of (lane, column) relative to an allocation base.
 __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) {
     return base + (lane << 16) + col;
@@ -309,6 +362,38 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
 }
+// max that returns NaN when either input is NaN
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// 2^x for a pair of x <= ~1 on the FMA pipe, to take part of the exponentials off the
+// multi-function unit: Cody-Waite style reduction x = j + f with j an integer (rounded by
+// adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a cubic fitted to it on that interval by
+// weighted least squares (relative error below 7.6e-5); then scaled by 2^j, built in the
+// exponent field (exact: j >= -125 keeps it a normal number).  x is clamped below at -125,
+// so results under 2^-125 (including x = -inf) come out as about 2^-125 instead of 0:
+// callers zero masked weights explicitly.  A NaN x gives NaN.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float &y0, float &y1) {
+    const uint64_t x = f32x2_pack(fmax_nan(x0, -125.f), fmax_nan(x1, -125.f));
+    const uint64_t t = fadd2(x, f32x2_pack(12582912.f, 12582912.f));           // 1.5 * 2^23 + j
+    const uint64_t xi = fadd2(t, f32x2_pack(-12582912.f, -12582912.f));         // j
+    const uint64_t f = ffma2(xi, f32x2_pack(-1.f, -1.f), x);                    // x - j
+    uint64_t p = ffma2(f32x2_pack(0.05517605319619179f, 0.05517605319619179f), f,
+                       f32x2_pack(0.24261149764060974f, 0.24261149764060974f));
+    p = ffma2(p, f, f32x2_pack(0.6932601928710938f, 0.6932601928710938f));
+    p = ffma2(p, f, f32x2_pack(0.9999280571937561f, 0.9999280571937561f));
+    float t0, t1;
+    f32x2_unpack(t, t0, t1);
+    // the low mantissa bits of t hold j; shifted into the exponent field (the constant's own
+    // bits shift out of the word) of 1.0, that is 2^j
+    const float s0 = __uint_as_float((__float_as_uint(t0) << 23) + 0x3F800000u);
+    const float s1 = __uint_as_float((__float_as_uint(t1) << 23) + 0x3F800000u);
+    f32x2_unpack(fmul2(p, f32x2_pack(s0, s1)), y0, y1);
+}
+
 // max of three floats in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;

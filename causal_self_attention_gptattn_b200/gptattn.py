@@ -33,6 +33,7 @@ EXPORTED = (
     "gptattn_status_string", "gptattn_version", "gptattn_profile_enable", "gptattn_profile_read",
     "gptattn_kernel_name", "gptattn_launch_count", "gptattn_selftest_wait_timeout", "gptattn_bwd_noalloc",
     "gptattn_last_error_string", "gptattn_layernorm", "gptattn_linear", "gptattn_attn_block_fwd",
+    "gptattn_selftest_exp2",
 )
 
 
@@ -122,6 +123,8 @@ def lib():
             L.gptattn_launch_count.restype = ctypes.c_ulonglong
             L.gptattn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, st]
             L.gptattn_selftest_wait_timeout.restype = i
+            L.gptattn_selftest_exp2.argtypes = [vp, vp, i, st]
+            L.gptattn_selftest_exp2.restype = i
             L.gptattn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, st]
             L.gptattn_bwd_noalloc.restype = i
             L.gptattn_last_error_string.argtypes = []
@@ -272,6 +275,10 @@ def gptattn_launch_count() -> int:
 
 def gptattn_selftest_wait_timeout(budget_ns: int, stream=None) -> int:
     return lib().gptattn_selftest_wait_timeout(budget_ns, _stream(stream))
+
+
+def gptattn_selftest_exp2(x, y, n: int, stream=None) -> int:
+    return lib().gptattn_selftest_exp2(_ptr(x), _ptr(y), n, _stream(stream))
 
 
 def check(status: int, where: str) -> None:

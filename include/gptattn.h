@@ -303,6 +303,20 @@ GPTATTN_API unsigned long long gptattn_launch_count(void);
  * budget_ns must be in [1000, 2000000000]. */
 GPTATTN_API gptattn_status gptattn_selftest_wait_timeout(unsigned long long budget_ns, gptattn_stream_t stream);
 
+/* ---- Exponential self-test (no counterpart on the pages) --------------------
+ * The backward kernel computes part of its softmax exponentials 2^x on the FMA
+ * pipe instead of the multi-function unit: x = j + f with j = round(x), 2^f by
+ * a cubic fitted on [-1/2, 1/2] by weighted least squares, j added to the
+ * exponent field (Cody-Waite style range reduction).  This entry point runs
+ * that routine on caller data so its accuracy can be tested: y[i] = the
+ * routine's 2^x[i] for i < n.  Stated behaviour: relative error below 7.6e-5
+ * for -125 <= x <= 1.5; x < -125 (including -inf) gives about 2^-125 rather
+ * than 0 (the kernels zero masked weights explicitly); NaN gives NaN.  x and y
+ * are device float arrays (4-byte aligned, may not overlap); n < 0 or a NULL /
+ * misaligned pointer -> GPTATTN_ERR_INVALID_ARG; n == 0 is a no-op.  Enqueued
+ * on `stream`, no synchronisation. */
+GPTATTN_API gptattn_status gptattn_selftest_exp2(const float *x, float *y, int n, gptattn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
