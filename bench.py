@@ -269,6 +269,68 @@ def aggregate_tflops(world: int, steps: int, flops_per_step: float, max_total_ms
     return world * steps * flops_per_step / (max_total_ms / 1e3) / 1e12
 
 
+def time_other_workload(ga, name, dev, s, flush, steps):
+    """One fwd+bwd step of another workload timed like the headline one (L2 flushed before
+    each step, CUDA events around it), then a per-kernel pass; returns its record."""
+    import torch
+
+    from causal_self_attention_gptattn_b200.workloads import by_name, workload_inputs
+    ow = by_name(name)
+    B, T, C, nh = ow.B, ow.T, ow.C, ow.n_head
+    dt = ga.GPTATTN_BF16
+    qkv_c, dy_c = workload_inputs(ow)
+    qkv, dy = qkv_c.to(dev), dy_c.to(dev)
+    y = torch.empty(B, T, C, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, nh, T, dtype=torch.float32, device=dev)
+    dqkv = torch.empty_like(qkv)
+    nb = ga.gptattn_bwd_workspace_bytes(B, T, C, nh, dt)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+    def step():
+        ga.check(ga.gptattn_fwd(qkv, y, lse, B, T, C, nh, dt, s), "gptattn_fwd")
+        ga.check(ga.gptattn_bwd(qkv, y, lse, dy, dqkv, ws, nb, B, T, C, nh, dt, s), "gptattn_bwd")
+
+    for _ in range(5):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    Ko = max(1, min(steps, 200))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ko)]
+    for a, b_ in evs:
+        flush.zero_()
+        a.record(s)
+        step()
+        b_.record(s)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b_) for a, b_ in evs) / Ko
+    ga.gptattn_profile_enable(4 * Ko + 64)
+    for _ in range(Ko):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    per = {}
+    for kname, kms in ga.gptattn_profile_read(4 * Ko + 64):
+        per.setdefault(kname, []).append(kms)
+    ga.gptattn_profile_enable(0)
+    ga.check(ga.gptattn_get_device_status(s), f"device status after {name}")
+    kern = {k: statistics.mean(v) for k, v in per.items()}
+    peaks, src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    bwd_ms = kern.get("bwd_bf16_sm100")
+    fwd_ms = kern.get("fwd_bf16_sm100")
+    return {"config": ow.describe(), "steps": Ko, "ms_per_step": ms, "flops_per_step": ow.flops_fwd_bwd(),
+            "value": ow.flops_fwd_bwd() / (ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "pct_of_measured_bf16_burst": ow.flops_fwd_bwd() / (ms / 1e3) / 1e12 / peak,
+            "kernels_ms": kern,
+            "roofline": {"bound": "tensor", "kernel": "bwd_bf16_sm100",
+                         "achieved": (ow.flops_bwd() / (bwd_ms / 1e3) / 1e12 if bwd_ms else None), "peak": peak,
+                         "unit": "TFLOP/s",
+                         "frac": (ow.flops_bwd() / (bwd_ms / 1e3) / 1e12 / peak if bwd_ms else None),
+                         "peak_source": f"{src} bf16 burst"},
+            "fwd_frac_of_peak": (ow.flops_fwd() / (fwd_ms / 1e3) / 1e12 / peak if fwd_ms else None),
+            "l2": "flushed before every timed step"}
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
 
@@ -651,6 +713,16 @@ def run_ours(args, w, rank, world, local_rank):
             "peak_source": f"{src_b} bf16 burst / copy bandwidth", "calls": Kb}
         del block_bufs
 
+    # ---- the other bf16 workloads of the configuration list, each timed like the headline
+    # workload (L2 flushed before every step, CUDA events per step), plus per-kernel times
+    # and the main backward kernel's fraction of the bf16 peak.  Single GPU only.
+    others = None
+    if not args.profile_run and world == 1 and dt == ga.GPTATTN_BF16:
+        others = {}
+        for oname in ("baby_gpt", "gpt2_124m", "gpt2_1p5b", "long_context"):
+            if oname != w.name:
+                others[oname] = time_other_workload(ga, oname, dev, s, flush, K)
+
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -707,6 +779,7 @@ def run_ours(args, w, rank, world, local_rank):
         "window": banded,
         "deterministic": det,
         "dropout": drop,
+        "other_workloads": others,
         "clocks": clocks,
         "wall_s_timed": wall1 - wall0,
     }

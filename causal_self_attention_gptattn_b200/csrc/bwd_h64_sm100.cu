@@ -370,8 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) {
                     tc_fence_after();
                     uint32_t sr[64];
-                    tmem_ld_x32(trow + kColS + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                    tmem_ld_x32(trow + kColS + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                    tmem_ld_x32_nowait(trow + kColS + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld_x32_nowait(trow + kColS + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                    tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                     tc_fence_before();
                     mbar_arrive(bar(kBarSEmpty));
                     const float4 *lse4 = reinterpret_cast<const float4 *>(sLse + st * 128 + 64 * half);

@@ -318,10 +318,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) continue;
                 tc_fence_after();
                 uint32_t sr[128];
-                tmem_ld_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld_x32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-                tmem_ld_x32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                // four loads in flight, one wait (the waits name every destination register)
+                tmem_ld_x32_nowait(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld_x32_nowait(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld_x32_nowait(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                tmem_ld_x32_nowait(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
                 tc_fence_before();
                 mbar_arrive(bar(kBarSEmpty + t));  // S buffer may take the next tile
                 if (j == qt) {
@@ -335,17 +340,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < 128; ++c)
                         if (c <= cut) sr[c] = __float_as_uint(-INFINITY);
                 }
-                float mp[4];
+                // row max: eight independent chains of 16 columns, then a short tree
+                float mp[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) mp[q] = __uint_as_float(sr[32 * q]);
+                for (int q = 0; q < 8; ++q) mp[q] = __uint_as_float(sr[16 * q]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
+                for (int c = 1; c < 15; c += 2)
 #pragma unroll
-                    for (int c = 1; c < 31; c += 2)
-                        mp[q] = fmax3(mp[q], __uint_as_float(sr[32 * q + c]), __uint_as_float(sr[32 * q + c + 1]));
-                const float mx = fmax3(fmax3(mp[0], mp[1], __uint_as_float(sr[31])),
-                                       fmax3(mp[2], mp[3], __uint_as_float(sr[63])),
-                                       fmax3(__uint_as_float(sr[95]), __uint_as_float(sr[127]), -INFINITY));
+                    for (int q = 0; q < 8; ++q)
+                        mp[q] = fmax3(mp[q], __uint_as_float(sr[16 * q + c]), __uint_as_float(sr[16 * q + c + 1]));
+#pragma unroll
+                for (int q = 0; q < 8; ++q) mp[q] = fmaxf(mp[q], __uint_as_float(sr[16 * q + 15]));
+                const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
                 const float m_cand = mx * scale_log2;
                 const bool grow = m_cand > mrow + 8.f;
                 const float m_new = grow ? m_cand : mrow;
