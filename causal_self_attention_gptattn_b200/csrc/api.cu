@@ -284,8 +284,7 @@ cudaError_t launch_selftest_timeout(DevCtx ctx, cudaStream_t s) {
 using namespace gptattn;
 
 namespace {
-// Shape checks shared by the windowed entry points: window >= 1; a window
-// narrower than T needs the head-size-64 kernels on the bf16 path.  Returns the
+// Shape checks shared by the windowed entry points: window >= 1.  Returns the
 // window the kernels get (kCausalWindow when nothing is cut).
 gptattn_status check_window(int window, int T, int hs, gptattn_dtype dt, int *kernel_window) {
     if (window < 1) return GPTATTN_ERR_INVALID_ARG;
@@ -293,7 +292,6 @@ gptattn_status check_window(int window, int T, int hs, gptattn_dtype dt, int *ke
         *kernel_window = kCausalWindow;
         return GPTATTN_OK;
     }
-    if (dt == GPTATTN_BF16 && hs != 64) return GPTATTN_ERR_UNSUPPORTED;
     *kernel_window = window;
     return GPTATTN_OK;
 }
@@ -346,11 +344,11 @@ gptattn_status fwd_impl(const void *qkv, void *y, float *lse, int B, int T, int 
 }  // namespace
 
 namespace {
-// Deterministic mode on the bf16 path needs the head-size-64 kernels and row
-// indices of the partial-tile buffer that fit 32-bit TMA coordinates.
+// Deterministic mode on the bf16 path needs row indices of the partial-tile
+// buffer that fit 32-bit TMA coordinates.
 gptattn_status check_det(int B, int T, int n_head, int hs, gptattn_dtype dt) {
     if (dt != GPTATTN_BF16) return GPTATTN_OK;
-    if (hs != 64) return GPTATTN_ERR_UNSUPPORTED;
+    (void)hs;
     if ((long long)B * n_head * det_slots(T) * kTile > 0x7fffffffLL) return GPTATTN_ERR_UNSUPPORTED;
     return GPTATTN_OK;
 }

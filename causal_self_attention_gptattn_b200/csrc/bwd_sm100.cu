@@ -11,13 +11,18 @@
 //
 // Three kernels:
 //   pre   D and lse*log2(e) per query row into the workspace; zero dQ accumulator
-//   main  one CTA per (key tile j, b, h); loops over query tiles i >= j:
+//   main  one CTA per (key tile j, b, h); loops over query tiles i >= j (for a
+//         local window only those its band reaches; the band's far edge is
+//         masked element-wise like the diagonal):
 //           S^T = K Q_i^T, dP^T = V dO_i^T          (tcgen05, TMEM)
 //           P^T (bf16) back into TMEM; dS^T (bf16) into shared memory
 //           dV += P^T dO_i (P from TMEM), dK += dS^T Q_i   (TMEM accumulators)
 //           dQ_i = dS K -> TMEM -> smem -> TMA reduce-add into the fp32 accumulator
 //         epilogue: dK * scale and dV -> bf16 -> TMA store into dqkv
 //   post  dQ accumulator * scale -> bf16 into dqkv[..., 0:C]
+// Deterministic mode (n_slots > 0): each (query tile, key tile) partial of dQ is
+// stored in a slot of its own and the postprocess sums a query tile's slots in
+// a fixed order, so the result does not depend on the order CTAs finish in.
 //
 // Main-kernel roles (10 warps):
 //   warp 0      TMA producer (K, V once; Q_i, dO_i, lse_i, D_i per iteration)
@@ -86,13 +91,16 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
     }
 }
 
-template <int HS>
+// kBand: a local window narrower than T (shorter query range, far-edge mask); the
+// causal instantiation compiles none of it.
+template <int HS, bool kBand>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
                     const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
                     const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C, int n_head,
-                    int T_pad, int n_t, int *status, unsigned long long budget_ns) {
+                    int T_pad, int n_t, int window, int n_slots, int *status, unsigned long long budget_ns) {
     using K = BwdCfg<HS>;
+    if constexpr (!kBand) window = 1 << 30;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -105,7 +113,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kt = blockIdx.x / BH;   // key tile; small kt = most query tiles = scheduled first
     const int b = bh / n_head;
     const int h = bh % n_head;
-    const int niter = n_t - kt;       // query tiles kt..n_t-1
+    // query tiles kt..: up to the last one the key tile's band reaches (all of them when causal)
+    const long long last_t = (long long)kt * kTile + kTile - 2 + window;  // largest key + window - 1
+    const int niter = (last_t / kTile < n_t ? (int)(last_t / kTile) : n_t - 1) - kt + 1;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K::kOffBar);
     auto bar = [&](int idx) -> uint32_t { return smem_u32(&bars[idx]); };
@@ -285,6 +295,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (c < row) p0 = 0.f;
                         if (c + 1 < row) p1 = 0.f;
                     }
+                    if (kBand && it * kTile + kTile - 1 >= window) {  // band's far edge: t - s < window
+                        const int cut = window + row - it * kTile;  // query columns >= cut are masked
+                        if (c >= cut) p0 = 0.f;
+                        if (c + 1 >= cut) p1 = 0.f;
+                    }
                     pk[c >> 1] = pack_bf16x2(p0, p1);
                 }
                 // columns [16ch, 16ch+16) were read in an earlier (or this) chunk
@@ -403,9 +418,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 named_bar_sync(2, 128);
                 if (leader && ok && !*abort_flag) {
-                    const int r0 = bh * T_pad + qt * kTile;
-                    tma_reduce_add_2d(&map_dq, sdQ, half * 64, r0);
-                    tma_reduce_add_2d(&map_dq, sdQ + kSlabBytes, half * 64 + 32, r0);
+                    if (n_slots == 0) {  // add into the (b, h, query tile) rows of the accumulator
+                        const int r0 = bh * T_pad + qt * kTile;
+                        tma_reduce_add_2d(&map_dq, sdQ, half * 64, r0);
+                        tma_reduce_add_2d(&map_dq, sdQ + kSlabBytes, half * 64 + 32, r0);
+                    } else {  // deterministic: a slot of its own per (query tile, key tile)
+                        const int r0 = (bh * n_slots + qt * (qt + 1) / 2 + kt) * kTile;
+                        tma_store_2d(&map_dq, sdQ, half * 64, r0);
+                        tma_store_2d(&map_dq, sdQ + kSlabBytes, half * 64 + 32, r0);
+                    }
                     bulk_commit_group();
                 }
             }
@@ -546,15 +567,15 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_det_kernel(const float *_
 template <int HS>
 cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
                              const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                             int n_head, int T_pad, DevCtx ctx, cudaStream_t s) {
+                             int n_head, int T_pad, int window, int n_slots, DevCtx ctx, cudaStream_t s) {
     using K = BwdCfg<HS>;
-    cudaError_t e = cudaFuncSetAttribute(bwd_bf16_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)K::kSmemBytes);
+    auto kern = window < T ? bwd_bf16_kernel<HS, true> : bwd_bf16_kernel<HS, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int n_t = ceil_div(T, kTile);
     const long long blocks = (long long)n_t * B * n_head;
-    return launch_pdl(bwd_bf16_kernel<HS>, dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_dy,
-                      map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, ctx.status, ctx.budget_ns);
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_dy, map_dqkv, map_dq,
+                      lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace
@@ -582,8 +603,9 @@ cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUten
     if (hs == 64)
         return launch_bwd_main_h64(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots,
                                    dp, ctx, s);
-    if (hs == 128 && window >= T && n_slots == 0 && dp.threshold == 0u)
-        return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, ctx, s);
+    if (hs == 128 && dp.threshold == 0u)
+        return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots,
+                                     ctx, s);
     return cudaErrorInvalidValue;
 }
 
@@ -601,6 +623,9 @@ cudaError_t launch_bwd_post_det_bf16(int hs, const float *part, void *dqkv, int 
     auto out = static_cast<__nv_bfloat16 *>(dqkv);
     if (hs == 64)
         return launch_pdl(bwd_post_det_kernel<64>, grid, dim3(kPPThreads), 0, s, part, out, T, C, n_head, n_slots, window);
+    if (hs == 128)
+        return launch_pdl(bwd_post_det_kernel<128>, grid, dim3(kPPThreads), 0, s, part, out, T, C, n_head, n_slots,
+                          window);
     return cudaErrorInvalidValue;
 }
 

@@ -9,6 +9,10 @@
 //     O  += P_j V_j                   (tcgen05 MMA, P read straight from TMEM)
 // over the key tiles j at or below the diagonal (tiles above it are skipped,
 // the diagonal tile is masked element-wise), then y = O / l and lse = m + ln l.
+// Local window (minGPT README page, reference notes on GPT-3: locally banded
+// attention): query t sees keys t-window < s <= t; key tiles below a query
+// tile's band are skipped and the band's lower edge is masked element-wise like
+// the diagonal.  window >= T is the causal case.
 //
 // Work item = a pair of consecutive query tiles (A = 2m, B = 2m+1) of one
 // (b, h); both share the K_j / V_j tiles.  One persistent CTA per SM walks
@@ -86,12 +90,21 @@ __device__ __forceinline__ int item_index(int k, int cta, int grid) {
     return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
 }
 
-template <int HS>
+// First key tile that query tile qt's band reaches.
+__device__ __forceinline__ int band_lo_tile(int qt, int window) {
+    const int s = qt * kTile - window + 1;
+    return s > 0 ? s / kTile : 0;
+}
+
+// kBand: a local window narrower than T (key-tile ranges and edge masks); the causal
+// instantiation compiles none of it.
+template <int HS, bool kBand>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
-                    float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int *status,
+                    float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, int *status,
                     unsigned long long budget_ns) {
     using K = FwdCfg<HS>;
+    if constexpr (!kBand) window = 1 << 30;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -165,7 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode(w, m, bh);
                 const int b = bh / n_head, h = bh % n_head;
                 const bool hasB = 2 * m + 1 < n_qt;
-                const int nkv = hasB ? 2 * m + 2 : 2 * m + 1;
+                const int jlo = kBand ? band_lo_tile(2 * m, window) : 0;
+                const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
                 const int qs = nq % K::kQStages;
                 if (nq >= K::kQStages &&
                     !(ok = mbar_wait(bar(K::kBarQEmpty + qs), (uint32_t)((nq / K::kQStages) & 1) ^ 1u, g)))
@@ -183,11 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_expect_tx(bar(K::kBarKFull + st), K::kTileBytes);
                     for (int s = 0; s < K::kSlabs; ++s)
                         tma_load_3d(sK(st) + s * kSlabBytes, &map_qkv, bar(K::kBarKFull + st), C + h * HS + 64 * s,
-                                    j * kTile, b);
+                                    (jlo + j) * kTile, b);
                     mbar_arrive_expect_tx(bar(K::kBarVFull + st), K::kTileBytes);
                     for (int s = 0; s < K::kSlabs; ++s)
                         tma_load_3d(sV(st) + s * kSlabBytes, &map_qkv, bar(K::kBarVFull + st), 2 * C + h * HS + 64 * s,
-                                    j * kTile, b);
+                                    (jlo + j) * kTile, b);
                     ++gkv;
                 }
             }
@@ -239,31 +253,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int m, bh;
                 decode(w, m, bh);
                 const bool hasB = 2 * m + 1 < n_qt;
-                const int nt[2] = {2 * m + 1, hasB ? 2 * m + 2 : 0};  // key tiles per tile stream
-                const int nkv = hasB ? nt[1] : nt[0];
+                // key tiles of each stream: [lo, hi] (a band narrower than T starts later); the
+                // item walks their union [jlo, jlo + nkv)
+                const int lo[2] = {kBand ? band_lo_tile(2 * m, window) : 0,
+                                   hasB ? (kBand ? band_lo_tile(2 * m + 1, window) : 0) : 1};
+                const int hi[2] = {2 * m, hasB ? 2 * m + 1 : 0};
+                const int jlo = lo[0];
+                const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
+                auto part = [&](int t, int jj) { return jj >= lo[t] && jj <= hi[t]; };
                 const int qs = n % K::kQStages;
                 if (!(ok = mbar_wait(bar(K::kBarQFull + qs), (uint32_t)(n / K::kQStages) & 1u, g))) break;
                 if (!(ok = mbar_wait(bar(K::kBarKFull + gkv % K::kKVStages), (uint32_t)(gkv / K::kKVStages) & 1u, g)))
                     break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t)
-                    if (nt[t] > 0) issue_S(qs, t, gkv % K::kKVStages);
+                    if (part(t, jlo)) issue_S(qs, t, gkv % K::kKVStages);
                 any = true;
                 for (int j = 0; j < nkv && ok; ++j) {
+                    const int jj = jlo + j;  // key tile
                     const int st = (gkv + j) % K::kKVStages;
+                    const uint32_t ph = (uint32_t)((gkv + j) / K::kKVStages) & 1u;
                     const int st1 = (gkv + j + 1) % K::kKVStages;
                     const uint32_t ph1 = (uint32_t)((gkv + j + 1) / K::kKVStages) & 1u;
-                    if (!(ok = mbar_wait(bar(K::kBarVFull + st), (uint32_t)((gkv + j) / K::kKVStages) & 1u, g))) break;
+                    if (!(ok = mbar_wait(bar(K::kBarVFull + st), ph, g))) break;
                     for (int t = 0; t < 2 && ok; ++t) {
-                        if (j >= nt[t]) continue;
+                        if (!part(t, jj)) continue;
+                        if (jj == lo[t] && jj > jlo) {  // this stream's band starts after the item's
+                            if (!(ok = mbar_wait(bar(K::kBarKFull + st), ph, g))) break;
+                            tc_fence_after();
+                            issue_S(qs, t, st);
+                        }
                         if (!(ok = mbar_wait(bar(K::kBarPFull + t), (uint32_t)it[t] & 1u, g))) break;
-                        if (j == 0 && items[t] > 0 &&
+                        if (jj == lo[t] && items[t] > 0 &&
                             !(ok = mbar_wait(bar(K::kBarOFree + t), (uint32_t)(items[t] - 1) & 1u, g)))
                             break;
                         tc_fence_after();
-                        issue_PV(t, st, j == 0);
+                        issue_PV(t, st, jj == lo[t]);
                         ++it[t];
-                        if (j + 1 < nt[t]) {
+                        if (jj + 1 <= hi[t]) {
                             if (!(ok = mbar_wait(bar(K::kBarKFull + st1), ph1, g))) break;
                             tc_fence_after();
                             issue_S(qs, t, st1);
@@ -307,15 +334,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (leader) mbar_arrive(bar(K::kBarQEmpty + qs));
                 continue;
             }
-            const int ntile = qt + 1;
+            const int jlo_t = kBand ? band_lo_tile(qt, window) : 0;
+            // key tiles at or below j_edge need the band's lower edge masked (a band narrower
+            // than T: query t sees keys t-window < s <= t)
+            const bool banded = kBand && qt * kTile + kTile - 1 - window >= 0;
+            const int j_edge = banded ? (qt * kTile + kTile - 1 - window) / kTile : -1;
             float mrow = -INFINITY;  // reference max of scaled scores (log2 units), lazily updated
             float l = 0.f;           // running normaliser of the fp32 weights
             float l_r = 0.f;         // running normaliser of the bf16-rounded weights
-            for (int j = 0; j < ntile; ++j, ++it) {
+            for (int j = jlo_t; j <= qt; ++j, ++it) {
                 if (ok) ok = warp_wait(bar(K::kBarSFull + t), (uint32_t)it & 1u, g);
                 if (!ok) continue;
                 tc_fence_after();
                 const bool diag = (j == qt);
+                const bool edge = j <= j_edge;
+                const int cut = (qt - j) * kTile + row - window;  // on an edge tile, columns <= cut are masked
                 // pass 1: row maximum
                 float mx = -INFINITY;
 #pragma unroll
@@ -327,6 +360,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int c = 0; c < 32; ++c)
                             if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
                     }
+                    if (kBand && edge) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (32 * ch + c <= cut) sr[c] = __float_as_uint(-INFINITY);
+                    }
                     float a = __uint_as_float(sr[0]), bb = __uint_as_float(sr[1]);
 #pragma unroll
                     for (int c = 2; c < 32; c += 2) a = fmax3(a, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
@@ -337,7 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool grow = m_cand > mrow + 8.f;
                 const float m_new = grow ? m_cand : mrow;
                 const float alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
-                const uint64_t negm2 = f32x2_pack(-m_new, -m_new);
+                // a row with no visible key yet (band edge) keeps weight 0, not NaN
+                const float m_use = (kBand && m_new == -INFINITY) ? 0.f : m_new;
+                const uint64_t negm2 = f32x2_pack(-m_use, -m_use);
                 // pass 2: weights, sums, P back into TMEM (bf16 pairs over columns already read)
                 uint64_t sum2 = f32x2_pack(0.f, 0.f), sumr2 = f32x2_pack(0.f, 0.f);
 #pragma unroll
@@ -348,6 +388,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
                             if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
+                    }
+                    if (kBand && edge) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (32 * ch + c <= cut) sr[c] = __float_as_uint(-INFINITY);
                     }
                     uint32_t pk[16];
 #pragma unroll
@@ -369,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 l = l * alpha + (s0 + s1);
                 l_r = l_r * alpha + (r0 + r1);
                 mrow = m_new;
-                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (j > jlo_t && __any_sync(0xffffffffu, alpha != 1.f)) {
                     // rescale O once the previous P V product of this tile has landed
                     ok = warp_wait(bar(K::kBarODone + t), (uint32_t)(it - 1) & 1u, g);
                     if (ok) {
@@ -443,10 +488,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int HS>
 cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
-                            int n_head, DevCtx ctx, cudaStream_t s) {
+                            int n_head, int window, DevCtx ctx, cudaStream_t s) {
     using K = FwdCfg<HS>;
-    cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<HS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)K::kSmemBytes);
+    auto kern = window < T ? fwd_bf16_kernel<HS, true> : fwd_bf16_kernel<HS, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
@@ -455,8 +500,8 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
     const int n_qt = ceil_div(T, kTile);
     const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    return launch_pdl(fwd_bf16_kernel<HS>, dim3((unsigned)grid), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_y, lse, B,
-                      T, C, n_head, n_qt, ctx.status, ctx.budget_ns);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_y, lse, B, T, C, n_head,
+                      n_qt, window, ctx.status, ctx.budget_ns);
 }
 
 }  // namespace
@@ -464,8 +509,7 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T,
                             int C, int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
     if (hs == 64) return launch_fwd_h64(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s);
-    if (hs == 128 && window >= T && dp.threshold == 0u)
-        return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, ctx, s);
+    if (hs == 128 && dp.threshold == 0u) return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, window, ctx, s);
     return cudaErrorInvalidValue;
 }
 

@@ -93,8 +93,7 @@ GPTATTN_API gptattn_status gptattn_fwd(const void *qkv, void *y, float *lse,
  * GPT-3 describe alternating with dense layers.  window >= 1; window >= T is
  * exactly the causal operation (the same kernels and results as gptattn_fwd /
  * gptattn_bwd).  Key tiles outside every query tile's band are skipped.
- * Supported: every fp32 head size; bf16 head size 64 for any window, bf16 head
- * size 128 only for window >= T (GPTATTN_ERR_UNSUPPORTED otherwise).
+ * Supported: every head size of gptattn_fwd, any window.
  * window < 1 -> GPTATTN_ERR_INVALID_ARG.  Other arguments, layouts, the
  * workspace (gptattn_bwd_workspace_bytes) and errors as in gptattn_fwd /
  * gptattn_bwd; the backward takes the y and lse of the windowed forward. */
@@ -113,7 +112,7 @@ GPTATTN_API gptattn_status gptattn_bwd_window(const void *qkv, const void *y, co
  * bit between runs.  This variant stores every (query tile, key tile) partial
  * of dQ in a workspace slot of its own and sums a query tile's partials in a
  * fixed order, so equal inputs give bit-identical dqkv on every run.  Same
- * arguments, semantics, support (bf16: head size 64 only, any window) and
+ * arguments, semantics, support (every head size, any window) and
  * errors as gptattn_bwd_window, with a larger workspace:
  * gptattn_bwd_det_workspace_bytes() (for bf16 it adds B * n_head *
  * ceil(T/128)(ceil(T/128)+1)/2 tiles of 128 x 64 fp32; (size_t)-1 for an

@@ -53,6 +53,17 @@ def test_det_bf16_parity(B, T, n_head, window):
     compare((y, lse, g), (ry, rl, rg), torch.bfloat16, f"det T={T} window {window}")
 
 
+@pytest.mark.parametrize("B,T,n_head,window", [(1, 300, 2, 10**9), (2, 520, 1, 200), (1, 129, 2, 10**9)])
+def test_det_bf16_head128_parity_and_repeatable(B, T, n_head, window):
+    qkv, dy = make_inputs(B, T, n_head, 128, dtype=torch.bfloat16, seed=1150 + T)
+    y, lse, gs, raws = run_det(qkv, dy, n_head, window, reps=2)
+    assert torch.equal(raws[1].view(torch.int16), raws[0].view(torch.int16)), "deterministic backward differs"
+    w = None if window >= T else window
+    ry, rl = oracle.forward(qkv, n_head, window=w)
+    rg = oracle.backward(qkv, dy, n_head, window=w)
+    compare((y, lse, gs[0]), (ry, rl, rg), torch.bfloat16, f"det hs128 T={T} window {window}")
+
+
 def test_det_bf16_bitwise_repeatable_at_full_size():
     """GPT-2 124M shape: three runs give bit-identical dqkv; they agree with the
     reduce-add backward within tolerance; sampled heads agree with the oracle."""

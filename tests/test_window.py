@@ -36,6 +36,35 @@ def test_window_bf16(B, T, n_head, window):
     compare(got, oracle_window(qkv, dy, n_head, window), torch.bfloat16, f"bf16 T={T} window {window}")
 
 
+# head size 128 (the long-context shape): bands inside a tile, across tiles, ragged T
+BF16_H128 = [(1, 300, 2, 1), (2, 520, 1, 100), (1, 384, 2, 128), (1, 777, 1, 300), (2, 200, 2, 255)]
+
+
+@pytest.mark.parametrize("B,T,n_head,window", BF16_H128)
+def test_window_bf16_head128(B, T, n_head, window):
+    qkv, dy = make_inputs(B, T, n_head, 128, dtype=torch.bfloat16, seed=960 + T + window)
+    got = run_fwd_bwd(qkv, dy, n_head, window=window)
+    compare(got, oracle_window(qkv, dy, n_head, window), torch.bfloat16, f"bf16 hs128 T={T} window {window}")
+
+
+def test_window_bf16_head128_long_context_sampled_heads():
+    """The GPT-3-style long-context shape (B=4, T=2048, 16 heads of 128) with a 512-token band, the
+    sparse layer of the alternating pattern; sampled heads against the oracle.  Inputs are N(0,1):
+    with the workload's doubled qkv (sharp softmax) the band leaves so few keys per row that the
+    bf16 rounding of the weights and of y alone gives y errors of 2.5-2.9e-2, above the 2e-2 the
+    causal configurations are held to (a CPU emulation of that arithmetic shows the same)."""
+    w = WORKLOADS[5]
+    qkv, dy = make_inputs(w.B, w.T, w.n_head, w.hs, dtype=torch.bfloat16, seed=1005)
+    y, lse, dqkv = run_fwd_bwd(qkv, dy, w.n_head, window=512)
+    batches, heads = [0, w.B - 1], [0, 15]
+    q_s = select_heads(qkv[batches].double().numpy(), w.n_head, 3, heads)
+    g_s = select_heads(dy[batches].double().numpy(), w.n_head, 1, heads)
+    ref = oracle_window(q_s, g_s, len(heads), 512)
+    got = (select_heads(y[batches], w.n_head, 1, heads), lse[batches][:, heads],
+           select_heads(dqkv[batches], w.n_head, 3, heads))
+    compare(got, ref, torch.bfloat16, "long_context window 512")
+
+
 def test_window_at_least_T_is_the_causal_path():
     """window >= T takes exactly the causal kernels: bit-identical outputs."""
     qkv, dy = make_inputs(2, 333, 2, 64, dtype=torch.bfloat16, seed=950)
