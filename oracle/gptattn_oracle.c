@@ -35,11 +35,13 @@
  *    same arithmetic.
  *  - "Let's build GPT" lecture page, chapter "scaling up the model! creating a
  *    few variables. adding dropout": dropout on the attention weights.  Read
- *    as inverted dropout after the softmax: weight P[t][s] is kept with
- *    probability 1-p and then scaled by 1/(1-p), else zeroed; lse stays the
+ *    as inverted dropout after the softmax: weight P[t][s] is dropped with
+ *    probability p and a kept weight is scaled by 1/(1-p); lse stays the
  *    logsumexp of the undropped scores.  The keep decision is a counter-based
  *    random number (Philox4x32-10, below), so the forward and the backward
- *    see the same mask without storing it.
+ *    see the same mask without storing it.  p is applied in steps of 1/256:
+ *    the drop probability is theta/256 with theta = round(256 p) (at most
+ *    255), and kept weights are scaled by 1/(1 - theta/256).
  *
  * Input packing (the projection output of a GPT-2 style block): qkv[B][T][3C]
  * row-major, q = columns [0,C), k = [C,2C), v = [2C,3C).  Output y[B][T][C]
@@ -101,20 +103,22 @@ void oracle_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], ui
     out[3] = c3;
 }
 
-/* Keep decision for attention weight (t, s) of batch-head pair bh: counter
- * (s / 4, t, bh, 0), key = the 64-bit seed, word s % 4; kept iff that word is
- * >= threshold, threshold = floor(p * 2^32). */
-static int dropout_keep(uint64_t seed, uint32_t threshold, int bh, int t, int s) {
-    const uint32_t ctr[4] = {(uint32_t)s >> 2, (uint32_t)t, (uint32_t)bh, 0u};
+/* Keep decision for attention weight (t, s) of batch-head pair bh.  One Philox
+ * call covers a 4 x 4 block of (query, key) pairs: counter (s / 4, t / 4, bh, 0),
+ * key = the 64-bit seed; the pair's 8 bits are byte s % 4 (least significant
+ * first) of output word t % 4.  Kept iff that byte is >= theta. */
+static int dropout_keep(uint64_t seed, uint32_t theta, int bh, int t, int s) {
+    const uint32_t ctr[4] = {(uint32_t)s >> 2, (uint32_t)t >> 2, (uint32_t)bh, 0u};
     const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
     uint32_t r[4];
     oracle_philox4x32_10(ctr, key, r);
-    return r[s & 3] >= threshold;
+    return ((r[t & 3] >> (8 * (s & 3))) & 0xFFu) >= theta;
 }
 
+/* theta = round(256 p), at most 255: the drop probability is theta / 256. */
 static uint32_t dropout_threshold(double p) {
-    const double x = floor(p * 4294967296.0);
-    return x >= 4294967295.0 ? 4294967295u : (uint32_t)x;
+    const double x = floor(256.0 * p + 0.5);
+    return x >= 255.0 ? 255u : (uint32_t)x;
 }
 
 #define ORACLE_OK 0
@@ -141,10 +145,12 @@ typedef struct {
     uint64_t seed;
 } Dropout;
 
-/* Factor applied to weight (t, s): 1/(1-p) if kept, 0 if dropped; exactly 1 without dropout. */
+/* Factor applied to weight (t, s): 1/(1 - theta/256) if kept, 0 if dropped; exactly 1
+ * without dropout. */
 static inline double drop_factor(const Dropout *dr, int bh, int t, int s) {
     if (dr->p <= 0.0) return 1.0;
-    return dropout_keep(dr->seed, dropout_threshold(dr->p), bh, t, s) ? 1.0 / (1.0 - dr->p) : 0.0;
+    const uint32_t theta = dropout_threshold(dr->p);
+    return dropout_keep(dr->seed, theta, bh, t, s) ? 1.0 / (1.0 - theta / 256.0) : 0.0;
 }
 
 /* First key position visible to query t, and last query position that sees key s. */

@@ -14,9 +14,11 @@ GPT-3 (alternating dense and locally banded sparse attention), read as: token
 t sees positions t-window < s <= t.  The dropout pins (``pin_dropout_*``) follow
 the lecture's chapter "scaling up the model! creating a few variables. adding
 dropout", read as inverted dropout on the attention weights with a Philox4x32-10
-keep mask (counter (s/4, t, b*n_head+h, 0), key = seed, word s%4, kept iff the
-word >= floor(p * 2^32)); the generator's own bits are pinned by the published
-known-answer vectors of Philox4x32-10 (``tests/golden/philox4x32_10_kat.json``).
+keep mask (one call per 4 x 4 block of (query t, key s) pairs: counter (s/4, t/4,
+b*n_head+h, 0), key = seed, byte s%4 of word t%4, kept iff that byte >= theta =
+round(256 p); kept weights scaled by 1/(1 - theta/256)); the generator's own bits
+are pinned by the published known-answer vectors of Philox4x32-10
+(``tests/golden/philox4x32_10_kat.json``).
 """
 from __future__ import annotations
 
@@ -456,15 +458,23 @@ def _mask_probe(orc, p, seed, T=64, n_head=2):
     return f
 
 
+def _theta(p):
+    """The 8-bit drop threshold: round(256 p), at most 255."""
+    return min(255, math.floor(256 * p + 0.5))
+
+
 def pin_dropout_mask_and_scale(orc):
-    """Inverted dropout: every visible weight is either 0 or scaled by exactly
-    1/(1-p); none above the diagonal; the keep rate is 1-p (binomial, 5 sigma);
-    the two heads get different masks."""
+    """Inverted dropout with p applied in steps of 1/256: every visible weight is
+    either 0 or scaled by exactly 1/(1 - theta/256), theta = round(256 p) (77 for
+    p = 0.3); none above the diagonal; the keep rate is 1 - theta/256 (binomial, 5
+    sigma); the two heads get different masks."""
     p = 0.3
     f = _mask_probe(orc, p, seed=11)
     T = f.shape[1]
     tril = np.tril(np.ones((T, T), dtype=bool))
     vals = f[:, tril]
+    assert _theta(p) == 77
+    p = _theta(p) / 256.0
     kept = np.abs(vals - 1.0 / (1.0 - p)) < 1e-12
     dropped = np.abs(vals) < 1e-15
     assert np.all(kept | dropped)
@@ -476,17 +486,18 @@ def pin_dropout_mask_and_scale(orc):
 
 
 def pin_dropout_counter_layout(orc):
-    """Weight (t, s) of batch-head pair bh is kept iff word s%4 of Philox4x32-10 at
-    counter (s/4, t, bh, 0) under key (seed low, seed high) is >= floor(p * 2^32):
-    the mapping the CUDA path must follow too."""
+    """Weight (t, s) of batch-head pair bh is kept iff byte s%4 (least significant
+    first) of word t%4 of Philox4x32-10 at counter (s/4, t/4, bh, 0) under key (seed
+    low, seed high) is >= round(256 p): the mapping the CUDA path must follow too."""
     p, seed = 0.45, (7 << 32) | 12345
     f = _mask_probe(orc, p, seed=seed, T=48, n_head=2)
-    thr = math.floor(p * 2.0 ** 32)
+    thr = _theta(p)
+    assert thr == 115
     for h in range(2):
         for t in range(48):
             for s_ in range(t + 1):
-                r = orc.philox([s_ // 4, t, h, 0], [seed & 0xFFFFFFFF, seed >> 32])
-                assert (r[s_ % 4] >= thr) == (f[h, t, s_] > 0), (h, t, s_)
+                r = orc.philox([s_ // 4, t // 4, h, 0], [seed & 0xFFFFFFFF, seed >> 32])
+                assert (((r[t % 4] >> (8 * (s_ % 4))) & 0xFF) >= thr) == (f[h, t, s_] > 0), (h, t, s_)
 
 
 def pin_dropout_lse_unchanged_and_unbiased(orc):

@@ -33,7 +33,10 @@ MUTANTS = [
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 1, h, d);",
      "acc += dS[(size_t)t * (size_t)T + s] * qkv_at(qkv, T, C, hs, b, s, 0, h, d);"),
     ("dK_missing_scale", "dk[(size_t)s * ld_dqkv + d] = acc * scale;", "dk[(size_t)s * ld_dqkv + d] = acc;"),
-    ("dropout_scale_missing", "? 1.0 / (1.0 - dr->p) : 0.0;", "? 1.0 : 0.0;"),
+    ("dropout_scale_missing", "? 1.0 / (1.0 - theta / 256.0) : 0.0;", "? 1.0 : 0.0;"),
+    ("dropout_scale_unquantised", "? 1.0 / (1.0 - theta / 256.0) : 0.0;", "? 1.0 / (1.0 - dr->p) : 0.0;"),
+    ("dropout_block_transposed", "return ((r[t & 3] >> (8 * (s & 3))) & 0xFFu) >= theta;",
+     "return ((r[s & 3] >> (8 * (t & 3))) & 0xFFu) >= theta;"),
     ("dropout_mask_ignored_in_dP", "acc *= drop_factor(&dr, b * n_head + h, t, s);", "acc *= 1.0 / (1.0 - dr.p);"),
     ("band_one_key_too_many", "return t - window + 1 > 0 ? t - window + 1 : 0;", "return t - window > 0 ? t - window : 0;"),
     ("band_last_query_dropped", "return s + window - 1 < T - 1 ? s + window - 1 : T - 1;",
