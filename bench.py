@@ -611,9 +611,19 @@ def run_ours(args, w, rank, world, local_rank):
             b_.record(s)
         torch.cuda.synchronize()
         to = sum(a.elapsed_time(b_) for a, b_ in evs)
+        ga.gptattn_profile_enable(4 * Ko + 64)
+        for _ in range(Ko):
+            flush.zero_()
+            step_drop()
+        torch.cuda.synchronize()
+        per_d = {}
+        for kname, kms in ga.gptattn_profile_read(4 * Ko + 64):
+            per_d.setdefault(kname, []).append(kms)
+        ga.gptattn_profile_enable(0)
         ga.check(ga.gptattn_get_device_status(s), "device status after the dropout steps")
         drop = {"dropout_p": 0.1, "steps": Ko, "ms_per_step": to / Ko, "value": flops * Ko / (to / 1e3) / 1e12,
-                "unit": "TFLOP/s", "flop_count": "as the plain step"}
+                "unit": "TFLOP/s", "flop_count": "as the plain step",
+                "kernels_ms": {k: statistics.mean(v) for k, v in per_d.items()}}
 
     # ---- decode (gptattn_decode): the last position of every sequence over the same qkv as a
     # key/value cache; HBM-bound, so its roofline is the measured copy bandwidth.  L2 flushed

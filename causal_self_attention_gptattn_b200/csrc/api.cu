@@ -301,10 +301,11 @@ gptattn_status check_window(int window, int T, int hs, gptattn_dtype dt, int *ke
 // the head-size-64 kernels.
 gptattn_status make_dropout(float p, unsigned long long seed, int hs, gptattn_dtype dt, DropoutParams *dp) {
     if (!(p >= 0.f && p < 1.f)) return GPTATTN_ERR_INVALID_ARG;
-    const double x = floor((double)p * 4294967296.0);
+    // p in steps of 1/256: theta = round(256 p), at most 255; drop probability theta/256
+    const double x = floor(256.0 * (double)p + 0.5);
     dp->seed = seed;
-    dp->threshold = x >= 4294967295.0 ? 4294967295u : (uint32_t)x;
-    dp->scale = dp->threshold ? 1.f / (1.f - p) : 1.f;
+    dp->threshold = x >= 255.0 ? 255u : (uint32_t)x;
+    dp->scale = dp->threshold ? (float)(1.0 / (1.0 - dp->threshold / 256.0)) : 1.f;
     if (dp->threshold && dt == GPTATTN_BF16 && hs != 64) return GPTATTN_ERR_UNSUPPORTED;
     return GPTATTN_OK;
 }

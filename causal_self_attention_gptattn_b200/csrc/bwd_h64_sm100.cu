@@ -411,14 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint32_t pk[32];
                     if constexpr (kDropout) {  // keep bits of this row's 64 columns; P^T dropped + rescaled
+                        // generator calls shared by the 4 lanes of this key row's 4 x 4 blocks
                         const uint32_t skey = (uint32_t)(kt * kTile + row);
-                        keepb[0] = keepb[1] = 0u;
-#pragma unroll 4
-                        for (int c = 0; c < 64; ++c) {
-                            const uint32_t tq = (uint32_t)((kt + it) * kTile + 64 * half + c);
-                            const uint32_t bits = dropout_keep4(dp.seed, dp.threshold, (uint32_t)bh, tq, skey & ~3u);
-                            keepb[c >> 5] |= ((bits >> (skey & 3u)) & 1u) << (c & 31);
-                        }
+                        const uint32_t tq0 = (uint32_t)((kt + it) * kTile + 64 * half);
+                        uint32_t kq[4];
+#pragma unroll
+                        for (int m = 0; m < 4; ++m)
+                            kq[m] = dropout_keep16_keys(dp.seed, dp.threshold, (uint32_t)bh, tq0 + 16u * m, skey, lane);
+                        keepb[0] = kq[0] | (kq[1] << 16);
+                        keepb[1] = kq[2] | (kq[3] << 16);
 #pragma unroll
                         for (int c = 0; c < 32; ++c) {
                             const float f0 = ((keepb[(2 * c) >> 5] >> ((2 * c) & 31)) & 1u) ? dp.scale : 0.f;

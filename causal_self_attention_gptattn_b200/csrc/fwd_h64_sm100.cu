@@ -9,8 +9,10 @@
 //                       O_A [384,448)  O_B [448,512)
 // Work item = query tiles A = 2m and B = 2m+1 of one (batch, head), sharing the
 // key/value tiles; one persistent CTA per SM walks the items longest first in
-// a snake order.  Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5
-// softmax of tile A, 6..9 softmax of tile B (one query row per thread).
+// a snake order.  Warpgroup 0: warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer (warps 2, 3 idle); warpgroup 1: softmax of tile A, warpgroup 2:
+// softmax of tile B (one query row per thread).  setmaxnreg moves registers
+// from warpgroup 0 to the softmax warpgroups.
 // Because P has its own buffer, a softmax warpgroup copies S_j to registers
 // in one pass and releases it immediately; the MMA warp then computes S_{j+1}
 // while the warpgroup exponentiates tile j, and P V of tile j runs while the
@@ -35,7 +37,11 @@
 namespace gptattn {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// register budgets per thread (sum = 3 x kLaunchRegs, what the CTA is launched with)
+constexpr int kLaunchRegs = 168;
+constexpr uint32_t kRegsCtl = 88, kRegsSoftmax = 208;
+static_assert(kRegsCtl + 2 * kRegsSoftmax == 3 * kLaunchRegs, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr int HS = 64;
@@ -98,6 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
     const int BH = B * n_head;
     const int n_pairs = (n_qt + 1) >> 1;
     const int n_items = n_pairs * BH;
@@ -149,143 +156,147 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_launch_dependents();
     griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
-    if (warp == 0) {
-        // ================================================================ producer
-        if (lane == 0) {
-            tma_prefetch_map(&map_qkv);
-            tma_prefetch_map(&map_y);
-            bool ok = true;
-            int nq = 0, gkv = 0;
-            for (int k = 0; ok; ++k) {
-                const int w = item_index(k, cta, grid);
-                if (w >= n_items) break;
-                int m, bh;
-                decode(w, m, bh);
-                const int b = bh / n_head, h = bh % n_head;
-                const bool hasB = 2 * m + 1 < n_qt;
-                const int jlo = band_lo_tile(2 * m, window);
-                const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
-                const int qs = nq % kQStages;
-                if (nq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + qs), (uint32_t)((nq / kQStages) & 1) ^ 1u, g)))
-                    break;
-                const uint32_t qb = bar(kBarQFull + qs);
-                mbar_arrive_expect_tx(qb, (hasB ? 2u : 1u) * kTileBytes);
-                for (int t = 0; t < (hasB ? 2 : 1); ++t)
-                    tma_load_3d(sQ(qs, t), &map_qkv, qb, h * HS, (2 * m + t) * kTile, b);
-                ++nq;
-                for (int j = 0; j < nkv; ++j) {
-                    const int st = gkv % kKVStages;
-                    const uint32_t ph = (uint32_t)(gkv / kKVStages) & 1u;
-                    if (gkv >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + st), ph ^ 1u, g))) break;
-                    mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
-                    tma_load_3d(sK(st), &map_qkv, bar(kBarKFull + st), C + h * HS, (jlo + j) * kTile, b);
-                    mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
-                    tma_load_3d(sV(st), &map_qkv, bar(kBarVFull + st), 2 * C + h * HS, (jlo + j) * kTile, b);
-                    ++gkv;
-                }
-            }
-            if (!ok || *abort_flag) {
-                for (int q = (nq > kQStages ? nq - kQStages : 0); q < nq; ++q)
-                    drain_wait(bar(kBarQFull + q % kQStages), (uint32_t)(q / kQStages) & 1u, budget_ns);
-                for (int q = (gkv > kKVStages ? gkv - kKVStages : 0); q < gkv; ++q) {
-                    drain_wait(bar(kBarKFull + q % kKVStages), (uint32_t)(q / kKVStages) & 1u, budget_ns);
-                    drain_wait(bar(kBarVFull + q % kKVStages), (uint32_t)(q / kKVStages) & 1u, budget_ns);
-                }
-            }
-        }
-    } else if (warp == 1) {
-        // ================================================================ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idPV = idesc_bf16_f32(128, HS, false, true);
-            const uint64_t dQ0 = sdesc_sw128(sQ(0, 0), 16, 1024);
-            const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
-            const uint64_t dV0 = sdesc_sw128(sV(0), kSlabBytes, 1024);
-            auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
-            bool ok = true, any = false;
-            int n = 0, gkv = 0;
-            int sc[2] = {0, 0};     // S issued per stream
-            int pc[2] = {0, 0};     // P V issued per stream
-            int items[2] = {0, 0};  // items that used each stream
-            auto issue_S = [&](int qs, int t, int st) {
-                const uint64_t a = at(dQ0, (uint32_t)(2 * qs + t) * kTileBytes);
-                const uint64_t bk = at(dK0, (uint32_t)st * kTileBytes);
-#pragma unroll
-                for (int kk = 0; kk < HS / 16; ++kk)
-                    umma_ss(tmem + kColS + 128u * t, at(a, kk * 32u), at(bk, kk * 32u), idS, kk > 0 ? 1u : 0u);
-                umma_commit(bar(kBarSFull + t));
-                ++sc[t];
-            };
-            auto issue_PV = [&](int t, int st, bool first) {
-                const uint64_t bv = at(dV0, (uint32_t)st * kTileBytes);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + kColO + 64u * t, tmem + kColP + 64u * t + 8u * kk, at(bv, kk * 2048u), idPV,
-                            (!first || kk > 0) ? 1u : 0u);
-                umma_commit(bar(kBarPVDone + t));
-                ++pc[t];
-            };
-            for (int k = 0; ok; ++k, ++n) {
-                const int w = item_index(k, cta, grid);
-                if (w >= n_items) break;
-                int m, bh;
-                decode(w, m, bh);
-                const bool hasB = 2 * m + 1 < n_qt;
-                // key tiles of each stream: [lo, hi]; the item walks their union [jlo, jlo + nkv)
-                const int lo[2] = {band_lo_tile(2 * m, window), hasB ? band_lo_tile(2 * m + 1, window) : 1};
-                const int hi[2] = {2 * m, hasB ? 2 * m + 1 : 0};
-                const int jlo = lo[0];
-                const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
-                auto part = [&](int t, int j) { return j >= lo[t] && j <= hi[t]; };
-                const int qs = n % kQStages;
-                if (!(ok = mbar_wait(bar(kBarQFull + qs), (uint32_t)(n / kQStages) & 1u, g))) break;
-                if (!(ok = mbar_wait(bar(kBarKFull + gkv % kKVStages), (uint32_t)(gkv / kKVStages) & 1u, g))) break;
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (!part(t, jlo)) continue;
-                    if (sc[t] > 0 && !(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
-                    tc_fence_after();
-                    issue_S(qs, t, gkv % kKVStages);
-                    any = true;
-                }
-                for (int j = 0; j < nkv && ok; ++j) {
-                    const int st = (gkv + j) % kKVStages;
-                    // S of the next key tile for each stream, as soon as its S buffer is free
-                    if (j + 1 < nkv) {
-                        const int st1 = (gkv + j + 1) % kKVStages;
-                        if (!(ok = mbar_wait(bar(kBarKFull + st1), (uint32_t)((gkv + j + 1) / kKVStages) & 1u, g))) break;
-                        for (int t = 0; t < 2 && ok; ++t) {
-                            if (!part(t, jlo + j + 1)) continue;
-                            if (!(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
-                            tc_fence_after();
-                            issue_S(qs, t, st1);
-                        }
-                        if (!ok) break;
+    if (wg == 0) {
+        regs_dec<kRegsCtl>();
+        if (warp == 0) {
+            // ================================================================ producer
+            if (lane == 0) {
+                tma_prefetch_map(&map_qkv);
+                tma_prefetch_map(&map_y);
+                bool ok = true;
+                int nq = 0, gkv = 0;
+                for (int k = 0; ok; ++k) {
+                    const int w = item_index(k, cta, grid);
+                    if (w >= n_items) break;
+                    int m, bh;
+                    decode(w, m, bh);
+                    const int b = bh / n_head, h = bh % n_head;
+                    const bool hasB = 2 * m + 1 < n_qt;
+                    const int jlo = band_lo_tile(2 * m, window);
+                    const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
+                    const int qs = nq % kQStages;
+                    if (nq >= kQStages && !(ok = mbar_wait(bar(kBarQEmpty + qs), (uint32_t)((nq / kQStages) & 1) ^ 1u, g)))
+                        break;
+                    const uint32_t qb = bar(kBarQFull + qs);
+                    mbar_arrive_expect_tx(qb, (hasB ? 2u : 1u) * kTileBytes);
+                    for (int t = 0; t < (hasB ? 2 : 1); ++t)
+                        tma_load_3d(sQ(qs, t), &map_qkv, qb, h * HS, (2 * m + t) * kTile, b);
+                    ++nq;
+                    for (int j = 0; j < nkv; ++j) {
+                        const int st = gkv % kKVStages;
+                        const uint32_t ph = (uint32_t)(gkv / kKVStages) & 1u;
+                        if (gkv >= kKVStages && !(ok = mbar_wait(bar(kBarKVEmpty + st), ph ^ 1u, g))) break;
+                        mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
+                        tma_load_3d(sK(st), &map_qkv, bar(kBarKFull + st), C + h * HS, (jlo + j) * kTile, b);
+                        mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
+                        tma_load_3d(sV(st), &map_qkv, bar(kBarVFull + st), 2 * C + h * HS, (jlo + j) * kTile, b);
+                        ++gkv;
                     }
-                    // P V of key tile j for each stream
-                    if (!(ok = mbar_wait(bar(kBarVFull + st), (uint32_t)((gkv + j) / kKVStages) & 1u, g))) break;
+                }
+                if (!ok || *abort_flag) {
+                    for (int q = (nq > kQStages ? nq - kQStages : 0); q < nq; ++q)
+                        drain_wait(bar(kBarQFull + q % kQStages), (uint32_t)(q / kQStages) & 1u, budget_ns);
+                    for (int q = (gkv > kKVStages ? gkv - kKVStages : 0); q < gkv; ++q) {
+                        drain_wait(bar(kBarKFull + q % kKVStages), (uint32_t)(q / kKVStages) & 1u, budget_ns);
+                        drain_wait(bar(kBarVFull + q % kKVStages), (uint32_t)(q / kKVStages) & 1u, budget_ns);
+                    }
+                }
+            }
+        } else if (warp == 1) {
+            // ================================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);
+                constexpr uint32_t idPV = idesc_bf16_f32(128, HS, false, true);
+                const uint64_t dQ0 = sdesc_sw128(sQ(0, 0), 16, 1024);
+                const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
+                const uint64_t dV0 = sdesc_sw128(sV(0), kSlabBytes, 1024);
+                auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+                bool ok = true, any = false;
+                int n = 0, gkv = 0;
+                int sc[2] = {0, 0};     // S issued per stream
+                int pc[2] = {0, 0};     // P V issued per stream
+                int items[2] = {0, 0};  // items that used each stream
+                auto issue_S = [&](int qs, int t, int st) {
+                    const uint64_t a = at(dQ0, (uint32_t)(2 * qs + t) * kTileBytes);
+                    const uint64_t bk = at(dK0, (uint32_t)st * kTileBytes);
+    #pragma unroll
+                    for (int kk = 0; kk < HS / 16; ++kk)
+                        umma_ss(tmem + kColS + 128u * t, at(a, kk * 32u), at(bk, kk * 32u), idS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar(kBarSFull + t));
+                    ++sc[t];
+                };
+                auto issue_PV = [&](int t, int st, bool first) {
+                    const uint64_t bv = at(dV0, (uint32_t)st * kTileBytes);
+    #pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_ts(tmem + kColO + 64u * t, tmem + kColP + 64u * t + 8u * kk, at(bv, kk * 2048u), idPV,
+                                (!first || kk > 0) ? 1u : 0u);
+                    umma_commit(bar(kBarPVDone + t));
+                    ++pc[t];
+                };
+                for (int k = 0; ok; ++k, ++n) {
+                    const int w = item_index(k, cta, grid);
+                    if (w >= n_items) break;
+                    int m, bh;
+                    decode(w, m, bh);
+                    const bool hasB = 2 * m + 1 < n_qt;
+                    // key tiles of each stream: [lo, hi]; the item walks their union [jlo, jlo + nkv)
+                    const int lo[2] = {band_lo_tile(2 * m, window), hasB ? band_lo_tile(2 * m + 1, window) : 1};
+                    const int hi[2] = {2 * m, hasB ? 2 * m + 1 : 0};
+                    const int jlo = lo[0];
+                    const int nkv = (hasB ? 2 * m + 2 : 2 * m + 1) - jlo;
+                    auto part = [&](int t, int j) { return j >= lo[t] && j <= hi[t]; };
+                    const int qs = n % kQStages;
+                    if (!(ok = mbar_wait(bar(kBarQFull + qs), (uint32_t)(n / kQStages) & 1u, g))) break;
+                    if (!(ok = mbar_wait(bar(kBarKFull + gkv % kKVStages), (uint32_t)(gkv / kKVStages) & 1u, g))) break;
                     for (int t = 0; t < 2 && ok; ++t) {
-                        if (!part(t, jlo + j)) continue;
-                        if (!(ok = mbar_wait(bar(kBarPFull + t), (uint32_t)pc[t] & 1u, g))) break;
-                        if (jlo + j == lo[t] && items[t] > 0 &&
-                            !(ok = mbar_wait(bar(kBarOFree + t), (uint32_t)(items[t] - 1) & 1u, g)))
-                            break;
+                        if (!part(t, jlo)) continue;
+                        if (sc[t] > 0 && !(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
                         tc_fence_after();
-                        issue_PV(t, st, jlo + j == lo[t]);
+                        issue_S(qs, t, gkv % kKVStages);
+                        any = true;
                     }
-                    if (ok) umma_commit(bar(kBarKVEmpty + st));
+                    for (int j = 0; j < nkv && ok; ++j) {
+                        const int st = (gkv + j) % kKVStages;
+                        // S of the next key tile for each stream, as soon as its S buffer is free
+                        if (j + 1 < nkv) {
+                            const int st1 = (gkv + j + 1) % kKVStages;
+                            if (!(ok = mbar_wait(bar(kBarKFull + st1), (uint32_t)((gkv + j + 1) / kKVStages) & 1u, g))) break;
+                            for (int t = 0; t < 2 && ok; ++t) {
+                                if (!part(t, jlo + j + 1)) continue;
+                                if (!(ok = mbar_wait(bar(kBarSEmpty + t), (uint32_t)(sc[t] - 1) & 1u, g))) break;
+                                tc_fence_after();
+                                issue_S(qs, t, st1);
+                            }
+                            if (!ok) break;
+                        }
+                        // P V of key tile j for each stream
+                        if (!(ok = mbar_wait(bar(kBarVFull + st), (uint32_t)((gkv + j) / kKVStages) & 1u, g))) break;
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (!part(t, jlo + j)) continue;
+                            if (!(ok = mbar_wait(bar(kBarPFull + t), (uint32_t)pc[t] & 1u, g))) break;
+                            if (jlo + j == lo[t] && items[t] > 0 &&
+                                !(ok = mbar_wait(bar(kBarOFree + t), (uint32_t)(items[t] - 1) & 1u, g)))
+                                break;
+                            tc_fence_after();
+                            issue_PV(t, st, jlo + j == lo[t]);
+                        }
+                        if (ok) umma_commit(bar(kBarKVEmpty + st));
+                    }
+                    gkv += nkv;
+                    items[0] += 1;
+                    items[1] += hasB ? 1 : 0;
                 }
-                gkv += nkv;
-                items[0] += 1;
-                items[1] += hasB ? 1 : 0;
-            }
-            if (any) {
-                umma_commit(bar(kBarDone));
-                drain_wait(bar(kBarDone), 0, budget_ns);
+                if (any) {
+                    umma_commit(bar(kBarDone));
+                    drain_wait(bar(kBarDone), 0, budget_ns);
+                }
             }
         }
     } else {
         // ================================================================ softmax warpgroups
-        const int t = (warp - 2) >> 2;
+        regs_inc<kRegsSoftmax>();
+        const int t = wg - 1;
         const int sp = warp & 3;
         const int row = sp * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
@@ -314,6 +325,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j_edge = (qt * kTile + kTile - 1 - window) / kTile;
             float mrow = -INFINITY, l = 0.f, l_r = 0.f;
             for (int j = jlo_t; j <= qt; ++j, ++it) {
+                // dropout keep bits of this row's 128 keys of tile j (bit c%32 of kb[c/32] <-> key
+                // j*128 + c), drawn before S is loaded so the generator's registers are free again
+                uint32_t kb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
+                if constexpr (kDropout) {
+                    const uint32_t t_row = (uint32_t)(qt * kTile + row);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint32_t bits = dropout_keep32_rows(dp.seed, dp.threshold, (uint32_t)bh, t_row,
+                                                                  (uint32_t)(j * kTile + 32 * q), lane);
+                        kb[0] = q == 0 ? bits : kb[0];
+                        kb[1] = q == 1 ? bits : kb[1];
+                        kb[2] = q == 2 ? bits : kb[2];
+                        kb[3] = q == 3 ? bits : kb[3];
+                    }
+                }
                 if (ok) ok = warp_wait(bar(kBarSFull + t), (uint32_t)it & 1u, g);
                 if (!ok) continue;
                 tc_fence_after();
@@ -367,22 +393,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the exponentials; with dropout the stored weights are masked, the sums are not
                 auto exps = [&](auto drop_tag) {
                     constexpr bool kDrop = decltype(drop_tag)::value;
-                    uint32_t keep4 = 0xFu;
-                    const uint32_t t_row = (uint32_t)(qt * kTile + row);
 #pragma unroll
                     for (int c = 0; c < 128; c += 2) {
-                        if constexpr (kDrop) {
-                            if ((c & 3) == 0)
-                                keep4 = dropout_keep4(dp.seed, dp.threshold, (uint32_t)bh, t_row, (uint32_t)(j * kTile + c));
-                        }
                         const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
                         float x0, x1;
                         f32x2_unpack(x, x0, x1);
                         const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         const uint32_t wv = pack_bf16x2(p0, p1);
                         if constexpr (kDrop) {
-                            const uint32_t m = (((keep4 >> (c & 3)) & 1u) ? 0x0000FFFFu : 0u) |
-                                               (((keep4 >> ((c + 1) & 3)) & 1u) ? 0xFFFF0000u : 0u);
+                            const uint32_t kw = kb[c >> 5];
+                            const uint32_t m = (((kw >> (c & 31)) & 1u) ? 0x0000FFFFu : 0u) |
+                                               (((kw >> ((c + 1) & 31)) & 1u) ? 0xFFFF0000u : 0u);
                             pk[c >> 1] = wv & m;
                         } else {
                             pk[c >> 1] = wv;
@@ -474,6 +495,12 @@ cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y,
     auto kern = dp.threshold != 0u ? fwd_h64_kernel<true> : fwd_h64_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
+    // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs per
+    // thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

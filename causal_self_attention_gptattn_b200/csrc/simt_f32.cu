@@ -17,7 +17,7 @@ namespace gptattn {
 namespace {
 
 // Dropout factor of the weight of query t for key s: 1 without dropout, else
-// 1/(1-p) if the Philox mask keeps it and 0 if not.
+// 1/(1 - theta/256) if the Philox mask keeps it and 0 if not.
 __device__ __forceinline__ float drop_factor(const DropoutParams &dp, int bh, int t, int s) {
     if (dp.threshold == 0u) return 1.f;
     const uint32_t bits = dropout_keep4(dp.seed, dp.threshold, (uint32_t)bh, (uint32_t)t, (uint32_t)(s & ~3));

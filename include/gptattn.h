@@ -130,13 +130,17 @@ GPTATTN_API gptattn_status gptattn_bwd_det(const void *qkv, const void *y, const
  *   dropout_p     probability of dropping an attention weight, 0 <= p < 1 (else
  *                 GPTATTN_ERR_INVALID_ARG).  Inverted dropout on the weights after
  *                 the softmax (the lecture page's chapter "scaling up the model! ...
- *                 adding dropout"): a kept weight is scaled by 1/(1-p); lse stays
- *                 the logsumexp of the undropped scores.  Weight (t, s) of batch b,
- *                 head h is kept iff word s%4 of Philox4x32-10 (Salmon et al.,
- *                 SC 2011) at counter (s/4, t, b*n_head+h, 0) under key
- *                 (seed & 0xffffffff, seed >> 32) is >= floor(p * 2^32); p < 2^-32
- *                 drops nothing.  The backward must get the forward's seed and p.
- *                 bf16 dropout needs head size 64.
+ *                 adding dropout"); lse stays the logsumexp of the undropped
+ *                 scores.  p is applied in steps of 1/256: with theta = round(256 p)
+ *                 (at most 255) a weight is dropped with probability theta/256 and
+ *                 a kept one is scaled by 1/(1 - theta/256); p < 1/512 drops
+ *                 nothing.  One Philox4x32-10 call (Salmon et al., SC 2011) covers
+ *                 a 4 x 4 block of (query t, key s) pairs of batch b, head h:
+ *                 counter (s/4, t/4, b*n_head+h, 0) under key (seed & 0xffffffff,
+ *                 seed >> 32); weight (t, s) is kept iff byte s%4 (least
+ *                 significant first) of output word t%4 is >= theta.  The backward
+ *                 must get the forward's seed and p.  bf16 dropout needs head size
+ *                 64.
  *   dropout_seed  the 64-bit Philox key.
  *   deterministic backward only: bit-identical results as gptattn_bwd_det (and
  *                 its workspace size). */

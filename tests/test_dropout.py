@@ -51,12 +51,13 @@ def test_dropout_mask_bits_match_the_oracle_generator():
     dy = torch.zeros(1, T, C)
     for dtype in (torch.float32, torch.bfloat16):
         y, _, _ = run_fwd_bwd(qkv.to(dtype), dy.to(dtype), n_head, opts=ga.Options(dropout_p=p, dropout_seed=seed))
-        thr = math.floor(float(np.float32(p)) * 2.0 ** 32)
+        thr = min(255, math.floor(256.0 * float(np.float32(p)) + 0.5))  # theta = round(256 p)
         for h in range(n_head):
             for t in range(T):
                 for s in range(t + 1):
-                    r = oracle.philox([s // 4, t, h, 0], [seed & 0xFFFFFFFF, seed >> 32])
-                    assert (r[s % 4] >= thr) == (y[0, t, h * hs + s] > 0), (str(dtype), h, t, s)
+                    r = oracle.philox([s // 4, t // 4, h, 0], [seed & 0xFFFFFFFF, seed >> 32])
+                    kept = ((r[t % 4] >> (8 * (s % 4))) & 0xFF) >= thr
+                    assert kept == (y[0, t, h * hs + s] > 0), (str(dtype), h, t, s)
 
 
 def test_dropout_zero_is_the_plain_path_and_seeds_matter():
