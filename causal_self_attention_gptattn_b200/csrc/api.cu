@@ -406,8 +406,11 @@ gptattn_status bwd_impl(const void *qkv, const void *y, const float *lse, const 
         return fail_cuda("tensor map encoding failed");
     const int n_slots = det ? (int)det_slots(T) : 0;
     const DevCtx ctx{status, kDefaultBudgetNs};
+    // dropout's scale s = 256 / (256 - theta) folded into the recomputed weights (log2 s) and D (1/s)
+    const float lse_bias = dp.threshold ? (float)log2(256.0 / (256.0 - dp.threshold)) : 0.f;
+    const float d_mul = dp.threshold ? (float)((256.0 - dp.threshold) / 256.0) : 1.f;
     cudaError_t e = run_kernel(kKBwdPreBf16, s, [&] {
-        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, !det, s);
+        return launch_bwd_pre_bf16(hs, y, dy, lse, D, lse2, dqacc, B, T, C, n_head, T_pad, !det, lse_bias, d_mul, s);
     });
     if (e == cudaSuccess)
         e = run_kernel(kKBwdMainBf16, s, [&] {

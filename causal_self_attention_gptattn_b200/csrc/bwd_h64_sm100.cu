@@ -71,8 +71,14 @@ constexpr uint32_t kOffdQ = kOffdS + 2 * kSlabBytes;             // 128 x 32 fp3
 constexpr uint32_t kOffLse = kOffdQ + kSlabBytes;                // kQStages x 128 fp32
 constexpr uint32_t kOffD = kOffLse + kQStages * 512;             // kQStages x 128 fp32
 constexpr uint32_t kOffBar = kOffD + kQStages * 512;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+constexpr uint32_t kBarArea = 512;
+// dropout keep bits, drawn ahead by warps 2 and 3: kMStages tiles of 128 key rows x 128 query bits
+constexpr int kMStages = 4;
+constexpr uint32_t kMaskTileBytes = 128u * 16u;
+constexpr uint32_t kOffM = kOffBar + kBarArea;
+template <bool kDropout>
+constexpr uint32_t smem_bytes() { return kOffM + (kDropout ? kMStages * kMaskTileBytes : 0u) + 1024; }
+static_assert(smem_bytes<true>() <= 227 * 1024, "shared memory");
 
 // TMEM columns
 constexpr uint32_t kColS = 0, kColdP = 128, kColP = 256, kColdV = 320, kColdK = 384, kColdQ = 448;
@@ -95,8 +101,11 @@ constexpr int kBardQEmpty = kBardQFull + 1;
 constexpr int kBarKdV = kBardQEmpty + 1;
 constexpr int kBarAccFree = kBarKdV + 1;
 constexpr int kBarDone = kBarAccFree + 1;
-constexpr int kNumBars = kBarDone + 1;
-static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
+constexpr int kBarMFull = kBarDone + 1;          // kMStages
+constexpr int kBarMEmpty = kBarMFull + kMStages;  // kMStages
+constexpr int kNumBars = kBarMEmpty + kMStages;
+static_assert(kNumBars * 8 + 16 <= kBarArea, "barrier area");
+constexpr int kMaskThreads = 64;
 
 constexpr int kSoftmaxThreads = 256;
 constexpr int kDrainThreads = 128;
@@ -154,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sdS = sbase + kOffdS, sdQ = sbase + kOffdQ;
     const float *sLse = reinterpret_cast<const float *>(smem + kOffLse);
     const float *sD = reinterpret_cast<const float *>(smem + kOffD);
+    auto sM = [&](int s) -> uint32_t { return sbase + kOffM + (uint32_t)s * kMaskTileBytes; };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKVStages; ++s) {
@@ -177,6 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(kBarKdV), 1);
         mbar_init(bar(kBarAccFree), kDrainThreads);
         mbar_init(bar(kBarDone), 1);
+        for (int s = 0; s < kMStages; ++s) {
+            mbar_init(bar(kBarMFull + s), kMaskThreads);
+            mbar_init(bar(kBarMEmpty + s), kSoftmaxThreads);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -343,6 +357,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                     drain_wait(bar(kBarDone), 0, budget_ns);
                 }
             }
+        } else {
+            // ================================================================ dropout mask (warps 2, 3)
+            if constexpr (kDropout) {
+                // thread -> key rows 4*kg .. 4*kg+3 and query columns 64*qh .. 64*qh+63 of every
+                // mask tile, tiles in the order the softmax warps use them
+                const int u = threadIdx.x - 64;
+                const int kg = u >> 1, qh = u & 1;
+                bool ok = true;
+                int gi = 0;
+                for (int k = 0; ok; ++k) {
+                    const int w = item_index(k, blockIdx.x, gridDim.x);
+                    if (w >= n_items) break;
+                    const int kt = w / BH, bh = w % BH;
+                    const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
+                    for (int it = 0; it < niter; ++it, ++gi) {
+                        const int ms = gi % kMStages;
+                        if (gi >= kMStages &&
+                            !(ok = warp_wait(bar(kBarMEmpty + ms), (uint32_t)((gi / kMStages) & 1) ^ 1u, g)))
+                            break;
+                        const uint32_t s0 = (uint32_t)(kt * kTile + 4 * kg);
+                        const uint32_t t0 = (uint32_t)((kt + it) * kTile + 64 * qh);
+                        uint32_t lo[4], hi[4];
+                        dropout_keep32x4_keys(dp.seed, dp.threshold, (uint32_t)bh, s0, t0, lo);
+                        dropout_keep32x4_keys(dp.seed, dp.threshold, (uint32_t)bh, s0, t0 + 32u, hi);
+                        const uint32_t dst = sM(ms) + (uint32_t)(4 * kg) * 16u + (uint32_t)qh * 8u;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) st_shared_v2(dst + (uint32_t)c * 16u, lo[c], hi[c]);
+                        mbar_arrive(bar(kBarMFull + ms));
+                    }
+                }
+            }
         }
     } else if (wg < 3) {
         regs_inc<kRegsSoftmax>();
@@ -363,10 +408,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = 0; it < niter; ++it, ++gi) {
                 const int st = gi % kQStages;
                 const uint32_t ph = (uint32_t)gi & 1u;
+                uint32_t keepb[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};  // dropout keep bits of the 64 columns
+                if constexpr (kDropout) {
+                    const int ms = gi % kMStages;
+                    if (ok) ok = warp_wait(bar(kBarMFull + ms), (uint32_t)(gi / kMStages) & 1u, g);
+                    if (ok) {
+                        const uint2 v = ld_shared_v2(sM(ms) + (uint32_t)row * 16u + (uint32_t)half * 8u);
+                        keepb[0] = v.x;
+                        keepb[1] = v.y;
+                        mbar_arrive(bar(kBarMEmpty + ms));
+                    }
+                }
                 if (ok) ok = warp_wait(bar(kBarQFull + st), (uint32_t)(gi / kQStages) & 1u, g);
                 if (ok) ok = warp_wait(bar(kBarSFull), ph, g);
                 float pf[64];  // P^T row segment, fp32
-                uint32_t keepb[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};  // dropout keep bits of the 64 columns
                 if (ok) {
                     tc_fence_after();
                     uint32_t sr[64];
@@ -410,21 +465,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (c >= cut) pf[c] = 0.f;
                     }
                     uint32_t pk[32];
-                    if constexpr (kDropout) {  // keep bits of this row's 64 columns; P^T dropped + rescaled
-                        // generator calls shared by the 4 lanes of this key row's 4 x 4 blocks
-                        const uint32_t skey = (uint32_t)(kt * kTile + row);
-                        const uint32_t tq0 = (uint32_t)((kt + it) * kTile + 64 * half);
-                        uint32_t kq[4];
-#pragma unroll
-                        for (int m = 0; m < 4; ++m)
-                            kq[m] = dropout_keep16_keys(dp.seed, dp.threshold, (uint32_t)bh, tq0 + 16u * m, skey, lane);
-                        keepb[0] = kq[0] | (kq[1] << 16);
-                        keepb[1] = kq[2] | (kq[3] << 16);
+                    if constexpr (kDropout) {  // P^T dropped with this row's 64 keep bits (already scaled)
 #pragma unroll
                         for (int c = 0; c < 32; ++c) {
-                            const float f0 = ((keepb[(2 * c) >> 5] >> ((2 * c) & 31)) & 1u) ? dp.scale : 0.f;
-                            const float f1 = ((keepb[(2 * c + 1) >> 5] >> ((2 * c + 1) & 31)) & 1u) ? dp.scale : 0.f;
-                            pk[c] = pack_bf16x2(pf[2 * c] * f0, pf[2 * c + 1] * f1);
+                            const int cc = (2 * c) & 31;
+                            pk[c] = pack_bf16x2(pf[2 * c], pf[2 * c + 1]) &
+                                    keep_pair_mask(keepb[(2 * c) >> 5] << (cc >> 2), (cc >> 1) & 1);
                         }
                     } else {
 #pragma unroll
@@ -453,7 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_before();
                             mbar_arrive(bar(kBardPEmpty));
                         }
-                        // dS^T = P^T o (dP^T o f - D); f = 1 without dropout
+                        // dS^T = P^T o (dP^T o f - D), f the dropout factor (1 without dropout); with
+                        // dropout the preprocess folded f's scale into lse and D, so pf holds P^T * scale
+                        // and D / scale arrives here: dS^T = pf o (dP^T o keep - D / scale)
                         auto ds_chunk = [&](auto drop_tag) {
                             constexpr bool kDrop = decltype(drop_tag)::value;
 #pragma unroll
@@ -465,15 +513,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     const float4 d = D4[2 * q + e];
                                     const int c = 8 * q + 4 * e;      // column within the half
                                     const int cr = 8 * qq + 4 * e;    // column within this dP chunk
-                                    uint64_t g01 = f32x2_pack(__uint_as_float(dr[cr]), __uint_as_float(dr[cr + 1]));
-                                    uint64_t g23 = f32x2_pack(__uint_as_float(dr[cr + 2]), __uint_as_float(dr[cr + 3]));
-                                    if constexpr (kDrop) {
-                                        auto fac = [&](int cc) {
-                                            return ((keepb[cc >> 5] >> (cc & 31)) & 1u) ? dp.scale : 0.f;
-                                        };
-                                        g01 = fmul2(g01, f32x2_pack(fac(c), fac(c + 1)));
-                                        g23 = fmul2(g23, f32x2_pack(fac(c + 2), fac(c + 3)));
+                                    uint32_t g[4] = {dr[cr], dr[cr + 1], dr[cr + 2], dr[cr + 3]};
+                                    if constexpr (kDrop) {  // dropped columns: dP^T o f = 0
+                                        const uint32_t ws = keepb[c >> 5] << ((c & 31) >> 2);
+#pragma unroll
+                                        for (int kk = 0; kk < 4; ++kk) g[kk] &= keep_word_mask(ws, kk);
                                     }
+                                    const uint64_t g01 = f32x2_pack(__uint_as_float(g[0]), __uint_as_float(g[1]));
+                                    const uint64_t g23 = f32x2_pack(__uint_as_float(g[2]), __uint_as_float(g[3]));
                                     const uint64_t a01 = fadd2(g01, f32x2_pack(d.x, d.y));
                                     const uint64_t a23 = fadd2(g23, f32x2_pack(d.z, d.w));
                                     const uint64_t s01 = fmul2(a01, f32x2_pack(pf[c], pf[c + 1]));
@@ -595,9 +642,10 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
                                 const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
                                 int n_head, int T_pad, int window, int n_slots, DropoutParams dp, DevCtx ctx,
                                 cudaStream_t s) {
-    auto kern = dp.threshold != 0u ? bwd_h64_persistent<true> : bwd_h64_persistent<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    const bool drop = dp.threshold != 0u;
+    auto kern = drop ? bwd_h64_persistent<true> : bwd_h64_persistent<false>;
+    const uint32_t smem = drop ? smem_bytes<true>() : smem_bytes<false>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs per
     // thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
@@ -612,7 +660,7 @@ cudaError_t launch_bwd_main_h64(const CUtensorMap &map_qkv, const CUtensorMap &m
     const int n_t = ceil_div(T, kTile);
     const long long items = (long long)n_t * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_dy, map_dqkv,
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), smem, s, map_qkv, map_dy, map_dqkv,
                       map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, dp, ctx.status, ctx.budget_ns);
 }
 

@@ -446,6 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // preprocess: per (b, h, t) store -D = -rowsum(dy o y) and -lse * log2(e)
 // (negated so the main kernels add them); rows t >= T of each (b, h) get
 // 0 and -inf (so the recomputed P there is 0); dQ accumulator zeroed.
+// With dropout (kept weights scaled by s = 1/(1-p)) the caller passes
+// lse_bias = log2(s) and d_mul = 1/s: the main kernel's recomputed weights are
+// then P * s, what the dV product needs, and dS = (P s) o (dP o keep - D / s).
 // ---------------------------------------------------------------------------
 // 128-thread blocks, so that a whole (B * n_head, T_pad / 128) grid is resident at once
 // for the usual sizes (16 blocks per SM).
@@ -460,7 +463,8 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
                                                       const __nv_bfloat16 *__restrict__ dy,
                                                       const float *__restrict__ lse, float *__restrict__ D,
                                                       float *__restrict__ lse2, float4 *__restrict__ dqacc, int T,
-                                                      int C, int n_head, int T_pad, int zero_acc) {
+                                                      int C, int n_head, int T_pad, int zero_acc, float lse_bias,
+                                                      float d_mul) {
     constexpr int kLanesPerRow = HS / 8;
     constexpr int kRowsPerPass = kPPThreads / kLanesPerRow;
     griddep_launch_dependents();
@@ -486,8 +490,8 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
 #pragma unroll
         for (int o = kLanesPerRow / 2; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
         if (part == 0) {  // stored negated: -D and -lse*log2(e); padded rows 0 and -inf
-            D[row0 + r + sub] = -d;
-            lse2[row0 + r + sub] = t < T ? -lse[(size_t)bh * T + t] * 1.4426950408889634f : -INFINITY;
+            D[row0 + r + sub] = -d * d_mul;
+            lse2[row0 + r + sub] = t < T ? -lse[(size_t)bh * T + t] * 1.4426950408889634f + lse_bias : -INFINITY;
         }
     }
     if (!zero_acc) return;
@@ -581,7 +585,8 @@ cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_
 }  // namespace
 
 cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
-                                float *dqacc, int B, int T, int C, int n_head, int T_pad, bool zero_acc, cudaStream_t s) {
+                                float *dqacc, int B, int T, int C, int n_head, int T_pad, bool zero_acc, float lse_bias,
+                                float d_mul, cudaStream_t s) {
     const dim3 grid((unsigned)(B * n_head), (unsigned)(T_pad / kTile));
     auto yy = static_cast<const __nv_bfloat16 *>(y);
     auto gg = static_cast<const __nv_bfloat16 *>(dy);
@@ -589,10 +594,10 @@ cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const flo
     const int za = zero_acc ? 1 : 0;
     if (hs == 64)
         return launch_pdl(bwd_pre_kernel<64>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad,
-                          za);
+                          za, lse_bias, d_mul);
     if (hs == 128)
         return launch_pdl(bwd_pre_kernel<128>, grid, dim3(kPPThreads), 0, s, yy, gg, lse, D, lse2, zz, T, C, n_head, T_pad,
-                          za);
+                          za, lse_bias, d_mul);
     return cudaErrorInvalidValue;
 }
 

@@ -37,11 +37,23 @@
 namespace gptattn {
 namespace {
 
-constexpr int kThreads = 384;
-// register budgets per thread (sum = 3 x kLaunchRegs, what the CTA is launched with)
-constexpr int kLaunchRegs = 168;
-constexpr uint32_t kRegsCtl = 88, kRegsSoftmax = 208;
-static_assert(kRegsCtl + 2 * kRegsSoftmax == 3 * kLaunchRegs, "register split");
+constexpr int kMStages = 4;  // dropout mask ring, per query-tile stream
+constexpr uint32_t kMaskTileBytes = 128u * 16u;  // 128 query rows x 128 keep bits
+
+// Threads and register budgets per thread.  The plain kernel has three
+// warpgroups (control, two softmax); with dropout a fourth draws the keep bits
+// into shared memory.  The budgets add up to (warpgroups x kLaunchRegs), what
+// the CTA is launched with.
+template <bool kDropout>
+struct FwdCfg {
+    static constexpr int kThreads = kDropout ? 512 : 384;
+    static constexpr int kLaunchRegs = kDropout ? 128 : 168;
+    static constexpr uint32_t kRegsCtl = kDropout ? 80 : 88;
+    static constexpr uint32_t kRegsSoftmax = kDropout ? 192 : 208;
+    static constexpr uint32_t kRegsMask = kDropout ? 48 : 0;
+    static constexpr uint32_t kMaskBytes = kDropout ? 2u * kMStages * kMaskTileBytes : 0u;
+    static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsMask == (kThreads / 128) * kLaunchRegs, "register split");
+};
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlabBytes = 128 * 128;
 constexpr int HS = 64;
@@ -52,8 +64,11 @@ constexpr uint32_t kOffQ = 0;                                   // kQStages x 2 
 constexpr uint32_t kOffK = kOffQ + kQStages * 2 * kTileBytes;    // kKVStages tiles
 constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;       // kKVStages tiles
 constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
-static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+constexpr uint32_t kBarArea = 512;
+constexpr uint32_t kOffM = kOffBar + kBarArea;                   // 2 streams x kMStages mask tiles
+template <bool kDropout>
+constexpr uint32_t smem_bytes() { return kOffM + FwdCfg<kDropout>::kMaskBytes + 1024; }
+static_assert(smem_bytes<true>() <= 227 * 1024, "shared memory");
 constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;  // + 128 t, + 64 t, + 64 t
 
 constexpr int kBarQFull = 0;
@@ -67,8 +82,10 @@ constexpr int kBarPFull = kBarSEmpty + 2;           // 2
 constexpr int kBarPVDone = kBarPFull + 2;           // 2
 constexpr int kBarOFree = kBarPVDone + 2;           // 2
 constexpr int kBarDone = kBarOFree + 2;
-constexpr int kNumBars = kBarDone + 1;
-static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
+constexpr int kBarMFull = kBarDone + 1;              // 2 x kMStages
+constexpr int kBarMEmpty = kBarMFull + 2 * kMStages;  // 2 x kMStages
+constexpr int kNumBars = kBarMEmpty + 2 * kMStages;
+static_assert(kNumBars * 8 + 16 <= kBarArea, "barrier area");
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitGuard &g) {
     bool ok = mbar_wait(bar, parity, g);
@@ -93,10 +110,11 @@ __device__ __forceinline__ int item_index(int k, int cta, int grid) {
 }
 
 template <bool kDropout>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
     fwd_h64_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
                    float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, DropoutParams dp,
                    int *status, unsigned long long budget_ns) {
+    using Cfg = FwdCfg<kDropout>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);
@@ -119,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto sQ = [&](int qs, int t) -> uint32_t { return sbase + kOffQ + (uint32_t)(2 * qs + t) * kTileBytes; };
     auto sK = [&](int st) -> uint32_t { return sbase + kOffK + (uint32_t)st * kTileBytes; };
     auto sV = [&](int st) -> uint32_t { return sbase + kOffV + (uint32_t)st * kTileBytes; };
+    auto sM = [&](int t, int st) -> uint32_t { return sbase + kOffM + (uint32_t)(t * kMStages + st) * kMaskTileBytes; };
     auto decode = [&](int w, int &m, int &bh) {
         m = n_pairs - 1 - w / BH;
         bh = w % BH;
@@ -140,6 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(kBarPFull + t), 128);
             mbar_init(bar(kBarPVDone + t), 1);
             mbar_init(bar(kBarOFree + t), 128);
+            for (int st = 0; st < kMStages; ++st) {
+                mbar_init(bar(kBarMFull + t * kMStages + st), 128);
+                mbar_init(bar(kBarMEmpty + t * kMStages + st), 128);
+            }
         }
         mbar_init(bar(kBarDone), 1);
         *abort_flag = 0;
@@ -157,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
     if (wg == 0) {
-        regs_dec<kRegsCtl>();
+        regs_dec<Cfg::kRegsCtl>();
         if (warp == 0) {
             // ================================================================ producer
             if (lane == 0) {
@@ -293,9 +316,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else {
+    } else if (wg <= 2) {
         // ================================================================ softmax warpgroups
-        regs_inc<kRegsSoftmax>();
+        regs_inc<Cfg::kRegsSoftmax>();
         const int t = wg - 1;
         const int sp = warp & 3;
         const int row = sp * 32 + lane;
@@ -326,19 +349,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             float mrow = -INFINITY, l = 0.f, l_r = 0.f;
             for (int j = jlo_t; j <= qt; ++j, ++it) {
                 // dropout keep bits of this row's 128 keys of tile j (bit c%32 of kb[c/32] <-> key
-                // j*128 + c), drawn before S is loaded so the generator's registers are free again
+                // j*128 + c), drawn ahead by the mask warpgroup; tile number `it` of this stream
                 uint32_t kb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
                 if constexpr (kDropout) {
-                    const uint32_t t_row = (uint32_t)(qt * kTile + row);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint32_t bits = dropout_keep32_rows(dp.seed, dp.threshold, (uint32_t)bh, t_row,
-                                                                  (uint32_t)(j * kTile + 32 * q), lane);
-                        kb[0] = q == 0 ? bits : kb[0];
-                        kb[1] = q == 1 ? bits : kb[1];
-                        kb[2] = q == 2 ? bits : kb[2];
-                        kb[3] = q == 3 ? bits : kb[3];
-                    }
+                    const int ms = it % kMStages;
+                    if (ok) ok = warp_wait(bar(kBarMFull + t * kMStages + ms), (uint32_t)(it / kMStages) & 1u, g);
+                    if (!ok) continue;
+                    const uint4 v = ld_shared_v4(sM(t, ms) + (uint32_t)row * 16u);
+                    kb[0] = v.x;
+                    kb[1] = v.y;
+                    kb[2] = v.z;
+                    kb[3] = v.w;
+                    mbar_arrive(bar(kBarMEmpty + t * kMStages + ms));
                 }
                 if (ok) ok = warp_wait(bar(kBarSFull + t), (uint32_t)it & 1u, g);
                 if (!ok) continue;
@@ -401,10 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         const uint32_t wv = pack_bf16x2(p0, p1);
                         if constexpr (kDrop) {
-                            const uint32_t kw = kb[c >> 5];
-                            const uint32_t m = (((kw >> (c & 31)) & 1u) ? 0x0000FFFFu : 0u) |
-                                               (((kw >> ((c + 1) & 31)) & 1u) ? 0xFFFF0000u : 0u);
-                            pk[c >> 1] = wv & m;
+                            const int cc = c & 31;
+                            pk[c >> 1] = wv & keep_pair_mask(kb[c >> 5] << (cc >> 2), (cc >> 1) & 1);
                         } else {
                             pk[c >> 1] = wv;
                         }
@@ -478,6 +498,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (leader) bulk_wait_group_0();
+    } else {
+        // ================================================================ dropout mask warpgroup
+        if constexpr (kDropout) {
+            regs_dec<Cfg::kRegsMask>();
+            // thread -> rows 4*rg .. 4*rg+3 and keys 32*kq .. 32*kq+31 of every mask tile;
+            // tiles in the order the softmax warpgroups use them (key tile by key tile,
+            // stream A before stream B), each stream through its own ring
+            const int rg = (warp & 3) * 8 + (lane >> 2), kq = lane & 3;
+            bool ok = true;
+            int mc[2] = {0, 0};
+            for (int k = 0; ok; ++k) {
+                const int w = item_index(k, cta, grid);
+                if (w >= n_items) break;
+                int m, bh;
+                decode(w, m, bh);
+                const bool hasB = 2 * m + 1 < n_qt;
+                const int lo[2] = {band_lo_tile(2 * m, window), hasB ? band_lo_tile(2 * m + 1, window) : 1};
+                const int hi[2] = {2 * m, hasB ? 2 * m + 1 : 0};
+                for (int j = lo[0]; j <= hi[1] || j <= hi[0]; ++j) {
+                    for (int t = 0; t < 2; ++t) {
+                        if (j < lo[t] || j > hi[t]) continue;
+                        const int ms = mc[t] % kMStages;
+                        if (mc[t] >= kMStages &&
+                            !(ok = warp_wait(bar(kBarMEmpty + t * kMStages + ms), (uint32_t)((mc[t] / kMStages) & 1) ^ 1u, g)))
+                            break;
+                        uint32_t bits[4];
+                        dropout_keep32x4(dp.seed, dp.threshold, (uint32_t)bh, (uint32_t)((2 * m + t) * kTile + 4 * rg),
+                                         (uint32_t)(j * kTile + 32 * kq), bits);
+                        const uint32_t dst = sM(t, ms) + (uint32_t)(4 * rg) * 16u + (uint32_t)kq * 4u;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) st_shared_u32(dst + (uint32_t)r * 16u, bits[r]);
+                        mbar_arrive(bar(kBarMFull + t * kMStages + ms));
+                        ++mc[t];
+                    }
+                    if (!ok) break;
+                }
+            }
+        }
     }
 
     tc_fence_before();
@@ -492,15 +550,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
                            int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
-    auto kern = dp.threshold != 0u ? fwd_h64_kernel<true> : fwd_h64_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    const bool drop = dp.threshold != 0u;
+    auto kern = drop ? fwd_h64_kernel<true> : fwd_h64_kernel<false>;
+    const uint32_t smem = drop ? smem_bytes<true>() : smem_bytes<false>();
+    const int threads = drop ? FwdCfg<true>::kThreads : FwdCfg<false>::kThreads;
+    const int launch_regs = drop ? FwdCfg<true>::kLaunchRegs : FwdCfg<false>::kLaunchRegs;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs per
     // thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
     cudaFuncAttributes fa{};
     e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    if (fa.numRegs != launch_regs) return cudaErrorInvalidConfiguration;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -508,7 +570,7 @@ cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y,
     const int n_qt = ceil_div(T, kTile);
     const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, s, map_qkv, map_y, lse, B, T, C,
+    return launch_pdl(kern, dim3((unsigned)grid), dim3((unsigned)threads), smem, s, map_qkv, map_y, lse, B, T, C,
                       n_head, n_qt, window, dp, ctx.status, ctx.budget_ns);
 }
 

@@ -60,10 +60,12 @@ cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMa
 cudaError_t launch_fwd_h64(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
                            int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s);
 
-// D[bh][t] = sum_d y*dy, lse2[bh][t] = lse*log2(e) (rows t >= T: 0 and +inf),
-// dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].
+// D[bh][t] = -d_mul * sum_d y*dy, lse2[bh][t] = -lse*log2(e) + lse_bias (rows t >= T: 0 and
+// -inf), dqacc zeroed.  Row stride of D/lse2 is T_pad; dqacc is [B*n_head*T_pad][hs].  Without
+// dropout lse_bias = 0 and d_mul = 1; with dropout scale s, log2(s) and 1/s.
 cudaError_t launch_bwd_pre_bf16(int hs, const void *y, const void *dy, const float *lse, float *D, float *lse2,
-                                float *dqacc, int B, int T, int C, int n_head, int T_pad, bool zero_acc, cudaStream_t s);
+                                float *dqacc, int B, int T, int C, int n_head, int T_pad, bool zero_acc, float lse_bias,
+                                float d_mul, cudaStream_t s);
 
 // map_dy: 3-D view (C, T, B) of dy; map_dqkv: 3-D view (3C, T, B) of dqkv;
 // map_dq: 2-D view (hs, B*n_head*T_pad) of dqacc (fp32), box (32, 128), 128-byte swizzle.

@@ -44,64 +44,72 @@ __device__ __forceinline__ uint32_t dropout_keep4(uint64_t seed, uint32_t theta,
     return keep_bits4(q == 0u ? r.x : q == 1u ? r.y : q == 2u ? r.z : r.w, theta);
 }
 
-// Keep bits of the 4 queries t0 .. t0+3 (t0 a multiple of 4) for key s: bit i <-> query t0 + i.
-__device__ __forceinline__ uint32_t dropout_keep4_keys(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t t0,
-                                                       uint32_t s) {
-    const uint4 r = philox4x32_10(make_uint4(s >> 2, t0 >> 2, bh, 0u), (uint32_t)seed, (uint32_t)(seed >> 32));
-    const uint32_t sh = 8u * (s & 3u);
-    return (((r.x >> sh) & 0xFFu) >= theta ? 1u : 0u) | (((r.y >> sh) & 0xFFu) >= theta ? 2u : 0u) |
-           (((r.z >> sh) & 0xFFu) >= theta ? 4u : 0u) | (((r.w >> sh) & 0xFFu) >= theta ? 8u : 0u);
+// Keep flags of the four bytes of w against theta (1..255), each in its byte's
+// top bit: bit 8i+7 <-> byte i >= theta, every other bit 0.  Even and odd
+// bytes are compared in two 16-bit lanes: byte + 256 - theta reaches bit 8 of
+// its lane exactly when byte >= theta, and no lane carries into the next.
+__device__ __forceinline__ uint32_t keep_msb4(uint32_t w, uint32_t theta) {
+    const uint32_t k = (256u - theta) * 0x00010001u;
+    const uint32_t e = (w & 0x00FF00FFu) + k;         // bits 8, 24: bytes 0, 2
+    const uint32_t o = ((w >> 8) & 0x00FF00FFu) + k;  // bits 8, 24: bytes 1, 3
+    return ((e >> 1) & 0x00800080u) | ((o << 7) & 0x80008000u);
 }
 
-// The same decisions with the generator calls shared by the four lanes that hold
-// four consecutive query rows (forward) or key rows (backward) of one 4 x 4 block
-// row: lanes 4k..4k+3 of a warp, the row's lane at position row % 4.  Each lane
-// draws a quarter of the blocks and the four exchange what the others need in
-// four shuffle rounds (in round k, lane r reads from lane (r + k) % 4, which sends
-// the part meant for lane (its own position - k) % 4).  Every lane of the warp
-// must call these together.
+// Packed keep words.  A word holds the flags of 32 consecutive columns; column
+// 4j + k (j = 0..7, k = 0..3) is bit 8k + 7 - j, so that (word << j) carries
+// columns 4j .. 4j+3 in the top bits of its four bytes, where one byte permute
+// with sign replication turns them into masks (keep_pair_mask, keep_word_mask).
 
-// Keep bits of keys s_base .. s_base+31 (s_base a multiple of 32) for query t:
-// bit i <-> key s_base + i.  Requires lane % 4 == t % 4.
-__device__ __forceinline__ uint32_t dropout_keep32_rows(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t t,
-                                                        uint32_t s_base, int lane) {
-    const int r = lane & 3;
-    uint32_t acc = 0u;
+// Keep words of keys s0 .. s0+31 (s0 a multiple of 32) for the four queries
+// t0 .. t0+3 (t0 a multiple of 4): out[r] for query t0 + r, column i = key
+// s0 + i.  Eight generator calls, one per 4 x 4 block.
+__device__ __forceinline__ void dropout_keep32x4(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t t0, uint32_t s0,
+                                                 uint32_t (&out)[4]) {
+    out[0] = out[1] = out[2] = out[3] = 0u;
+#pragma unroll 2
+    for (int blk = 0; blk < 8; ++blk) {
+        const uint4 r = philox4x32_10(make_uint4((s0 >> 2) + (uint32_t)blk, t0 >> 2, bh, 0u), (uint32_t)seed,
+                                      (uint32_t)(seed >> 32));
+        out[0] |= keep_msb4(r.x, theta) >> blk;
+        out[1] |= keep_msb4(r.y, theta) >> blk;
+        out[2] |= keep_msb4(r.z, theta) >> blk;
+        out[3] |= keep_msb4(r.w, theta) >> blk;
+    }
+}
+
+// Keep words of queries t0 .. t0+31 (t0 a multiple of 32) for the four keys
+// s0 .. s0+3 (s0 a multiple of 4): out[c] for key s0 + c, column i = query
+// t0 + i.  Eight generator calls, one per 4 x 4 block.
+__device__ __forceinline__ void dropout_keep32x4_keys(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t s0,
+                                                      uint32_t t0, uint32_t (&out)[4]) {
+    out[0] = out[1] = out[2] = out[3] = 0u;
+#pragma unroll 2
+    for (int blk = 0; blk < 8; ++blk) {
+        const uint4 r = philox4x32_10(make_uint4(s0 >> 2, (t0 >> 2) + (uint32_t)blk, bh, 0u), (uint32_t)seed,
+                                      (uint32_t)(seed >> 32));
+        // byte c of word q: (query 4*blk + q, key s0 + c); gather byte c of the four words
 #pragma unroll
-    for (int hb = 0; hb < 2; ++hb) {  // key groups 4*hb .. 4*hb+3 of 4 keys; this lane draws group 4*hb + r
-        const uint4 blk = philox4x32_10(make_uint4((s_base >> 2) + 4u * hb + r, t >> 2, bh, 0u), (uint32_t)seed,
-                                        (uint32_t)(seed >> 32));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int w = (r - k) & 3;  // the row (word) wanted by the lane reading this one
-            const uint32_t send = w == 0 ? blk.x : w == 1 ? blk.y : w == 2 ? blk.z : blk.w;
-            const int src = (r + k) & 3;
-            const uint32_t got = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | src);
-            acc |= keep_bits4(got, theta) << (4 * (4 * hb + src));
+        for (int c = 0; c < 4; ++c) {
+            const uint32_t sel = (uint32_t)c | ((4u + (uint32_t)c) << 4);
+            out[c] |= keep_msb4(__byte_perm(__byte_perm(r.x, r.y, sel), __byte_perm(r.z, r.w, sel), 0x5410), theta) >>
+                      blk;
         }
     }
-    return acc;
 }
 
-// Keep bits of queries t_base .. t_base+15 (t_base a multiple of 16) for key s:
-// bit i <-> query t_base + i.  Requires lane % 4 == s % 4.
-__device__ __forceinline__ uint32_t dropout_keep16_keys(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t t_base,
-                                                        uint32_t s, int lane) {
-    const int r = lane & 3;
-    // this lane draws the block of queries t_base + 4r .. t_base + 4r + 3
-    const uint4 blk = philox4x32_10(make_uint4(s >> 2, (t_base >> 2) + r, bh, 0u), (uint32_t)seed,
-                                    (uint32_t)(seed >> 32));
-    uint32_t acc = 0u;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const uint32_t d = (uint32_t)((r - k) & 3);  // key position (byte) wanted by the reading lane
-        const uint32_t sel = d | ((4u + d) << 4);
-        const uint32_t send = __byte_perm(__byte_perm(blk.x, blk.y, sel), __byte_perm(blk.z, blk.w, sel), 0x5410);
-        const int src = (r + k) & 3;
-        const uint32_t got = __shfl_sync(0xFFFFFFFFu, send, (lane & ~3) | src);
-        acc |= keep_bits4(got, theta) << (4 * src);
-    }
-    return acc;
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+// Mask of the bf16 pair of columns 4j + 2h, 4j + 2h + 1 (0xFFFF per kept
+// column), from ws = word << j.
+__device__ __forceinline__ uint32_t keep_pair_mask(uint32_t ws, int h) {
+    return prmt_b32(ws, 0u, h ? 0xBBAAu : 0x9988u);
+}
+// Mask of the 32-bit value of column 4j + k (all ones if kept), from ws = word << j.
+__device__ __forceinline__ uint32_t keep_word_mask(uint32_t ws, int k) {
+    return prmt_b32(ws, 0u, 0x8888u | (0x1111u * (uint32_t)k));
 }
 
 // Dropout parameters as the kernels take them: threshold 0 means no dropout.
