@@ -364,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // mask tile, tiles in the order the softmax warps use them
                 const int u = threadIdx.x - 64;
                 const int kg = u >> 1, qh = u & 1;
+                const uint32_t t7 = theta_low7(dp.threshold);
                 bool ok = true;
                 int gi = 0;
                 for (int k = 0; ok; ++k) {
@@ -379,8 +380,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t s0 = (uint32_t)(kt * kTile + 4 * kg);
                         const uint32_t t0 = (uint32_t)((kt + it) * kTile + 64 * qh);
                         uint32_t lo[4], hi[4];
-                        dropout_keep32x4_keys(dp.seed, dp.threshold, (uint32_t)bh, s0, t0, lo);
-                        dropout_keep32x4_keys(dp.seed, dp.threshold, (uint32_t)bh, s0, t0 + 32u, hi);
+                        if (dp.threshold >= 128u) {
+                            dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
+                            dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
+                        } else {
+                            dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
+                            dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
+                        }
                         const uint32_t dst = sM(ms) + (uint32_t)(4 * kg) * 16u + (uint32_t)qh * 8u;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) st_shared_v2(dst + (uint32_t)c * 16u, lo[c], hi[c]);

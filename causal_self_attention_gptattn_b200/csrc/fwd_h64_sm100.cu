@@ -506,6 +506,7 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
             // tiles in the order the softmax warpgroups use them (key tile by key tile,
             // stream A before stream B), each stream through its own ring
             const int rg = (warp & 3) * 8 + (lane >> 2), kq = lane & 3;
+            const uint32_t t7 = theta_low7(dp.threshold);
             bool ok = true;
             int mc[2] = {0, 0};
             for (int k = 0; ok; ++k) {
@@ -524,8 +525,11 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
                             !(ok = warp_wait(bar(kBarMEmpty + t * kMStages + ms), (uint32_t)((mc[t] / kMStages) & 1) ^ 1u, g)))
                             break;
                         uint32_t bits[4];
-                        dropout_keep32x4(dp.seed, dp.threshold, (uint32_t)bh, (uint32_t)((2 * m + t) * kTile + 4 * rg),
-                                         (uint32_t)(j * kTile + 32 * kq), bits);
+                        const uint32_t t0 = (uint32_t)((2 * m + t) * kTile + 4 * rg), s0 = (uint32_t)(j * kTile + 32 * kq);
+                        if (dp.threshold >= 128u)
+                            dropout_keep32x4<true>(dp.seed, t7, (uint32_t)bh, t0, s0, bits);
+                        else
+                            dropout_keep32x4<false>(dp.seed, t7, (uint32_t)bh, t0, s0, bits);
                         const uint32_t dst = sM(t, ms) + (uint32_t)(4 * rg) * 16u + (uint32_t)kq * 4u;
 #pragma unroll
                         for (int r = 0; r < 4; ++r) st_shared_u32(dst + (uint32_t)r * 16u, bits[r]);

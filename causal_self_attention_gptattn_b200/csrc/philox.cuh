@@ -44,16 +44,19 @@ __device__ __forceinline__ uint32_t dropout_keep4(uint64_t seed, uint32_t theta,
     return keep_bits4(q == 0u ? r.x : q == 1u ? r.y : q == 2u ? r.z : r.w, theta);
 }
 
-// Keep flags of the four bytes of w against theta (1..255), each in its byte's
-// top bit: bit 8i+7 <-> byte i >= theta, every other bit 0.  Even and odd
-// bytes are compared in two 16-bit lanes: byte + 256 - theta reaches bit 8 of
-// its lane exactly when byte >= theta, and no lane carries into the next.
-__device__ __forceinline__ uint32_t keep_msb4(uint32_t w, uint32_t theta) {
-    const uint32_t k = (256u - theta) * 0x00010001u;
-    const uint32_t e = (w & 0x00FF00FFu) + k;         // bits 8, 24: bytes 0, 2
-    const uint32_t o = ((w >> 8) & 0x00FF00FFu) + k;  // bits 8, 24: bytes 1, 3
-    return ((e >> 1) & 0x00800080u) | ((o << 7) & 0x80008000u);
+// Keep flags of the four bytes of w against theta, each in its byte's top bit:
+// bit 8i+7 <-> byte i >= theta, every other bit 0.  t7 holds theta mod 128 in
+// every byte; kHigh = (theta >= 128).  Setting each byte's top bit and
+// subtracting t7 never borrows across bytes, and leaves the top bit set exactly
+// when the byte's low seven bits reach theta's; the byte's own top bit then
+// decides: with theta < 128 a set top bit is enough, with theta >= 128 it is
+// required.
+template <bool kHigh>
+__device__ __forceinline__ uint32_t keep_msb4(uint32_t w, uint32_t t7) {
+    const uint32_t d = (w | 0x80808080u) - t7;
+    return kHigh ? (w & d & 0x80808080u) : ((w | d) & 0x80808080u);
 }
+__device__ __forceinline__ uint32_t theta_low7(uint32_t theta) { return (theta & 0x7Fu) * 0x01010101u; }
 
 // Packed keep words.  A word holds the flags of 32 consecutive columns; column
 // 4j + k (j = 0..7, k = 0..3) is bit 8k + 7 - j, so that (word << j) carries
@@ -63,37 +66,42 @@ __device__ __forceinline__ uint32_t keep_msb4(uint32_t w, uint32_t theta) {
 // Keep words of keys s0 .. s0+31 (s0 a multiple of 32) for the four queries
 // t0 .. t0+3 (t0 a multiple of 4): out[r] for query t0 + r, column i = key
 // s0 + i.  Eight generator calls, one per 4 x 4 block.
-__device__ __forceinline__ void dropout_keep32x4(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t t0, uint32_t s0,
+template <bool kHigh>
+__device__ __forceinline__ void dropout_keep32x4(uint64_t seed, uint32_t t7, uint32_t bh, uint32_t t0, uint32_t s0,
                                                  uint32_t (&out)[4]) {
     out[0] = out[1] = out[2] = out[3] = 0u;
 #pragma unroll 2
     for (int blk = 0; blk < 8; ++blk) {
         const uint4 r = philox4x32_10(make_uint4((s0 >> 2) + (uint32_t)blk, t0 >> 2, bh, 0u), (uint32_t)seed,
                                       (uint32_t)(seed >> 32));
-        out[0] |= keep_msb4(r.x, theta) >> blk;
-        out[1] |= keep_msb4(r.y, theta) >> blk;
-        out[2] |= keep_msb4(r.z, theta) >> blk;
-        out[3] |= keep_msb4(r.w, theta) >> blk;
+        out[0] |= keep_msb4<kHigh>(r.x, t7) >> blk;
+        out[1] |= keep_msb4<kHigh>(r.y, t7) >> blk;
+        out[2] |= keep_msb4<kHigh>(r.z, t7) >> blk;
+        out[3] |= keep_msb4<kHigh>(r.w, t7) >> blk;
     }
 }
 
 // Keep words of queries t0 .. t0+31 (t0 a multiple of 32) for the four keys
 // s0 .. s0+3 (s0 a multiple of 4): out[c] for key s0 + c, column i = query
-// t0 + i.  Eight generator calls, one per 4 x 4 block.
-__device__ __forceinline__ void dropout_keep32x4_keys(uint64_t seed, uint32_t theta, uint32_t bh, uint32_t s0,
+// t0 + i.  Eight generator calls, one per 4 x 4 block; each call's flags
+// (word q = query, byte c = key) are transposed to (word c, byte q).
+template <bool kHigh>
+__device__ __forceinline__ void dropout_keep32x4_keys(uint64_t seed, uint32_t t7, uint32_t bh, uint32_t s0,
                                                       uint32_t t0, uint32_t (&out)[4]) {
     out[0] = out[1] = out[2] = out[3] = 0u;
 #pragma unroll 2
     for (int blk = 0; blk < 8; ++blk) {
         const uint4 r = philox4x32_10(make_uint4(s0 >> 2, (t0 >> 2) + (uint32_t)blk, bh, 0u), (uint32_t)seed,
                                       (uint32_t)(seed >> 32));
-        // byte c of word q: (query 4*blk + q, key s0 + c); gather byte c of the four words
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint32_t sel = (uint32_t)c | ((4u + (uint32_t)c) << 4);
-            out[c] |= keep_msb4(__byte_perm(__byte_perm(r.x, r.y, sel), __byte_perm(r.z, r.w, sel), 0x5410), theta) >>
-                      blk;
-        }
+        const uint32_t m0 = keep_msb4<kHigh>(r.x, t7), m1 = keep_msb4<kHigh>(r.y, t7);
+        const uint32_t m2 = keep_msb4<kHigh>(r.z, t7), m3 = keep_msb4<kHigh>(r.w, t7);
+        // 4 x 4 byte transpose: interleave bytes of (m0, m1) and of (m2, m3), then halves
+        const uint32_t a = __byte_perm(m0, m1, 0x5140), b = __byte_perm(m0, m1, 0x7362);
+        const uint32_t c = __byte_perm(m2, m3, 0x5140), d = __byte_perm(m2, m3, 0x7362);
+        out[0] |= __byte_perm(a, c, 0x5410) >> blk;
+        out[1] |= __byte_perm(a, c, 0x7632) >> blk;
+        out[2] |= __byte_perm(b, d, 0x5410) >> blk;
+        out[3] |= __byte_perm(b, d, 0x7632) >> blk;
     }
 }
 

@@ -39,25 +39,29 @@ def test_dropout_bf16(B, T, n_head, p, window):
     compare(got, ref(qkv, dy, n_head, p, seed, window=window or None), torch.bfloat16, f"bf16 dropout {p} w {window}")
 
 
-def test_dropout_mask_bits_match_the_oracle_generator():
-    """Zero queries and v = identity expose every weight's dropout factor in y;
-    the kept set must equal the oracle generator's decision bit for bit."""
-    T, n_head, hs, p, seed = 64, 2, 64, 0.37, 0x0123456789ABCDEF
+@pytest.mark.parametrize("p", [0.37, 0.7])  # theta = 95 and 179: both sides of 128
+def test_dropout_mask_bits_match_the_oracle_generator(p):
+    """Zero queries and v = identity expose every weight's dropout factor in y
+    (forward); dy[t] = e_t exposes it in dV[s, t] = P[t, s] f[t, s] (backward).
+    Both kept sets must equal the oracle generator's decision bit for bit."""
+    T, n_head, hs, seed = 64, 2, 64, 0x0123456789ABCDEF
     C = n_head * hs
     qkv = torch.zeros(1, T, 3 * C)
     qkv[0, :, C:2 * C] = torch.randn(T, C, generator=torch.Generator().manual_seed(5))
+    dy = torch.zeros(1, T, C)
     for h in range(n_head):
         qkv[0, :, 2 * C + h * hs:2 * C + (h + 1) * hs] = torch.eye(T)
-    dy = torch.zeros(1, T, C)
+        dy[0, :, h * hs:(h + 1) * hs] = torch.eye(T)
+    thr = min(255, math.floor(256.0 * float(np.float32(p)) + 0.5))  # theta = round(256 p)
     for dtype in (torch.float32, torch.bfloat16):
-        y, _, _ = run_fwd_bwd(qkv.to(dtype), dy.to(dtype), n_head, opts=ga.Options(dropout_p=p, dropout_seed=seed))
-        thr = min(255, math.floor(256.0 * float(np.float32(p)) + 0.5))  # theta = round(256 p)
+        y, _, dqkv = run_fwd_bwd(qkv.to(dtype), dy.to(dtype), n_head, opts=ga.Options(dropout_p=p, dropout_seed=seed))
         for h in range(n_head):
             for t in range(T):
                 for s in range(t + 1):
                     r = oracle.philox([s // 4, t // 4, h, 0], [seed & 0xFFFFFFFF, seed >> 32])
                     kept = ((r[t % 4] >> (8 * (s % 4))) & 0xFF) >= thr
-                    assert kept == (y[0, t, h * hs + s] > 0), (str(dtype), h, t, s)
+                    assert kept == (y[0, t, h * hs + s] > 0), ("forward", str(dtype), h, t, s)
+                    assert kept == (dqkv[0, s, 2 * C + h * hs + t] > 0), ("backward", str(dtype), h, t, s)
 
 
 def test_dropout_zero_is_the_plain_path_and_seeds_matter():
