@@ -467,11 +467,21 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
                                                       float d_mul) {
     constexpr int kLanesPerRow = HS / 8;
     constexpr int kRowsPerPass = kPPThreads / kLanesPerRow;
-    griddep_launch_dependents();
-    griddep_wait();
     const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
     const int sub = threadIdx.x / kLanesPerRow, part = threadIdx.x % kLanesPerRow;
     const size_t row0 = (size_t)bh * T_pad + (size_t)blockIdx.y * kTile;
+    griddep_launch_dependents();
+    // The accumulator tile is zeroed before the wait for the previous kernel: no kernel of
+    // this library that may still run reads it (the postprocess kernels, its only readers,
+    // let their dependents start only after their reads), so the zeroing overlaps the
+    // previous kernel's tail.
+    if (zero_acc) {
+        float4 *acc = dqacc + row0 * (HS / 4);
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int i = threadIdx.x; i < kTile * HS / 4; i += kPPThreads) acc[i] = z;
+    }
+    griddep_wait();
 #pragma unroll
     for (int r = 0; r < kTile; r += kRowsPerPass) {
         const int t = blockIdx.y * kTile + r + sub;
@@ -494,11 +504,6 @@ __global__ void __launch_bounds__(kPPThreads) bwd_pre_kernel(const __nv_bfloat16
             lse2[row0 + r + sub] = t < T ? -lse[(size_t)bh * T + t] * 1.4426950408889634f + lse_bias : -INFINITY;
         }
     }
-    if (!zero_acc) return;
-    float4 *acc = dqacc + row0 * (HS / 4);
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int i = threadIdx.x; i < kTile * HS / 4; i += kPPThreads) acc[i] = z;
 }
 
 // postprocess: dq = bf16(dqacc * scale) into dqkv[..., 0:C].  Grid (B * n_head,
@@ -509,7 +514,6 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_kernel(const float *__res
                                                        int T, int C, int n_head, int T_pad) {
     constexpr int kPerRow = HS / 8;
     const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
-    griddep_launch_dependents();
     griddep_wait();
     const int bh = blockIdx.x, b = bh / n_head, h = bh % n_head;
     const int t0 = blockIdx.y * kTile;
@@ -528,6 +532,9 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_kernel(const float *__res
             *reinterpret_cast<uint4 *>(dst + (size_t)r * (size_t)(3 * C) + (size_t)k * 8) = o;
         }
     }
+    // dependents may start only now: the next call's preprocess zeroes this accumulator
+    // before it waits for this kernel
+    griddep_launch_dependents();
 }
 
 // deterministic postprocess: dq = bf16(scale * sum over key tiles j of partial(i, j)),
@@ -538,7 +545,6 @@ template <int HS>
 __global__ void __launch_bounds__(kPPThreads) bwd_post_det_kernel(const float *__restrict__ part,
                                                            __nv_bfloat16 *__restrict__ dqkv, int T, int C, int n_head,
                                                            int n_slots, int window) {
-    griddep_launch_dependents();
     griddep_wait();
     constexpr int kPerRow = HS / 8;
     const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
@@ -566,6 +572,7 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_det_kernel(const float *_
         o.w = pack_bf16x2(acc[6] * scale, acc[7] * scale);
         *reinterpret_cast<uint4 *>(dst + (size_t)r * (size_t)(3 * C) + (size_t)k * 8) = o;
     }
+    griddep_launch_dependents();  // after the reads of the workspace, as in bwd_post_kernel
 }
 
 template <int HS>
