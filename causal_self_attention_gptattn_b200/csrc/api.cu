@@ -296,9 +296,8 @@ gptattn_status check_window(int window, int T, int hs, gptattn_dtype dt, int *ke
     return GPTATTN_OK;
 }
 
-// Dropout probability -> kernel parameters (threshold floor(p * 2^32); a p so small
-// that the threshold is 0 drops nothing).  p must be in [0, 1); a bf16 dropout needs
-// the head-size-64 kernels.
+// Dropout probability -> kernel parameters (threshold theta = round(256 p), at most
+// 255; a p so small that theta is 0 drops nothing).  p must be in [0, 1).
 gptattn_status make_dropout(float p, unsigned long long seed, int hs, gptattn_dtype dt, DropoutParams *dp) {
     if (!(p >= 0.f && p < 1.f)) return GPTATTN_ERR_INVALID_ARG;
     // p in steps of 1/256: theta = round(256 p), at most 255; drop probability theta/256
@@ -306,7 +305,6 @@ gptattn_status make_dropout(float p, unsigned long long seed, int hs, gptattn_dt
     dp->seed = seed;
     dp->threshold = x >= 255.0 ? 255u : (uint32_t)x;
     dp->scale = dp->threshold ? (float)(1.0 / (1.0 - dp->threshold / 256.0)) : 1.f;
-    if (dp->threshold && dt == GPTATTN_BF16 && hs != 64) return GPTATTN_ERR_UNSUPPORTED;
     return GPTATTN_OK;
 }
 

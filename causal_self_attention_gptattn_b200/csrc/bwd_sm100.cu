@@ -24,11 +24,17 @@
 // stored in a slot of its own and the postprocess sums a query tile's slots in
 // a fixed order, so the result does not depend on the order CTAs finish in.
 //
-// Main-kernel roles (10 warps):
+// Main-kernel roles (10 warps; 12 with dropout):
 //   warp 0      TMA producer (K, V once; Q_i, dO_i, lse_i, D_i per iteration)
 //   warp 1      TMEM owner + MMA issuer
 //   warps 2..5  "softmax" warps, one key row each: P, dS, final dK/dV epilogue
 //   warps 6..9  dQ drain warps, one query row each: TMEM -> smem -> TMA reduce
+//   warps 10,11 with dropout: the keep words of each (key tile, query tile),
+//               drawn a few tiles ahead into a shared-memory ring
+// Dropout (inverted, Philox mask of philox.cuh): the preprocess folds the
+// scale 1/(1-p) into lse and D, so the recomputed weights are P * scale; P^T
+// goes to the dV product with dropped weights zeroed, and
+// dS = (P scale) o (dP o keep - D / scale).
 // TMEM columns: S^T [0,128) (P^T packed into [0,64)), dP^T [128,256),
 // dV [256,256+hs), dK [256+hs, 256+2hs).  dQ: hs=64 at [384,448); hs=128 in
 // two 64-column halves at [64,128) and [192,256), the parts of S^T / dP^T that
@@ -39,12 +45,16 @@
 namespace gptattn {
 namespace {
 
-constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlabBytes = 128 * 128;
+// dropout keep words: kMStages tiles of 128 key rows x 128 query columns (16 bytes a row)
+constexpr int kMStages = 4;
+constexpr uint32_t kMaskTileBytes = 128u * 16u;
+constexpr int kMaskThreads = 64;
 
-template <int HS>
+template <int HS, bool kDropout = false>
 struct BwdCfg {
+    static constexpr int kThreads = kDropout ? 320 + kMaskThreads : 320;
     static constexpr int kSlabs = HS / 64;
     static constexpr uint32_t kTileBytes = 128u * HS * 2u;
     static constexpr int kStages = (HS == 64) ? 2 : 1;
@@ -57,7 +67,8 @@ struct BwdCfg {
     static constexpr uint32_t kOffLse = kOffdQ + 2 * kSlabBytes;         // kStages x 128 fp32
     static constexpr uint32_t kOffD = kOffLse + kStages * 512;
     static constexpr uint32_t kOffBar = kOffD + kStages * 512;
-    static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;
+    static constexpr uint32_t kOffM = kOffBar + 256;
+    static constexpr uint32_t kSmemBytes = kOffM + (kDropout ? kMStages * kMaskTileBytes : 0u) + 1024;
     static constexpr uint32_t kColS = 0, kColdP = 128, kColdV = 256, kColdK = 256 + HS;
     static constexpr uint32_t kColdQ0 = (HS == 64) ? 384 : 64;
     static constexpr uint32_t kColdQ1 = 192;  // second half, hs = 128 only
@@ -74,7 +85,9 @@ struct BwdCfg {
     static constexpr int kBardQEmpty = kBardQFull + 1;
     static constexpr int kBarKdV = kBardQEmpty + 1;
     static constexpr int kBarDone = kBarKdV + 1;
-    static constexpr int kNumBars = kBarDone + 1;
+    static constexpr int kBarMFull = kBarDone + 1;          // kMStages
+    static constexpr int kBarMEmpty = kBarMFull + kMStages;  // kMStages
+    static constexpr int kNumBars = kBarMEmpty + kMStages;
     static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -93,13 +106,14 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 
 // kBand: a local window narrower than T (shorter query range, far-edge mask); the
 // causal instantiation compiles none of it.
-template <int HS, bool kBand>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int HS, bool kBand, bool kDropout>
+__global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
     bwd_bf16_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_dy,
                     const __grid_constant__ CUtensorMap map_dqkv, const __grid_constant__ CUtensorMap map_dq,
                     const float *__restrict__ lse2, const float *__restrict__ Dvec, int B, int T, int C, int n_head,
-                    int T_pad, int n_t, int window, int n_slots, int *status, unsigned long long budget_ns) {
-    using K = BwdCfg<HS>;
+                    int T_pad, int n_t, int window, int n_slots, DropoutParams dp, int *status,
+                    unsigned long long budget_ns) {
+    using K = BwdCfg<HS, kDropout>;
     if constexpr (!kBand) window = 1 << 30;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -129,9 +143,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sdS = sbase + K::kOffdS, sdQ = sbase + K::kOffdQ;
     const float *sLse = reinterpret_cast<const float *>(smem + K::kOffLse);
     const float *sD = reinterpret_cast<const float *>(smem + K::kOffD);
+    const uint32_t sM = sbase + K::kOffM;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(K::kBarKV), 1);
+        for (int s = 0; s < kMStages; ++s) {
+            mbar_init(bar(K::kBarMFull + s), kMaskThreads);
+            mbar_init(bar(K::kBarMEmpty + s), 128);
+        }
         for (int s = 0; s < K::kStages; ++s) {
             mbar_init(bar(K::kBarFull + s), 1);
             mbar_init(bar(K::kBarEmpty + s), 1);
@@ -276,6 +295,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < niter; ++it) {
             const int st = it % K::kStages;
             const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
+            // dropout keep words of this key row's 128 query columns (bit layout of philox.cuh)
+            uint32_t kb[4] = {0u, 0u, 0u, 0u};
+            if constexpr (kDropout) {
+                const int ms = it % kMStages;
+                if (!(ok = warp_wait(bar(K::kBarMFull + ms), (uint32_t)(it / kMStages) & 1u, g))) break;
+                const uint4 v = ld_shared_v4(sM + (uint32_t)ms * kMaskTileBytes + (uint32_t)row * 16u);
+                kb[0] = v.x;
+                kb[1] = v.y;
+                kb[2] = v.z;
+                kb[3] = v.w;
+                mbar_arrive(bar(K::kBarMEmpty + ms));
+            }
             ok = warp_wait(bar(K::kBarFull + st), ph, g) && warp_wait(bar(K::kBarS), (uint32_t)it & 1u, g);
             if (!ok) break;
             tc_fence_after();
@@ -302,8 +333,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     pk[c >> 1] = pack_bf16x2(p0, p1);
                 }
-                // columns [16ch, 16ch+16) were read in an earlier (or this) chunk
-                tmem_st_x16(trow + K::kColS + 16 * ch, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * ch]));
+                // columns [16ch, 16ch+16) were read in an earlier (or this) chunk; with dropout the
+                // dV product gets the dropped weights zeroed, dS below the undropped ones
+                if constexpr (kDropout) {
+                    uint32_t pm[16];
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) pm[q] = pk[16 * ch + q] & keep_pair_mask(kb[ch] << (q >> 1), q & 1);
+                    tmem_st_x16(trow + K::kColS + 16 * ch, pm);
+                } else {
+                    tmem_st_x16(trow + K::kColS + 16 * ch, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * ch]));
+                }
             }
             tmem_st_wait();
             tc_fence_before();
@@ -317,6 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int ch = 0; ch < 4; ++ch) {
                 uint32_t dr[32];
                 tmem_ld_x32(trow + K::kColdP + 32 * ch, dr);
+                if constexpr (kDropout) {  // dropped columns: dP^T o keep = 0
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) dr[e] &= keep_word_mask(kb[ch] << (e >> 2), e & 3);
+                }
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -378,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit_group();
             bulk_wait_group_0();
         }
-    } else {
+    } else if (warp < 10) {
         // ------------------------------------------------------------ dQ drain warps (query rows)
         const int sp = warp & 3;
         const int row = sp * 32 + lane;
@@ -432,6 +475,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (leader) bulk_wait_group_0();
+    } else {
+        // ------------------------------------------------------------ dropout keep words (warps 10, 11)
+        if constexpr (kDropout) {
+            // thread -> key rows 4*kg .. 4*kg+3 and query columns 64*qh .. 64*qh+63 of every tile
+            const int u = threadIdx.x - 320, kg = u >> 1, qh = u & 1;
+            const uint32_t t7 = theta_low7(dp.threshold);
+            const uint32_t s0 = (uint32_t)(kt * kTile + 4 * kg);
+            for (int it = 0; it < niter; ++it) {
+                const int ms = it % kMStages;
+                if (it >= kMStages && !warp_wait(bar(K::kBarMEmpty + ms), (uint32_t)((it / kMStages) & 1) ^ 1u, g))
+                    break;
+                const uint32_t t0 = (uint32_t)((kt + it) * kTile + 64 * qh);
+                uint32_t lo[4], hi[4];
+                if (dp.threshold >= 128u) {
+                    dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
+                    dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
+                } else {
+                    dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
+                    dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
+                }
+                const uint32_t dst = sM + (uint32_t)ms * kMaskTileBytes + (uint32_t)(4 * kg) * 16u + (uint32_t)qh * 8u;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) st_shared_v2(dst + (uint32_t)c * 16u, lo[c], hi[c]);
+                mbar_arrive(bar(K::kBarMFull + ms));
+            }
+        }
     }
 
     tc_fence_before();
@@ -575,18 +644,36 @@ __global__ void __launch_bounds__(kPPThreads) bwd_post_det_kernel(const float *_
     griddep_launch_dependents();  // after the reads of the workspace, as in bwd_post_kernel
 }
 
-template <int HS>
-cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
-                             const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
-                             int n_head, int T_pad, int window, int n_slots, DevCtx ctx, cudaStream_t s) {
-    using K = BwdCfg<HS>;
-    auto kern = window < T ? bwd_bf16_kernel<HS, true> : bwd_bf16_kernel<HS, false>;
+template <int HS, bool kBand, bool kDropout>
+cudaError_t launch_main_variant(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
+                                const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
+                                int n_head, int T_pad, int window, int n_slots, DropoutParams dp, DevCtx ctx,
+                                cudaStream_t s) {
+    using K = BwdCfg<HS, kDropout>;
+    auto kern = bwd_bf16_kernel<HS, kBand, kDropout>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int n_t = ceil_div(T, kTile);
     const long long blocks = (long long)n_t * B * n_head;
-    return launch_pdl(kern, dim3((unsigned)blocks), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_dy, map_dqkv, map_dq,
-                      lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, ctx.status, ctx.budget_ns);
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(K::kThreads), K::kSmemBytes, s, map_qkv, map_dy, map_dqkv,
+                      map_dq, lse2, D, B, T, C, n_head, T_pad, n_t, window, n_slots, dp, ctx.status, ctx.budget_ns);
+}
+
+template <int HS>
+cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_dy, const CUtensorMap &map_dqkv,
+                             const CUtensorMap &map_dq, const float *lse2, const float *D, int B, int T, int C,
+                             int n_head, int T_pad, int window, int n_slots, DropoutParams dp, DevCtx ctx,
+                             cudaStream_t s) {
+    const bool band = window < T, drop = dp.threshold != 0u;
+    if (band)
+        return drop ? launch_main_variant<HS, true, true>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
+                                                          T_pad, window, n_slots, dp, ctx, s)
+                    : launch_main_variant<HS, true, false>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
+                                                           T_pad, window, n_slots, dp, ctx, s);
+    return drop ? launch_main_variant<HS, false, true>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
+                                                       T_pad, window, n_slots, dp, ctx, s)
+                : launch_main_variant<HS, false, false>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
+                                                        T_pad, window, n_slots, dp, ctx, s);
 }
 
 }  // namespace
@@ -615,9 +702,9 @@ cudaError_t launch_bwd_main_bf16(int hs, const CUtensorMap &map_qkv, const CUten
     if (hs == 64)
         return launch_bwd_main_h64(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots,
                                    dp, ctx, s);
-    if (hs == 128 && dp.threshold == 0u)
+    if (hs == 128)
         return launch_main_impl<128>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots,
-                                     ctx, s);
+                                     dp, ctx, s);
     return cudaErrorInvalidValue;
 }
 

@@ -31,14 +31,19 @@
 // Every barrier wait is bounded; on a timeout all roles stop, drain and exit.
 #include <type_traits>
 
+#include "fwd_common.cuh"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
 namespace gptattn {
 namespace {
 
-constexpr int kMStages = 4;  // dropout mask ring, per query-tile stream
-constexpr uint32_t kMaskTileBytes = 128u * 16u;  // 128 query rows x 128 keep bits
+using fwdc::band_lo_tile;
+using fwdc::drain_wait;
+using fwdc::item_index;
+using fwdc::kMaskRingBytes;
+using fwdc::kMStages;
+using fwdc::warp_wait;
 
 // Threads and register budgets per thread.  The plain kernel has three
 // warpgroups (control, two softmax); with dropout a fourth draws the keep bits
@@ -51,7 +56,7 @@ struct FwdCfg {
     static constexpr uint32_t kRegsCtl = kDropout ? 80 : 88;
     static constexpr uint32_t kRegsSoftmax = kDropout ? 192 : 208;
     static constexpr uint32_t kRegsMask = kDropout ? 48 : 0;
-    static constexpr uint32_t kMaskBytes = kDropout ? 2u * kMStages * kMaskTileBytes : 0u;
+    static constexpr uint32_t kMaskBytes = kDropout ? kMaskRingBytes : 0u;
     static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsMask == (kThreads / 128) * kLaunchRegs, "register split");
 };
 constexpr uint32_t kTmemCols = 512;
@@ -87,27 +92,6 @@ constexpr int kBarMEmpty = kBarMFull + 2 * kMStages;  // 2 x kMStages
 constexpr int kNumBars = kBarMEmpty + 2 * kMStages;
 static_assert(kNumBars * 8 + 16 <= kBarArea, "barrier area");
 
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitGuard &g) {
-    bool ok = mbar_wait(bar, parity, g);
-    return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > budget_ns) break;
-    }
-}
-
-// First key tile that query tile qt's band reaches.
-__device__ __forceinline__ int band_lo_tile(int qt, int window) {
-    const int s = qt * kTile - window + 1;
-    return s > 0 ? s / kTile : 0;
-}
-
-__device__ __forceinline__ int item_index(int k, int cta, int grid) {
-    return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
-}
 
 template <bool kDropout>
 __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
@@ -137,11 +121,7 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
     auto sQ = [&](int qs, int t) -> uint32_t { return sbase + kOffQ + (uint32_t)(2 * qs + t) * kTileBytes; };
     auto sK = [&](int st) -> uint32_t { return sbase + kOffK + (uint32_t)st * kTileBytes; };
     auto sV = [&](int st) -> uint32_t { return sbase + kOffV + (uint32_t)st * kTileBytes; };
-    auto sM = [&](int t, int st) -> uint32_t { return sbase + kOffM + (uint32_t)(t * kMStages + st) * kMaskTileBytes; };
-    auto decode = [&](int w, int &m, int &bh) {
-        m = n_pairs - 1 - w / BH;
-        bh = w % BH;
-    };
+    auto decode = [&](int w, int &m, int &bh) { fwdc::decode_item(w, n_pairs, BH, m, bh); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kQStages; ++s) {
@@ -352,15 +332,8 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
                 // j*128 + c), drawn ahead by the mask warpgroup; tile number `it` of this stream
                 uint32_t kb[4] = {0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu};
                 if constexpr (kDropout) {
-                    const int ms = it % kMStages;
-                    if (ok) ok = warp_wait(bar(kBarMFull + t * kMStages + ms), (uint32_t)(it / kMStages) & 1u, g);
+                    if (ok) ok = fwdc::mask_take(sbase + kOffM, bar(kBarMFull), bar(kBarMEmpty), t, it, row, g, kb);
                     if (!ok) continue;
-                    const uint4 v = ld_shared_v4(sM(t, ms) + (uint32_t)row * 16u);
-                    kb[0] = v.x;
-                    kb[1] = v.y;
-                    kb[2] = v.z;
-                    kb[3] = v.w;
-                    mbar_arrive(bar(kBarMEmpty + t * kMStages + ms));
                 }
                 if (ok) ok = warp_wait(bar(kBarSFull + t), (uint32_t)it & 1u, g);
                 if (!ok) continue;
@@ -502,43 +475,8 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
         // ================================================================ dropout mask warpgroup
         if constexpr (kDropout) {
             regs_dec<Cfg::kRegsMask>();
-            // thread -> rows 4*rg .. 4*rg+3 and keys 32*kq .. 32*kq+31 of every mask tile;
-            // tiles in the order the softmax warpgroups use them (key tile by key tile,
-            // stream A before stream B), each stream through its own ring
-            const int rg = (warp & 3) * 8 + (lane >> 2), kq = lane & 3;
-            const uint32_t t7 = theta_low7(dp.threshold);
-            bool ok = true;
-            int mc[2] = {0, 0};
-            for (int k = 0; ok; ++k) {
-                const int w = item_index(k, cta, grid);
-                if (w >= n_items) break;
-                int m, bh;
-                decode(w, m, bh);
-                const bool hasB = 2 * m + 1 < n_qt;
-                const int lo[2] = {band_lo_tile(2 * m, window), hasB ? band_lo_tile(2 * m + 1, window) : 1};
-                const int hi[2] = {2 * m, hasB ? 2 * m + 1 : 0};
-                for (int j = lo[0]; j <= hi[1] || j <= hi[0]; ++j) {
-                    for (int t = 0; t < 2; ++t) {
-                        if (j < lo[t] || j > hi[t]) continue;
-                        const int ms = mc[t] % kMStages;
-                        if (mc[t] >= kMStages &&
-                            !(ok = warp_wait(bar(kBarMEmpty + t * kMStages + ms), (uint32_t)((mc[t] / kMStages) & 1) ^ 1u, g)))
-                            break;
-                        uint32_t bits[4];
-                        const uint32_t t0 = (uint32_t)((2 * m + t) * kTile + 4 * rg), s0 = (uint32_t)(j * kTile + 32 * kq);
-                        if (dp.threshold >= 128u)
-                            dropout_keep32x4<true>(dp.seed, t7, (uint32_t)bh, t0, s0, bits);
-                        else
-                            dropout_keep32x4<false>(dp.seed, t7, (uint32_t)bh, t0, s0, bits);
-                        const uint32_t dst = sM(t, ms) + (uint32_t)(4 * rg) * 16u + (uint32_t)kq * 4u;
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) st_shared_u32(dst + (uint32_t)r * 16u, bits[r]);
-                        mbar_arrive(bar(kBarMFull + t * kMStages + ms));
-                        ++mc[t];
-                    }
-                    if (!ok) break;
-                }
-            }
+            fwdc::mask_producer(dp, sbase + kOffM, bar(kBarMFull), bar(kBarMEmpty), n_items, n_pairs, BH, n_qt, window,
+                                cta, grid, g);
         }
     }
 

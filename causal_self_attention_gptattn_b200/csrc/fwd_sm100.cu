@@ -29,21 +29,39 @@
 // The softmax keeps the running max lazily (rescaling O only when the max
 // grows by more than 2^8) and normalises y by the sum of the bf16-rounded
 // weights that the P V product used; lse uses the sum of the fp32 weights.
+// Dropout (lecture chapter "adding dropout", read as inverted dropout on the
+// weights): P goes into TMEM with dropped weights zeroed, l and the rounded-
+// weight sum stay those of the undropped weights, and the epilogue scales y by
+// 1/(1-p).  The keep words come from a fourth warpgroup that draws them a few
+// tiles ahead (fwd_common.cuh); the dropout instantiation therefore places the
+// roles in whole warpgroups (warps 0-3: producer, MMA issuer, two idle; 4-11:
+// softmax; 12-15: mask) and moves registers to the softmax warps with setmaxnreg.
 // Every barrier wait is bounded (sm100_ptx.cuh); on a timeout all roles stop
 // issuing work, drain and exit.
+#include "fwd_common.cuh"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
-
 
 namespace gptattn {
 namespace {
 
-constexpr int kThreads = 320;
+using fwdc::band_lo_tile;
+using fwdc::drain_wait;
+using fwdc::item_index;
+using fwdc::warp_wait;
+
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlabBytes = 128 * 128;  // 128 rows x 128 bytes (64 bf16 columns), one swizzle slab
 
-template <int HS>
+template <int HS, bool kDropout>
 struct FwdCfg {
+    // warp 0 producer, warp 1 MMA issuer, eight softmax warps from kSoftBase on; with
+    // dropout, warps 12-15 draw the mask and registers move by setmaxnreg (launch: 128)
+    static constexpr int kThreads = kDropout ? 512 : 320;
+    static constexpr int kSoftBase = kDropout ? 4 : 2;
+    static constexpr int kLaunchRegs = 128;
+    static constexpr uint32_t kRegsCtl = 96, kRegsSoftmax = 192, kRegsMask = 32;
+    static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsMask == 4 * kLaunchRegs, "register split");
     static constexpr int kSlabs = HS / 64;
     static constexpr uint32_t kTileBytes = 128u * HS * 2u;
     static constexpr int kQStages = (HS == 64) ? 2 : 1;   // pairs of Q tiles
@@ -52,7 +70,10 @@ struct FwdCfg {
     static constexpr uint32_t kOffK = kOffQ + kQStages * 2 * kTileBytes;     // kKVStages tiles
     static constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;        // kKVStages tiles
     static constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
-    static constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;             // + slack for 1024-byte alignment
+    static constexpr uint32_t kBarArea = 512;
+    static constexpr uint32_t kOffM = kOffBar + kBarArea;                     // dropout keep-word rings
+    static constexpr uint32_t kSmemBytes =
+        kOffM + (kDropout ? fwdc::kMaskRingBytes : 0u) + 1024;                // + slack for 1024-byte alignment
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
     static constexpr uint32_t kColS = 0;    // + 128 * tile
     static constexpr uint32_t kColO = 256;  // + HS * tile
@@ -67,43 +88,20 @@ struct FwdCfg {
     static constexpr int kBarODone = kBarPFull + 2;            // 2
     static constexpr int kBarOFree = kBarODone + 2;            // 2
     static constexpr int kBarDone = kBarOFree + 2;
-    static constexpr int kNumBars = kBarDone + 1;
-    static_assert(kNumBars * 8 + 16 <= 256, "barrier area");
+    static constexpr int kBarMFull = kBarDone + 1;                     // 2 x fwdc::kMStages
+    static constexpr int kBarMEmpty = kBarMFull + 2 * fwdc::kMStages;  // 2 x fwdc::kMStages
+    static constexpr int kNumBars = kBarMEmpty + 2 * fwdc::kMStages;
+    static_assert(kNumBars * 8 + 16 <= kBarArea, "barrier area");
 };
-
-// Warp-uniform bounded wait (all 32 lanes call it; all get the same answer).
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitGuard &g) {
-    bool ok = mbar_wait(bar, parity, g);
-    return __all_sync(0xffffffffu, ok);
-}
-
-// Wait used only while draining after an abort: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t budget_ns) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > budget_ns) break;
-    }
-}
-
-// Item k of this CTA in the snake walk over items sorted longest first.
-__device__ __forceinline__ int item_index(int k, int cta, int grid) {
-    return (k & 1) ? (k * grid + (grid - 1 - cta)) : (k * grid + cta);
-}
-
-// First key tile that query tile qt's band reaches.
-__device__ __forceinline__ int band_lo_tile(int qt, int window) {
-    const int s = qt * kTile - window + 1;
-    return s > 0 ? s / kTile : 0;
-}
 
 // kBand: a local window narrower than T (key-tile ranges and edge masks); the causal
 // instantiation compiles none of it.
-template <int HS, bool kBand>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int HS, bool kBand, bool kDropout>
+__global__ void __launch_bounds__(FwdCfg<HS, kDropout>::kThreads, 1)
     fwd_bf16_kernel(const __grid_constant__ CUtensorMap map_qkv, const __grid_constant__ CUtensorMap map_y,
-                    float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, int *status,
-                    unsigned long long budget_ns) {
-    using K = FwdCfg<HS>;
+                    float *__restrict__ lse, int B, int T, int C, int n_head, int n_qt, int window, DropoutParams dp,
+                    int *status, unsigned long long budget_ns) {
+    using K = FwdCfg<HS, kDropout>;
     if constexpr (!kBand) window = 1 << 30;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
@@ -128,10 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto sV = [&](int st) -> uint32_t { return sbase + K::kOffV + (uint32_t)st * K::kTileBytes; };
 
     // item -> (pair m, batch*head); pairs with the most key tiles first
-    auto decode = [&](int w, int &m, int &bh) {
-        m = n_pairs - 1 - w / BH;
-        bh = w % BH;
-    };
+    auto decode = [&](int w, int &m, int &bh) { fwdc::decode_item(w, n_pairs, BH, m, bh); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < K::kQStages; ++s) {
@@ -148,6 +143,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(K::kBarPFull + t), 128);
             mbar_init(bar(K::kBarODone + t), 1);
             mbar_init(bar(K::kBarOFree + t), 128);
+            for (int st = 0; st < fwdc::kMStages; ++st) {
+                mbar_init(bar(K::kBarMFull + t * fwdc::kMStages + st), 128);
+                mbar_init(bar(K::kBarMEmpty + t * fwdc::kMStages + st), 128);
+            }
         }
         mbar_init(bar(K::kBarDone), 1);
         *abort_flag = 0;
@@ -164,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     griddep_launch_dependents();
     griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
+    if (warp < K::kSoftBase) {
+        if constexpr (kDropout) regs_dec<K::kRegsCtl>();
     if (warp == 0) {
         // ================================================================ producer
         if (lane == 0) {
@@ -308,9 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 drain_wait(bar(K::kBarDone), 0, budget_ns);
             }
         }
-    } else {
+    }
+    } else if (warp < K::kSoftBase + 8) {
         // ================================================================ softmax warpgroups
-        const int t = (warp - 2) >> 2;           // tile stream: 0 = A, 1 = B
+        if constexpr (kDropout) regs_inc<K::kRegsSoftmax>();
+        const int t = (warp - K::kSoftBase) >> 2;  // tile stream: 0 = A, 1 = B
         const int sp = warp & 3;                 // TMEM sub-partition this warp may access
         const int row = sp * 32 + lane;          // query row within the tile
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
@@ -343,6 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             float l = 0.f;           // running normaliser of the fp32 weights
             float l_r = 0.f;         // running normaliser of the bf16-rounded weights
             for (int j = jlo_t; j <= qt; ++j, ++it) {
+                // dropout keep words of this row's 128 keys of tile j (bit layout of philox.cuh)
+                uint32_t kb[4] = {0u, 0u, 0u, 0u};
+                if constexpr (kDropout) {
+                    if (ok) ok = fwdc::mask_take(sbase + K::kOffM, bar(K::kBarMFull), bar(K::kBarMEmpty), t, it, row, g, kb);
+                    if (!ok) continue;
+                }
                 if (ok) ok = warp_wait(bar(K::kBarSFull + t), (uint32_t)it & 1u, g);
                 if (!ok) continue;
                 tc_fence_after();
@@ -402,7 +411,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         f32x2_unpack(x, x0, x1);
                         const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
                         const uint32_t wv = pack_bf16x2(p0, p1);
-                        pk[c >> 1] = wv;
+                        // with dropout the stored weights are masked, the sums are not
+                        if constexpr (kDropout)
+                            pk[c >> 1] = wv & keep_pair_mask(kb[ch] << (c >> 2), (c >> 1) & 1);
+                        else
+                            pk[c >> 1] = wv;
                         sum2 = fadd2(sum2, f32x2_pack(p0, p1));
                         sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
                     }
@@ -439,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok) ok = warp_wait(bar(K::kBarODone + t), (uint32_t)(it - 1) & 1u, g);
             if (ok) {
                 tc_fence_after();
-                const float inv_l = 1.f / l_r;
+                const float inv_l = (kDropout ? dp.scale : 1.f) / l_r;  // 1/(1-p) with dropout
 #pragma unroll
                 for (int c0 = 0; c0 < HS; c0 += 32) {
                     uint32_t o[32];
@@ -476,6 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (leader) bulk_wait_group_0();
+    } else {
+        // ================================================================ dropout mask warpgroup
+        if constexpr (kDropout) {
+            regs_dec<K::kRegsMask>();
+            fwdc::mask_producer(dp, sbase + K::kOffM, bar(K::kBarMFull), bar(K::kBarMEmpty), n_items, n_pairs, BH, n_qt,
+                                window, cta, grid, g);
+        }
     }
 
     tc_fence_before();
@@ -486,13 +506,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int HS>
-cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
-                            int n_head, int window, DevCtx ctx, cudaStream_t s) {
-    using K = FwdCfg<HS>;
-    auto kern = window < T ? fwd_bf16_kernel<HS, true> : fwd_bf16_kernel<HS, false>;
+template <int HS, bool kBand, bool kDropout>
+cudaError_t launch_fwd_variant(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
+                               int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
+    using K = FwdCfg<HS, kDropout>;
+    auto kern = fwd_bf16_kernel<HS, kBand, kDropout>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
+    if constexpr (kDropout) {
+        // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs
+        // per thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
+        cudaFuncAttributes fa{};
+        e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != K::kLaunchRegs) return cudaErrorInvalidConfiguration;
+    }
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -500,8 +528,19 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
     const int n_qt = ceil_div(T, kTile);
     const long long items = (long long)((n_qt + 1) / 2) * B * n_head;
     const int grid = (int)(items < sms ? items : sms);
-    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), K::kSmemBytes, s, map_qkv, map_y, lse, B, T, C, n_head,
-                      n_qt, window, ctx.status, ctx.budget_ns);
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(K::kThreads), K::kSmemBytes, s, map_qkv, map_y, lse, B, T, C,
+                      n_head, n_qt, window, dp, ctx.status, ctx.budget_ns);
+}
+
+template <int HS>
+cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T, int C,
+                            int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
+    const bool band = window < T, drop = dp.threshold != 0u;
+    if (band)
+        return drop ? launch_fwd_variant<HS, true, true>(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s)
+                    : launch_fwd_variant<HS, true, false>(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s);
+    return drop ? launch_fwd_variant<HS, false, true>(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s)
+                : launch_fwd_variant<HS, false, false>(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s);
 }
 
 }  // namespace
@@ -509,7 +548,7 @@ cudaError_t launch_fwd_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_y
 cudaError_t launch_fwd_bf16(int hs, const CUtensorMap &map_qkv, const CUtensorMap &map_y, float *lse, int B, int T,
                             int C, int n_head, int window, DropoutParams dp, DevCtx ctx, cudaStream_t s) {
     if (hs == 64) return launch_fwd_h64(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s);
-    if (hs == 128 && dp.threshold == 0u) return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, window, ctx, s);
+    if (hs == 128) return launch_fwd_impl<128>(map_qkv, map_y, lse, B, T, C, n_head, window, dp, ctx, s);
     return cudaErrorInvalidValue;
 }
 

@@ -139,8 +139,7 @@ GPTATTN_API gptattn_status gptattn_bwd_det(const void *qkv, const void *y, const
  *                 counter (s/4, t/4, b*n_head+h, 0) under key (seed & 0xffffffff,
  *                 seed >> 32); weight (t, s) is kept iff byte s%4 (least
  *                 significant first) of output word t%4 is >= theta.  The backward
- *                 must get the forward's seed and p.  bf16 dropout needs head size
- *                 64.
+ *                 must get the forward's seed and p.
  *   dropout_seed  the 64-bit Philox key.
  *   deterministic backward only: bit-identical results as gptattn_bwd_det (and
  *                 its workspace size). */
