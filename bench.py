@@ -49,6 +49,8 @@ def parse_args():
     p.add_argument("--skip-cpu-baseline", action="store_true")
     p.add_argument("--profile-run", action="store_true",
                    help="warm-up and timed steps only (no clock sampling, e2e or CPU leg): for ncu captures")
+    p.add_argument("--dropout-run", action="store_true",
+                   help="warm-up and timed fwd+bwd steps with attention dropout p = 0.1 only: for ncu captures")
     p.add_argument("--block-run", action="store_true",
                    help="only the attention sub-block call, warm-up + steps times: for ncu captures of its kernels")
     return p.parse_args()
@@ -59,9 +61,9 @@ def parse_args():
 # only while the sources it was taken on are unchanged (sha256 over the files).
 MEASURED_TRAFFIC = {
     ("bwd_bf16_sm100", "gpt2_124m"): {
-        "bytes": 197.432064e6 + 80.436480e6,
+        "bytes": 195.355648e6 + 79.649792e6,
         "sources": ("bwd_h64_sm100.cu", "sm100_ptx.cuh", "kernels.h"),
-        "sha256": "ed096c12a99349b8ca9175cfb8877050559a9cf5fa3632b977ed7156930b5488",
+        "sha256": "a5f1022c355b3c73e1002df88e4693f60a56d00f4be3904dc3aecc123cefef23",
         "capture": "profiles/bwd_h64_persistent_gpt2_124m.md",
     },
 }
@@ -367,6 +369,22 @@ def run_ours(args, w, rank, world, local_rank):
             print(json.dumps({"block_run": "ok", "calls": args.warmup + args.steps}), flush=True)
         return
 
+    if args.dropout_run:
+        o = ga.Options(dropout_p=0.1, dropout_seed=1234)
+        nb_o = ga.gptattn_bwd_opts_workspace_bytes(B, T, C, nh, o, dt)
+        ws_o = torch.empty(max(nb_o, 256), dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup + args.steps):
+            flush.zero_()
+            ga.check(ga.gptattn_fwd_opts(qkv, y, lse, B, T, C, nh, o, dt, s), "gptattn_fwd_opts")
+            ga.check(ga.gptattn_bwd_opts(qkv, y, lse, dy, dqkv, ws_o, nb_o, B, T, C, nh, o, dt, s), "gptattn_bwd_opts")
+        torch.cuda.synchronize()
+        ga.check(ga.gptattn_get_device_status(s), "device status after the dropout steps")
+        if dist is not None:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"dropout_run": "ok", "steps": args.warmup + args.steps}), flush=True)
+        return
+
     def step(q=qkv, g=dy):
         ga.check(ga.gptattn_fwd(q, y, lse, B, T, C, nh, dt, s), "gptattn_fwd")
         ga.check(ga.gptattn_bwd(q, y, lse, g, dqkv, ws, nbytes, B, T, C, nh, dt, s), "gptattn_bwd")
@@ -525,7 +543,7 @@ def run_ours(args, w, rank, world, local_rank):
     # with only the band's key tiles; FLOPs counted over the visible (query, key) pairs,
     # 14 * hs per pair (4 fwd + 10 bwd), which is the causal count 7*B*nh*T^2*hs for a full band.
     banded = None
-    if not args.profile_run and (dt == ga.GPTATTN_F32 or w.hs == 64):
+    if not args.profile_run:
         W = 256
         pairs = sum(min(t + 1, W) for t in range(T))
         flops_w = 14.0 * w.hs * B * nh * pairs
@@ -559,7 +577,7 @@ def run_ours(args, w, rank, world, local_rank):
     # ---- deterministic backward (gptattn_bwd_det): the same step with dQ partials stored per
     # (query tile, key tile) and summed in a fixed order instead of reduce-added.
     det = None
-    if not args.profile_run and (dt == ga.GPTATTN_F32 or w.hs == 64):
+    if not args.profile_run:
         nb_det = ga.gptattn_bwd_det_workspace_bytes(B, T, C, nh, dt)
         ws_det = torch.empty(max(nb_det, 256), dtype=torch.uint8, device=dev)
 
@@ -590,7 +608,7 @@ def run_ours(args, w, rank, world, local_rank):
     # the Philox keep mask generated in the forward and again in the backward; FLOPs counted as
     # for the plain step (the mask adds no matrix work).
     drop = None
-    if not args.profile_run and (dt == ga.GPTATTN_F32 or w.hs == 64):
+    if not args.profile_run:
         o = ga.Options(dropout_p=0.1, dropout_seed=1234)
         nb_o = ga.gptattn_bwd_opts_workspace_bytes(B, T, C, nh, o, dt)
 
