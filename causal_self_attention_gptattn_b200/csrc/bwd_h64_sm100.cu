@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0;; ++k, ++n) {
             const int w = item_index(k, blockIdx.x, gridDim.x);
             if (w >= n_items) break;
-            const int kt = w / BH, bh = w % BH;
+            const int kt = w / BH;
             const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
             for (int it = 0; it < niter; ++it, ++gi) {
                 const int st = gi % kQStages;

@@ -66,14 +66,20 @@ def test_window_bf16_head128_long_context_sampled_heads():
 
 
 def test_window_at_least_T_is_the_causal_path():
-    """window >= T takes exactly the causal kernels: bit-identical outputs."""
-    qkv, dy = make_inputs(2, 333, 2, 64, dtype=torch.bfloat16, seed=950)
-    a = run_fwd_bwd(qkv, dy, 2)
-    b = run_fwd_bwd(qkv, dy, 2, window=333)
-    c = run_fwd_bwd(qkv, dy, 2, window=10**6)
-    for x, y_, z in zip(a, b, c):
-        assert np.array_equal(x[np.isfinite(x)], y_[np.isfinite(y_)])
-        assert np.array_equal(x[np.isfinite(x)], z[np.isfinite(z)])
+    """window >= T takes exactly the causal kernels: y, lse, dK and dV bit-identical.  dQ is
+    summed over key tiles by fp32 reduce-adds whose order is not fixed (the deterministic
+    backward is the bitwise-reproducible one), so it is held to one bf16 rounding step."""
+    B, T, nh, hs = 2, 333, 2, 64
+    C = nh * hs
+    qkv, dy = make_inputs(B, T, nh, hs, dtype=torch.bfloat16, seed=950)
+    a = run_fwd_bwd(qkv, dy, nh)
+    for other in (run_fwd_bwd(qkv, dy, nh, window=T), run_fwd_bwd(qkv, dy, nh, window=10**6)):
+        for x, z in zip(a[:2], other[:2]):  # y, lse
+            assert np.array_equal(x, z)
+        assert np.array_equal(a[2][..., C:], other[2][..., C:])  # dK, dV
+        dq_a, dq_o = a[2][..., :C], other[2][..., :C]
+        assert np.allclose(dq_a, dq_o, rtol=2.0 ** -7, atol=1e-6 * np.abs(dq_a).max()), \
+            np.abs(dq_a - dq_o).max()
 
 
 def test_window_band_locality():
