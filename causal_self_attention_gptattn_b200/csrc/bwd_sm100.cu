@@ -17,15 +17,18 @@
 //           S^T = K Q_i^T, dP^T = V dO_i^T          (tcgen05, TMEM)
 //           P^T (bf16) back into TMEM; dS^T (bf16) into shared memory
 //           dV += P^T dO_i (P from TMEM), dK += dS^T Q_i   (TMEM accumulators)
-//           dQ_i = dS K -> TMEM -> smem -> TMA reduce-add into the fp32 accumulator
+//           dQ_i = dS K -> TMEM -> smem (32 columns at a time) -> TMA reduce-add
+//           into the fp32 accumulator
 //         epilogue: dK * scale and dV -> bf16 -> TMA store into dqkv
 //   post  dQ accumulator * scale -> bf16 into dqkv[..., 0:C]
 // Deterministic mode (n_slots > 0): each (query tile, key tile) partial of dQ is
 // stored in a slot of its own and the postprocess sums a query tile's slots in
 // a fixed order, so the result does not depend on the order CTAs finish in.
 //
-// Main-kernel roles (10 warps; 12 with dropout):
-//   warp 0      TMA producer (K, V once; Q_i, dO_i, lse_i, D_i per iteration)
+// Main kernel (head size 128; head size 64 has the persistent bwd_h64_sm100.cu).
+// Roles (10 warps; 12 with dropout):
+//   warp 0      TMA producer (K, V once; Q_i with lse_i and D_i through a two-stage
+//               ring, dO_i through one buffer refilled once dV_i has read it)
 //   warp 1      TMEM owner + MMA issuer
 //   warps 2..5  "softmax" warps, one key row each: P, dS, final dK/dV epilogue
 //   warps 6..9  dQ drain warps, one query row each: TMEM -> smem -> TMA reduce
@@ -35,10 +38,11 @@
 // scale 1/(1-p) into lse and D, so the recomputed weights are P * scale; P^T
 // goes to the dV product with dropped weights zeroed, and
 // dS = (P scale) o (dP o keep - D / scale).
-// TMEM columns: S^T [0,128) (P^T packed into [0,64)), dP^T [128,256),
-// dV [256,256+hs), dK [256+hs, 256+2hs).  dQ: hs=64 at [384,448); hs=128 in
-// two 64-column halves at [64,128) and [192,256), the parts of S^T / dP^T that
-// are free once P^T and dS^T have been produced.
+// TMEM columns: S^T [0,128) (P^T packed into [0,64)), dP^T [128,256), dV
+// [256,384), dK [384,512); dQ_i in the dP^T columns once the softmax warps have
+// read dP_i^T.  MMA order per query tile i: dV_i, S_{i+1} | dK_i, dQ_i, dP_{i+1}:
+// the next scores are computed while the softmax warps form dS_i, and dP_{i+1}
+// waits only for dQ_i to be drained out of its columns.
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -52,32 +56,38 @@ constexpr int kMStages = 4;
 constexpr uint32_t kMaskTileBytes = 128u * 16u;
 constexpr int kMaskThreads = 64;
 
+// Head size 128 only (head size 64 has its own persistent kernel).  Q_i travels with
+// -lse_i*log2(e) and -D_i through a two-stage ring; dO_i has a single buffer, refilled
+// once dV_i has read it; the dQ staging is one 16 KB slab (32 fp32 columns).
 template <int HS, bool kDropout = false>
 struct BwdCfg {
+    static_assert(HS == 128, "head size 128");
     static constexpr int kThreads = kDropout ? 320 + kMaskThreads : 320;
     static constexpr int kSlabs = HS / 64;
     static constexpr uint32_t kTileBytes = 128u * HS * 2u;
-    static constexpr int kStages = (HS == 64) ? 2 : 1;
+    static constexpr int kQStages = 2;
     static constexpr uint32_t kOffK = 0;
     static constexpr uint32_t kOffV = kOffK + kTileBytes;
-    static constexpr uint32_t kOffQ = kOffV + kTileBytes;
-    static constexpr uint32_t kOffdO = kOffQ + kStages * kTileBytes;
-    static constexpr uint32_t kOffdS = kOffdO + kStages * kTileBytes;  // 128 x 128 bf16, two slabs
-    static constexpr uint32_t kOffdQ = kOffdS + 2 * kSlabBytes;          // 128 x 64 fp32 staging, two slabs
-    static constexpr uint32_t kOffLse = kOffdQ + 2 * kSlabBytes;         // kStages x 128 fp32
-    static constexpr uint32_t kOffD = kOffLse + kStages * 512;
-    static constexpr uint32_t kOffBar = kOffD + kStages * 512;
+    static constexpr uint32_t kOffQ = kOffV + kTileBytes;                // kQStages tiles
+    static constexpr uint32_t kOffdO = kOffQ + kQStages * kTileBytes;    // one tile
+    static constexpr uint32_t kOffdS = kOffdO + kTileBytes;              // 128 x 128 bf16, two slabs
+    static constexpr uint32_t kOffdQ = kOffdS + 2 * kSlabBytes;          // 128 x 32 fp32 staging, one slab
+    static constexpr uint32_t kOffLse = kOffdQ + kSlabBytes;             // kQStages x 128 fp32
+    static constexpr uint32_t kOffD = kOffLse + kQStages * 512;
+    static constexpr uint32_t kOffBar = kOffD + kQStages * 512;
     static constexpr uint32_t kOffM = kOffBar + 256;
     static constexpr uint32_t kSmemBytes = kOffM + (kDropout ? kMStages * kMaskTileBytes : 0u) + 1024;
+    // TMEM: S^T (P^T packed into its first 64 columns), dP^T, dV, dK; dQ_i in the dP^T
+    // columns once the softmax warps have read dP_i^T, in two 64-column halves
     static constexpr uint32_t kColS = 0, kColdP = 128, kColdV = 256, kColdK = 256 + HS;
-    static constexpr uint32_t kColdQ0 = (HS == 64) ? 384 : 64;
-    static constexpr uint32_t kColdQ1 = 192;  // second half, hs = 128 only
-    static constexpr bool kDqAliases = (HS == 128);
+    static constexpr uint32_t kColdQ0 = 128, kColdQ1 = 192;
     // barriers
     static constexpr int kBarKV = 0;
-    static constexpr int kBarFull = 1;                 // kStages
-    static constexpr int kBarEmpty = kBarFull + kStages;  // kStages
-    static constexpr int kBarS = kBarEmpty + kStages;
+    static constexpr int kBarQFull = 1;                    // kQStages: Q_i, lse_i, D_i landed
+    static constexpr int kBarQEmpty = kBarQFull + kQStages;  // kQStages: dK_i has read Q_i
+    static constexpr int kBardOFull = kBarQEmpty + kQStages;
+    static constexpr int kBardOEmpty = kBardOFull + 1;     // dV_i has read dO_i
+    static constexpr int kBarS = kBardOEmpty + 1;
     static constexpr int kBardP = kBarS + 1;
     static constexpr int kBarP = kBardP + 1;
     static constexpr int kBardS = kBarP + 1;
@@ -139,7 +149,7 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
 
     const uint32_t sK = sbase + K::kOffK, sV = sbase + K::kOffV;
     auto sQ = [&](int st) -> uint32_t { return sbase + K::kOffQ + st * K::kTileBytes; };
-    auto sdO = [&](int st) -> uint32_t { return sbase + K::kOffdO + st * K::kTileBytes; };
+    const uint32_t sdO = sbase + K::kOffdO;
     const uint32_t sdS = sbase + K::kOffdS, sdQ = sbase + K::kOffdQ;
     const float *sLse = reinterpret_cast<const float *>(smem + K::kOffLse);
     const float *sD = reinterpret_cast<const float *>(smem + K::kOffD);
@@ -151,10 +161,12 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             mbar_init(bar(K::kBarMFull + s), kMaskThreads);
             mbar_init(bar(K::kBarMEmpty + s), 128);
         }
-        for (int s = 0; s < K::kStages; ++s) {
-            mbar_init(bar(K::kBarFull + s), 1);
-            mbar_init(bar(K::kBarEmpty + s), 1);
+        for (int s = 0; s < K::kQStages; ++s) {
+            mbar_init(bar(K::kBarQFull + s), 1);
+            mbar_init(bar(K::kBarQEmpty + s), 1);
         }
+        mbar_init(bar(K::kBardOFull), 1);
+        mbar_init(bar(K::kBardOEmpty), 1);
         mbar_init(bar(K::kBarS), 1);
         mbar_init(bar(K::kBardP), 1);
         mbar_init(bar(K::kBarP), 128);
@@ -188,31 +200,36 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                 tma_load_3d(sK + s * kSlabBytes, &map_qkv, bar(K::kBarKV), col_k + 64 * s, kt * kTile, b);
                 tma_load_3d(sV + s * kSlabBytes, &map_qkv, bar(K::kBarKV), col_v + 64 * s, kt * kTile, b);
             }
-            int issued = 0;
+            int q_issued = 0, do_issued = 0;
             bool ok = true;
-            for (int it = 0; it < niter; ++it) {
+            for (int it = 0; it < niter && ok; ++it) {
                 const int qt = kt + it;
-                const int st = it % K::kStages;
-                const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
-                if (it >= K::kStages && !mbar_wait(bar(K::kBarEmpty + st), ph ^ 1u, g)) {
-                    ok = false;
+                const int st = it % K::kQStages;
+                // Q_i, -lse_i*log2(e), -D_i into stage st once dK of tile i-2 has read it
+                if (it >= K::kQStages &&
+                    !(ok = mbar_wait(bar(K::kBarQEmpty + st), (uint32_t)((it / K::kQStages) & 1) ^ 1u, g)))
                     break;
-                }
-                const uint32_t fb = bar(K::kBarFull + st);
-                mbar_arrive_expect_tx(fb, 2 * K::kTileBytes + 1024);
-                for (int s = 0; s < K::kSlabs; ++s) {
+                const uint32_t fb = bar(K::kBarQFull + st);
+                mbar_arrive_expect_tx(fb, K::kTileBytes + 1024);
+                for (int s = 0; s < K::kSlabs; ++s)
                     tma_load_3d(sQ(st) + s * kSlabBytes, &map_qkv, fb, col_q + 64 * s, qt * kTile, b);
-                    tma_load_3d(sdO(st) + s * kSlabBytes, &map_dy, fb, h * HS + 64 * s, qt * kTile, b);
-                }
                 const size_t rowoff = (size_t)bh * (size_t)T_pad + (size_t)qt * kTile;
                 bulk_load(sbase + K::kOffLse + st * 512, lse2 + rowoff, 512, fb);
                 bulk_load(sbase + K::kOffD + st * 512, Dvec + rowoff, 512, fb);
-                issued = it + 1;
+                q_issued = it + 1;
+                // dO_i into its single buffer once dV of tile i-1 has read it
+                if (it >= 1 && !(ok = mbar_wait(bar(K::kBardOEmpty), (uint32_t)((it - 1) & 1), g))) break;
+                mbar_arrive_expect_tx(bar(K::kBardOFull), K::kTileBytes);
+                for (int s = 0; s < K::kSlabs; ++s)
+                    tma_load_3d(sdO + s * kSlabBytes, &map_dy, bar(K::kBardOFull), h * HS + 64 * s, qt * kTile, b);
+                do_issued = it + 1;
             }
             if (!ok || *abort_flag) {
+                // let this CTA's last copies land before shared memory is released
                 drain_wait(bar(K::kBarKV), 0, budget_ns);
-                for (int it = (issued > K::kStages ? issued - K::kStages : 0); it < issued; ++it)
-                    drain_wait(bar(K::kBarFull + it % K::kStages), (uint32_t)(it / K::kStages) & 1u, budget_ns);
+                for (int q = (q_issued > K::kQStages ? q_issued - K::kQStages : 0); q < q_issued; ++q)
+                    drain_wait(bar(K::kBarQFull + q % K::kQStages), (uint32_t)(q / K::kQStages) & 1u, budget_ns);
+                if (do_issued > 0) drain_wait(bar(K::kBardOFull), (uint32_t)((do_issued - 1) & 1), budget_ns);
             }
         }
     } else if (warp == 1) {
@@ -223,14 +240,8 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             constexpr uint32_t idQ = idesc_bf16_f32(128, 64, true, true);      // dQ half (A = dS, M-major)
             bool ok = mbar_wait(bar(K::kBarKV), 0, g);
             bool any = false;
-            for (int it = 0; it < niter && ok; ++it) {
-                const int st = it % K::kStages;
-                const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
-                if (!(ok = mbar_wait(bar(K::kBarFull + st), ph, g))) break;
-                if (K::kDqAliases && it > 0 && !(ok = mbar_wait(bar(K::kBardQEmpty), (uint32_t)(it - 1) & 1u, g)))
-                    break;
-                tc_fence_after();
-                // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+            // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+            auto issue_S = [&](int st) {
 #pragma unroll
                 for (int kk = 0; kk < HS / 16; ++kk) {
                     const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
@@ -238,21 +249,42 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                             idSS, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar(K::kBarS));
+            };
+            auto issue_dP = [&]() {
 #pragma unroll
                 for (int kk = 0; kk < HS / 16; ++kk) {
                     const uint32_t koff = (uint32_t)(kk >> 2) * kSlabBytes + (uint32_t)(kk & 3) * 32u;
-                    umma_ss(tmem + K::kColdP, sdesc_sw128(sV + koff, 16, 1024), sdesc_sw128(sdO(st) + koff, 16, 1024),
+                    umma_ss(tmem + K::kColdP, sdesc_sw128(sV + koff, 16, 1024), sdesc_sw128(sdO + koff, 16, 1024),
                             idSS, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar(K::kBardP));
+            };
+            // Order per tile i: dV_i, S_{i+1} | dK_i, dQ_i, dP_{i+1}.  S_{i+1} goes right after dV_i
+            // (which has read P_i^T out of the S^T columns), so the softmax warps find the next
+            // scores ready when they finish dS_i; dP_{i+1} waits for dQ_i, which shares its
+            // columns, to be drained.
+            if (ok && (ok = mbar_wait(bar(K::kBarQFull), 0, g)) && (ok = mbar_wait(bar(K::kBardOFull), 0, g))) {
+                tc_fence_after();
+                issue_S(0);
+                issue_dP();
                 any = true;
+            }
+            for (int it = 0; it < niter && ok; ++it) {
+                const int st = it % K::kQStages;
                 // dV += P^T dO   (A = P^T in TMEM, K = query rows)
                 if (!(ok = mbar_wait(bar(K::kBarP), (uint32_t)it & 1u, g))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     umma_ts(tmem + K::kColdV, tmem + K::kColS + 8u * kk,
-                            sdesc_sw128(sdO(st) + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                            sdesc_sw128(sdO + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(bar(K::kBardOEmpty));  // dO_i read by dP_i and dV_i
+                if (it + 1 < niter) {
+                    const int st1 = (it + 1) % K::kQStages;
+                    if (!(ok = mbar_wait(bar(K::kBarQFull + st1), (uint32_t)(((it + 1) / K::kQStages) & 1), g))) break;
+                    tc_fence_after();
+                    issue_S(st1);
+                }
                 // dK += dS^T Q   (A = dS^T in smem, key rows x query cols, K-major)
                 if (!(ok = mbar_wait(bar(K::kBardS), (uint32_t)it & 1u, g))) break;
                 tc_fence_after();
@@ -262,12 +294,9 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                     umma_ss(tmem + K::kColdK, sdesc_sw128(sdS + koff, 16, 1024),
                             sdesc_sw128(sQ(st) + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(bar(K::kBarEmpty + st));  // Q_i / dO_i / lse_i / D_i no longer needed
-                // dQ_i = dS K   (A = dS, M-major view of the same smem; B = K, N-major)
-                if (!K::kDqAliases && it > 0 &&
-                    !(ok = mbar_wait(bar(K::kBardQEmpty), (uint32_t)(it - 1) & 1u, g)))
-                    break;
-                tc_fence_after();
+                umma_commit(bar(K::kBarQEmpty + st));  // Q_i, lse_i, D_i no longer needed
+                // dQ_i = dS K   (A = dS, M-major view of the same smem; B = K, N-major), into the
+                // dP^T columns, which the softmax warps read out before they stored dS_i
 #pragma unroll
                 for (int half = 0; half < HS / 64; ++half) {
                     const uint32_t dcol = half == 0 ? K::kColdQ0 : K::kColdQ1;
@@ -278,6 +307,12 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                                 kk > 0 ? 1u : 0u);
                 }
                 umma_commit(bar(K::kBardQFull));
+                if (it + 1 < niter) {
+                    if (!(ok = mbar_wait(bar(K::kBardOFull), (uint32_t)((it + 1) & 1), g))) break;
+                    if (!(ok = mbar_wait(bar(K::kBardQEmpty), (uint32_t)it & 1u, g))) break;
+                    tc_fence_after();
+                    issue_dP();
+                }
             }
             if (ok) umma_commit(bar(K::kBarKdV));
             if (any || ok) {
@@ -293,8 +328,8 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
         const float scale_log2 = (HS == 64 ? 0.125f : 0.08838834764831845f) * 1.4426950408889634f;
         bool ok = true;
         for (int it = 0; it < niter; ++it) {
-            const int st = it % K::kStages;
-            const uint32_t ph = (uint32_t)(it / K::kStages) & 1u;
+            const int st = it % K::kQStages;
+            const uint32_t ph = (uint32_t)(it / K::kQStages) & 1u;
             // dropout keep words of this key row's 128 query columns (bit layout of philox.cuh)
             uint32_t kb[4] = {0u, 0u, 0u, 0u};
             if constexpr (kDropout) {
@@ -307,7 +342,7 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                 kb[3] = v.w;
                 mbar_arrive(bar(K::kBarMEmpty + ms));
             }
-            ok = warp_wait(bar(K::kBarFull + st), ph, g) && warp_wait(bar(K::kBarS), (uint32_t)it & 1u, g);
+            ok = warp_wait(bar(K::kBarQFull + st), ph, g) && warp_wait(bar(K::kBarS), (uint32_t)it & 1u, g);
             if (!ok) break;
             tc_fence_after();
             const float *lse_i = sLse + st * 128;
@@ -392,7 +427,7 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             for (int which = 0; which < 2; ++which) {
                 const uint32_t col = which == 0 ? K::kColdV : K::kColdK;
                 const float mul = which == 0 ? 1.f : scale;
-                const uint32_t stage_buf = which == 0 ? sQ(0) : sdO(0);
+                const uint32_t stage_buf = which == 0 ? sQ(0) : sdO;
 #pragma unroll
                 for (int c0 = 0; c0 < HS; c0 += 32) {
                     uint32_t o[32];
@@ -416,7 +451,7 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
         if (warp == 2 && lane == 0 && !*abort_flag) {
             for (int s = 0; s < K::kSlabs; ++s) {
                 tma_store_3d(&map_dqkv, sQ(0) + s * kSlabBytes, 2 * C + h * HS + 64 * s, kt * kTile, b);
-                tma_store_3d(&map_dqkv, sdO(0) + s * kSlabBytes, C + h * HS + 64 * s, kt * kTile, b);
+                tma_store_3d(&map_dqkv, sdO + s * kSlabBytes, C + h * HS + 64 * s, kt * kTile, b);
             }
             bulk_commit_group();
             bulk_wait_group_0();
@@ -433,43 +468,36 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
         for (int it = 0; it < niter; ++it) {
             const int qt = kt + it;
             if (ok) ok = warp_wait(bar(K::kBardQFull), (uint32_t)it & 1u, g);
-            if (ok) tc_fence_after();
+            // both 64-column halves out of TMEM first, so that dP_{i+1} may take the columns
+            uint32_t v[HS];
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-            for (int half = 0; half < HS / 64; ++half) {
-                uint32_t v[64];
-                const uint32_t dcol = half == 0 ? K::kColdQ0 : K::kColdQ1;
-                if (ok) {
-                    tmem_ld_x32(trow + dcol, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                    tmem_ld_x32(trow + dcol + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-                    if (half == HS / 64 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(bar(K::kBardQEmpty));
-                    }
-                }
-                if (leader) bulk_wait_group_read_0();  // staging free again
+                for (int c = 0; c < HS; c += 32)
+                    tmem_ld_x32(trow + (c < 64 ? K::kColdQ0 + c : K::kColdQ1 + (c - 64)),
+                                *reinterpret_cast<uint32_t(*)[32]>(&v[c]));
+                tc_fence_before();
+                mbar_arrive(bar(K::kBardQEmpty));
+            }
+            // then 32 columns at a time through the staging slab
+#pragma unroll
+            for (int u = 0; u < HS / 32; ++u) {
+                if (leader) bulk_wait_group_read_0();  // the slab's previous copy-out has read it
                 named_bar_sync(2, 128);
                 if (ok) {
+                    const uint32_t rbase = sdQ + (uint32_t)row * 128u;
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const uint32_t rbase = sdQ + (uint32_t)u * kSlabBytes + (uint32_t)row * 128u;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), v[32 * u + 4 * q],
-                                         v[32 * u + 4 * q + 1], v[32 * u + 4 * q + 2], v[32 * u + 4 * q + 3]);
-                    }
+                    for (int q = 0; q < 8; ++q)
+                        st_shared_v4(rbase + (((uint32_t)q ^ (uint32_t)(row & 7)) << 4), v[32 * u + 4 * q],
+                                     v[32 * u + 4 * q + 1], v[32 * u + 4 * q + 2], v[32 * u + 4 * q + 3]);
                     fence_proxy_async_smem();
                 }
                 named_bar_sync(2, 128);
                 if (leader && ok && !*abort_flag) {
-                    if (n_slots == 0) {  // add into the (b, h, query tile) rows of the accumulator
-                        const int r0 = bh * T_pad + qt * kTile;
-                        tma_reduce_add_2d(&map_dq, sdQ, half * 64, r0);
-                        tma_reduce_add_2d(&map_dq, sdQ + kSlabBytes, half * 64 + 32, r0);
-                    } else {  // deterministic: a slot of its own per (query tile, key tile)
-                        const int r0 = (bh * n_slots + qt * (qt + 1) / 2 + kt) * kTile;
-                        tma_store_2d(&map_dq, sdQ, half * 64, r0);
-                        tma_store_2d(&map_dq, sdQ + kSlabBytes, half * 64 + 32, r0);
-                    }
+                    if (n_slots == 0)  // add into the (b, h, query tile) rows of the accumulator
+                        tma_reduce_add_2d(&map_dq, sdQ, 32 * u, bh * T_pad + qt * kTile);
+                    else  // deterministic: a slot of its own per (query tile, key tile)
+                        tma_store_2d(&map_dq, sdQ, 32 * u, (bh * n_slots + qt * (qt + 1) / 2 + kt) * kTile);
                     bulk_commit_group();
                 }
             }
@@ -665,15 +693,12 @@ cudaError_t launch_main_impl(const CUtensorMap &map_qkv, const CUtensorMap &map_
                              int n_head, int T_pad, int window, int n_slots, DropoutParams dp, DevCtx ctx,
                              cudaStream_t s) {
     const bool band = window < T, drop = dp.threshold != 0u;
-    if (band)
-        return drop ? launch_main_variant<HS, true, true>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
-                                                          T_pad, window, n_slots, dp, ctx, s)
-                    : launch_main_variant<HS, true, false>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
-                                                           T_pad, window, n_slots, dp, ctx, s);
-    return drop ? launch_main_variant<HS, false, true>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
-                                                       T_pad, window, n_slots, dp, ctx, s)
-                : launch_main_variant<HS, false, false>(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head,
-                                                        T_pad, window, n_slots, dp, ctx, s);
+    auto run = [&](auto kern_launch) {
+        return kern_launch(map_qkv, map_dy, map_dqkv, map_dq, lse2, D, B, T, C, n_head, T_pad, window, n_slots, dp, ctx,
+                           s);
+    };
+    if (band) return drop ? run(launch_main_variant<HS, true, true>) : run(launch_main_variant<HS, true, false>);
+    return drop ? run(launch_main_variant<HS, false, true>) : run(launch_main_variant<HS, false, false>);
 }
 
 }  // namespace
