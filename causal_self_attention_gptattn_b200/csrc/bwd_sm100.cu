@@ -26,14 +26,15 @@
 // a fixed order, so the result does not depend on the order CTAs finish in.
 //
 // Main kernel (head size 128; head size 64 has the persistent bwd_h64_sm100.cu).
-// Roles (10 warps; 12 with dropout):
+// Four warpgroups, registers moved among them by setmaxnreg:
 //   warp 0      TMA producer (K, V once; Q_i with lse_i and D_i through a two-stage
 //               ring, dO_i through one buffer refilled once dV_i has read it)
 //   warp 1      TMEM owner + MMA issuer
-//   warps 2..5  "softmax" warps, one key row each: P, dS, final dK/dV epilogue
-//   warps 6..9  dQ drain warps, one query row each: TMEM -> smem -> TMA reduce
-//   warps 10,11 with dropout: the keep words of each (key tile, query tile),
+//   warps 2,3   with dropout: the keep words of each (key tile, query tile),
 //               drawn a few tiles ahead into a shared-memory ring
+//   warps 4..11 "softmax" warps, one key row and 64 query columns each (two
+//               warpgroups, one per half of the query tile): P, dS, dK/dV epilogue
+//   warps 12..15 dQ drain, one query row each: TMEM -> smem -> TMA reduce
 // Dropout (inverted, Philox mask of philox.cuh): the preprocess folds the
 // scale 1/(1-p) into lse and D, so the recomputed weights are P * scale; P^T
 // goes to the dV product with dropped weights zeroed, and
@@ -62,7 +63,12 @@ constexpr int kMaskThreads = 64;
 template <int HS, bool kDropout = false>
 struct BwdCfg {
     static_assert(HS == 128, "head size 128");
-    static constexpr int kThreads = kDropout ? 320 + kMaskThreads : 320;
+    // four warpgroups: control (producer, MMA issuer; with dropout two mask warps), two softmax
+    // warpgroups (64 query columns each), the dQ drain; registers moved by setmaxnreg
+    static constexpr int kThreads = 512;
+    static constexpr int kLaunchRegs = 128;
+    static constexpr uint32_t kRegsCtl = 64, kRegsSoftmax = 136, kRegsDrain = 176;
+    static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsDrain == 4 * kLaunchRegs, "register split");
     static constexpr int kSlabs = HS / 64;
     static constexpr uint32_t kTileBytes = 128u * HS * 2u;
     static constexpr int kQStages = 2;
@@ -159,7 +165,7 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
         mbar_init(bar(K::kBarKV), 1);
         for (int s = 0; s < kMStages; ++s) {
             mbar_init(bar(K::kBarMFull + s), kMaskThreads);
-            mbar_init(bar(K::kBarMEmpty + s), 128);
+            mbar_init(bar(K::kBarMEmpty + s), 256);
         }
         for (int s = 0; s < K::kQStages; ++s) {
             mbar_init(bar(K::kBarQFull + s), 1);
@@ -169,8 +175,8 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
         mbar_init(bar(K::kBardOEmpty), 1);
         mbar_init(bar(K::kBarS), 1);
         mbar_init(bar(K::kBardP), 1);
-        mbar_init(bar(K::kBarP), 128);
-        mbar_init(bar(K::kBardS), 128);
+        mbar_init(bar(K::kBarP), 256);
+        mbar_init(bar(K::kBardS), 256);
         mbar_init(bar(K::kBardQFull), 1);
         mbar_init(bar(K::kBardQEmpty), 128);
         mbar_init(bar(K::kBarKdV), 1);
@@ -189,6 +195,8 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
     griddep_launch_dependents();
     griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
+    if (warp < 4) {
+        regs_dec<K::kRegsCtl>();
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -276,7 +284,8 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + K::kColdV, tmem + K::kColS + 8u * kk,
+                    // A = P^T: query columns 16kk.. sit packed in half kk/4's S^T columns
+                    umma_ts(tmem + K::kColdV, tmem + K::kColS + 64u * (uint32_t)(kk >> 2) + 8u * (uint32_t)(kk & 3),
                             sdesc_sw128(sdO + kk * 2048u, kSlabBytes, 1024), idAcc, (it > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(bar(K::kBardOEmpty));  // dO_i read by dP_i and dV_i
                 if (it + 1 < niter) {
@@ -320,43 +329,72 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                 drain_wait(bar(K::kBarDone), 0, budget_ns);
             }
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------------------ softmax warps (key rows)
+    } else {
+        // ------------------------------------------------------------ dropout keep words (warps 2, 3)
+        if constexpr (kDropout) {
+            // thread -> key rows 4*kg .. 4*kg+3 and query columns 64*qh .. 64*qh+63 of every tile
+            const int u = threadIdx.x - 64, kg = u >> 1, qh = u & 1;
+            const uint32_t t7 = theta_low7(dp.threshold);
+            const uint32_t s0 = (uint32_t)(kt * kTile + 4 * kg);
+            for (int it = 0; it < niter; ++it) {
+                const int ms = it % kMStages;
+                if (it >= kMStages && !warp_wait(bar(K::kBarMEmpty + ms), (uint32_t)((it / kMStages) & 1) ^ 1u, g))
+                    break;
+                const uint32_t t0 = (uint32_t)((kt + it) * kTile + 64 * qh);
+                uint32_t lo[4], hi[4];
+                if (dp.threshold >= 128u) {
+                    dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
+                    dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
+                } else {
+                    dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
+                    dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
+                }
+                const uint32_t dst = sM + (uint32_t)ms * kMaskTileBytes + (uint32_t)(4 * kg) * 16u + (uint32_t)qh * 8u;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) st_shared_v2(dst + (uint32_t)c * 16u, lo[c], hi[c]);
+                mbar_arrive(bar(K::kBarMFull + ms));
+            }
+        }
+    }
+    } else if (warp < 12) {
+        // ------------------------------------------------------------ softmax warpgroups (key rows)
+        regs_inc<K::kRegsSoftmax>();
+        const int half = (warp >> 2) - 1;  // query columns 64*half .. 64*half+63 of each tile
         const int sp = warp & 3;
         const int row = sp * 32 + lane;  // key row within the tile
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
-        const float scale_log2 = (HS == 64 ? 0.125f : 0.08838834764831845f) * 1.4426950408889634f;
+        const float scale_log2 = 0.08838834764831845f * 1.4426950408889634f;
         bool ok = true;
         for (int it = 0; it < niter; ++it) {
             const int st = it % K::kQStages;
             const uint32_t ph = (uint32_t)(it / K::kQStages) & 1u;
-            // dropout keep words of this key row's 128 query columns (bit layout of philox.cuh)
-            uint32_t kb[4] = {0u, 0u, 0u, 0u};
+            // dropout keep words of this key row's 64 query columns (bit layout of philox.cuh)
+            uint32_t kb[2] = {0u, 0u};
             if constexpr (kDropout) {
                 const int ms = it % kMStages;
                 if (!(ok = warp_wait(bar(K::kBarMFull + ms), (uint32_t)(it / kMStages) & 1u, g))) break;
-                const uint4 v = ld_shared_v4(sM + (uint32_t)ms * kMaskTileBytes + (uint32_t)row * 16u);
+                const uint2 v = ld_shared_v2(sM + (uint32_t)ms * kMaskTileBytes + (uint32_t)row * 16u + (uint32_t)half * 8u);
                 kb[0] = v.x;
                 kb[1] = v.y;
-                kb[2] = v.z;
-                kb[3] = v.w;
                 mbar_arrive(bar(K::kBarMEmpty + ms));
             }
             ok = warp_wait(bar(K::kBarQFull + st), ph, g) && warp_wait(bar(K::kBarS), (uint32_t)it & 1u, g);
             if (!ok) break;
             tc_fence_after();
-            const float *lse_i = sLse + st * 128;
-            const float *D_i = sD + st * 128;
-            uint32_t pk[64];  // P^T row, bf16 pairs
+            const float *lse_i = sLse + st * 128 + 64 * half;
+            const float *D_i = sD + st * 128 + 64 * half;
+            uint32_t pk[32];  // P^T row segment, bf16 pairs
+            // this half's S^T columns in, P^T packed back over the first 32 of them
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t sr[32];
-                tmem_ld_x32(trow + K::kColS + 32 * ch, sr);
+                tmem_ld_x32(trow + K::kColS + 64 * half + 32 * ch, sr);
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int c = 32 * ch + e;
-                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, lse_i[c]));
-                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), scale_log2, lse_i[c + 1]));
+                    const int cl = 32 * ch + e;      // column within the half
+                    const int c = 64 * half + cl;    // query column within the tile
+                    float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), scale_log2, lse_i[cl]));
+                    float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), scale_log2, lse_i[cl + 1]));
                     if (it == 0) {  // diagonal tile: query c sees key row only if row <= c
                         if (c < row) p0 = 0.f;
                         if (c + 1 < row) p1 = 0.f;
@@ -366,17 +404,18 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                         if (c >= cut) p0 = 0.f;
                         if (c + 1 >= cut) p1 = 0.f;
                     }
-                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                    pk[cl >> 1] = pack_bf16x2(p0, p1);
                 }
-                // columns [16ch, 16ch+16) were read in an earlier (or this) chunk; with dropout the
-                // dV product gets the dropped weights zeroed, dS below the undropped ones
+                // packed columns [16ch, 16ch+16) of this half were read in an earlier (or this) chunk;
+                // with dropout the dV product gets the dropped weights zeroed, dS below the undropped ones
                 if constexpr (kDropout) {
                     uint32_t pm[16];
 #pragma unroll
                     for (int q = 0; q < 16; ++q) pm[q] = pk[16 * ch + q] & keep_pair_mask(kb[ch] << (q >> 1), q & 1);
-                    tmem_st_x16(trow + K::kColS + 16 * ch, pm);
+                    tmem_st_x16(trow + K::kColS + 64 * half + 16 * ch, pm);
                 } else {
-                    tmem_st_x16(trow + K::kColS + 16 * ch, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * ch]));
+                    tmem_st_x16(trow + K::kColS + 64 * half + 16 * ch,
+                                *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * ch]));
                 }
             }
             tmem_st_wait();
@@ -387,10 +426,12 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             if (ok && it > 0) ok = warp_wait(bar(K::kBardQFull), (uint32_t)(it - 1) & 1u, g);  // dS buffer free
             if (!ok) break;
             tc_fence_after();
+            // dS^T row `row`, this half's query columns = slab `half`, 16-byte chunks 4*ch .. 4*ch+3
+            const uint32_t rbase = sdS + (uint32_t)half * kSlabBytes + (uint32_t)row * 128u;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; ch < 2; ++ch) {
                 uint32_t dr[32];
-                tmem_ld_x32(trow + K::kColdP + 32 * ch, dr);
+                tmem_ld_x32(trow + K::kColdP + 64 * half + 32 * ch, dr);
                 if constexpr (kDropout) {  // dropped columns: dP^T o keep = 0
 #pragma unroll
                     for (int e = 0; e < 32; ++e) dr[e] &= keep_word_mask(kb[ch] << (e >> 2), e & 3);
@@ -398,17 +439,15 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const int c = 32 * ch + e;
-                    const uint32_t pp = pk[c >> 1];
-                    const float ds0 = bf16lo_to_f32(pp) * (__uint_as_float(dr[e]) + D_i[c]);
-                    const float ds1 = bf16hi_to_f32(pp) * (__uint_as_float(dr[e + 1]) + D_i[c + 1]);
+                    const int cl = 32 * ch + e;
+                    const uint32_t pp = pk[cl >> 1];
+                    const float ds0 = bf16lo_to_f32(pp) * (__uint_as_float(dr[e]) + D_i[cl]);
+                    const float ds1 = bf16hi_to_f32(pp) * (__uint_as_float(dr[e + 1]) + D_i[cl + 1]);
                     w[e >> 1] = pack_bf16x2(ds0, ds1);
                 }
-                // dS^T row `row`, query columns [32ch, 32ch+32): slab ch/2, 16-byte chunks 4*(ch&1)..+3
-                const uint32_t rbase = sdS + (uint32_t)(ch >> 1) * kSlabBytes + (uint32_t)row * 128u;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t chunk = (uint32_t)(4 * (ch & 1) + q);
+                    const uint32_t chunk = (uint32_t)(4 * ch + q);
                     st_shared_v4(rbase + ((chunk ^ (uint32_t)(row & 7)) << 4), w[4 * q], w[4 * q + 1], w[4 * q + 2],
                                  w[4 * q + 3]);
                 }
@@ -418,37 +457,37 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             mbar_arrive(bar(K::kBardS));
         }
         // -------------------------------------------------------- dK / dV epilogue
+        // this half's 64 columns of dV and dK (scaled) -> bf16 -> slab `half` of the staging
+        // tiles (dV in the stage-0 Q buffer, dK in the dO buffer, both free once the last MMAs ran)
         if (ok) ok = warp_wait(bar(K::kBarKdV), 0, g);
         if (ok) {
             tc_fence_after();
-            const float scale = (HS == 64 ? 0.125f : 0.08838834764831845f);
-            // staging: dV tile in the Q buffer of stage 0, dK tile in the dO buffer of stage 0
+            const float scale = 0.08838834764831845f;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                const uint32_t col = which == 0 ? K::kColdV : K::kColdK;
+                const uint32_t col = (which == 0 ? K::kColdV : K::kColdK) + 64u * (uint32_t)half;
                 const float mul = which == 0 ? 1.f : scale;
-                const uint32_t stage_buf = which == 0 ? sQ(0) : sdO;
+                const uint32_t rbase0 = (which == 0 ? sQ(0) : sdO) + (uint32_t)half * kSlabBytes + (uint32_t)row * 128u;
 #pragma unroll
-                for (int c0 = 0; c0 < HS; c0 += 32) {
+                for (int c0 = 0; c0 < 64; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld_x32(trow + col + c0, o);
                     uint32_t w[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c)
                         w[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * mul, __uint_as_float(o[2 * c + 1]) * mul);
-                    const uint32_t rbase = stage_buf + (uint32_t)(c0 >> 6) * kSlabBytes + (uint32_t)row * 128u;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint32_t chunk = (uint32_t)(((c0 & 63) >> 3) + q);
-                        st_shared_v4(rbase + ((chunk ^ (uint32_t)(row & 7)) << 4), w[4 * q], w[4 * q + 1],
+                        const uint32_t chunk = (uint32_t)((c0 >> 3) + q);
+                        st_shared_v4(rbase0 + ((chunk ^ (uint32_t)(row & 7)) << 4), w[4 * q], w[4 * q + 1],
                                      w[4 * q + 2], w[4 * q + 3]);
                     }
                 }
             }
             fence_proxy_async_smem();
         }
-        named_bar_sync(1, 128);
-        if (warp == 2 && lane == 0 && !*abort_flag) {
+        named_bar_sync(1, 256);
+        if (warp == 4 && lane == 0 && !*abort_flag) {
             for (int s = 0; s < K::kSlabs; ++s) {
                 tma_store_3d(&map_dqkv, sQ(0) + s * kSlabBytes, 2 * C + h * HS + 64 * s, kt * kTile, b);
                 tma_store_3d(&map_dqkv, sdO + s * kSlabBytes, C + h * HS + 64 * s, kt * kTile, b);
@@ -456,12 +495,13 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             bulk_commit_group();
             bulk_wait_group_0();
         }
-    } else if (warp < 10) {
-        // ------------------------------------------------------------ dQ drain warps (query rows)
+    } else {
+        // ------------------------------------------------------------ dQ drain warpgroup (query rows)
+        regs_inc<K::kRegsDrain>();
         const int sp = warp & 3;
         const int row = sp * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(sp * 32) << 16);
-        const bool leader = (warp == 6 && lane == 0);
+        const bool leader = (warp == 12 && lane == 0);
         // Every thread of this role executes the same sequence of named
         // barriers whatever happens; after a failed wait the work is skipped.
         bool ok = true;
@@ -503,32 +543,6 @@ __global__ void __launch_bounds__(BwdCfg<HS, kDropout>::kThreads, 1)
             }
         }
         if (leader) bulk_wait_group_0();
-    } else {
-        // ------------------------------------------------------------ dropout keep words (warps 10, 11)
-        if constexpr (kDropout) {
-            // thread -> key rows 4*kg .. 4*kg+3 and query columns 64*qh .. 64*qh+63 of every tile
-            const int u = threadIdx.x - 320, kg = u >> 1, qh = u & 1;
-            const uint32_t t7 = theta_low7(dp.threshold);
-            const uint32_t s0 = (uint32_t)(kt * kTile + 4 * kg);
-            for (int it = 0; it < niter; ++it) {
-                const int ms = it % kMStages;
-                if (it >= kMStages && !warp_wait(bar(K::kBarMEmpty + ms), (uint32_t)((it / kMStages) & 1) ^ 1u, g))
-                    break;
-                const uint32_t t0 = (uint32_t)((kt + it) * kTile + 64 * qh);
-                uint32_t lo[4], hi[4];
-                if (dp.threshold >= 128u) {
-                    dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
-                    dropout_keep32x4_keys<true>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
-                } else {
-                    dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0, lo);
-                    dropout_keep32x4_keys<false>(dp.seed, t7, (uint32_t)bh, s0, t0 + 32u, hi);
-                }
-                const uint32_t dst = sM + (uint32_t)ms * kMaskTileBytes + (uint32_t)(4 * kg) * 16u + (uint32_t)qh * 8u;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) st_shared_v2(dst + (uint32_t)c * 16u, lo[c], hi[c]);
-                mbar_arrive(bar(K::kBarMFull + ms));
-            }
-        }
     }
 
     tc_fence_before();
@@ -681,6 +695,12 @@ cudaError_t launch_main_variant(const CUtensorMap &map_qkv, const CUtensorMap &m
     auto kern = bwd_bf16_kernel<HS, kBand, kDropout>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
+    // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs per
+    // thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != K::kLaunchRegs) return cudaErrorInvalidConfiguration;
     const int n_t = ceil_div(T, kTile);
     const long long blocks = (long long)n_t * B * n_head;
     return launch_pdl(kern, dim3((unsigned)blocks), dim3(K::kThreads), K::kSmemBytes, s, map_qkv, map_dy, map_dqkv,
