@@ -128,3 +128,41 @@ def test_bf16_many_short_sequences():
     qkv, dy = make_inputs(32, 130, 32, 64, dtype=torch.bfloat16, seed=130)
     got = run_fwd_bwd(qkv, dy, 32)
     compare(got, oracle_all(qkv, dy, 32), torch.bfloat16, "1024 x 130")
+
+
+@pytest.mark.parametrize("hs", [64, 128])
+def test_bf16_max_length_closed_form(hs):
+    """T = 16384 (128 query tiles per (b, h)) against closed forms instead of the oracle: with
+    q = 0 every score is 0, so each weight is 1/(t+1) and
+        y[t] = mean(v[0..t]),  lse[t] = ln(t+1),  dV[s] = sum_{t >= s} dy[t] / (t+1),  dK = 0,
+        dQ[t] = scale / (t+1) * sum_{s <= t} (dy[t].v[s] - dy[t].y[t]) k[s]
+    (the softmax Jacobian with P[t, s] = 1/(t+1))."""
+    B, T, nh = 1, 16384, 2
+    C = nh * hs
+    g = torch.Generator().manual_seed(16384 + hs)
+    qkv = torch.randn(B, T, 3 * C, generator=g)
+    qkv[:, :, :C] = 0.0
+    dy = torch.randn(B, T, C, generator=g)
+    qkv, dy = qkv.to(torch.bfloat16), dy.to(torch.bfloat16)
+    y, lse, dqkv = run_fwd_bwd(qkv, dy, nh)
+    k = qkv[0, :, C:2 * C].double().numpy()
+    v = qkv[0, :, 2 * C:].double().numpy()
+    g_ = dy[0].double().numpy()
+    n = np.arange(1, T + 1, dtype=np.float64)[:, None]
+    y_ref = np.cumsum(v, axis=0) / n
+    dv_ref = np.cumsum((g_ / n)[::-1], axis=0)[::-1]
+    assert np.abs(y[0] - y_ref).max() <= 2e-2
+    assert np.abs(lse[0] - np.log(n[:, 0])[None, :]).max() <= 1e-2
+    assert np.array_equal(dqkv[0, :, C:2 * C], np.zeros((T, C)))
+    dv = dqkv[0, :, 2 * C:]
+    assert np.abs(dv - dv_ref).max() <= 5e-2 * np.abs(dv_ref).max()
+    scale = 1.0 / np.sqrt(hs)
+    rows = [0, 1, 127, 128, 4095, 8191, 12000, T - 1]
+    dq_ref = np.zeros((len(rows), C))
+    for i, t in enumerate(rows):
+        for h in range(nh):
+            cs = slice(h * hs, (h + 1) * hs)
+            a = v[:t + 1, cs] @ g_[t, cs] - g_[t, cs] @ y_ref[t, cs]  # dP[t, s] - D[t]
+            dq_ref[i, cs] = scale / (t + 1) * (a @ k[:t + 1, cs])
+    dq = dqkv[0, rows, :C]
+    assert np.abs(dq - dq_ref).max() <= 5e-2 * np.abs(dq_ref).max(), np.abs(dq - dq_ref).max()
