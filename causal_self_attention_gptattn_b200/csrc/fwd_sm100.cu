@@ -57,11 +57,12 @@ template <int HS, bool kDropout>
 struct FwdCfg {
     // warp 0 producer, warp 1 MMA issuer, eight softmax warps from kSoftBase on; with
     // dropout, warps 12-15 draw the mask and registers move by setmaxnreg (launch: 128)
-    static constexpr int kThreads = kDropout ? 512 : 320;
-    static constexpr int kSoftBase = kDropout ? 4 : 2;
-    static constexpr int kLaunchRegs = 128;
-    static constexpr uint32_t kRegsCtl = 96, kRegsSoftmax = 192, kRegsMask = 32;
-    static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsMask == 4 * kLaunchRegs, "register split");
+    static constexpr int kThreads = kDropout ? 512 : 384;
+    static constexpr int kSoftBase = 4;
+    static constexpr int kLaunchRegs = kDropout ? 128 : 168;
+    static constexpr uint32_t kRegsCtl = kDropout ? 96 : 104, kRegsSoftmax = kDropout ? 192 : 200,
+                              kRegsMask = kDropout ? 32 : 0;
+    static_assert(kRegsCtl + 2 * kRegsSoftmax + kRegsMask == (kThreads / 128) * kLaunchRegs, "register split");
     static constexpr int kSlabs = HS / 64;
     static constexpr uint32_t kTileBytes = 128u * HS * 2u;
     static constexpr int kQStages = (HS == 64) ? 2 : 1;   // pairs of Q tiles
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(FwdCfg<HS, kDropout>::kThreads, 1)
     griddep_wait();  // the previous kernel's outputs (qkv, y, lse, dy, workspace) are complete
 
     if (warp < K::kSoftBase) {
-        if constexpr (kDropout) regs_dec<K::kRegsCtl>();
+        regs_dec<K::kRegsCtl>();
     if (warp == 0) {
         // ================================================================ producer
         if (lane == 0) {
@@ -312,7 +313,7 @@ __global__ void __launch_bounds__(FwdCfg<HS, kDropout>::kThreads, 1)
     }
     } else if (warp < K::kSoftBase + 8) {
         // ================================================================ softmax warpgroups
-        if constexpr (kDropout) regs_inc<K::kRegsSoftmax>();
+        regs_inc<K::kRegsSoftmax>();
         const int t = (warp - K::kSoftBase) >> 2;  // tile stream: 0 = A, 1 = B
         const int sp = warp & 3;                 // TMEM sub-partition this warp may access
         const int row = sp * 32 + lane;          // query row within the tile
@@ -358,68 +359,130 @@ __global__ void __launch_bounds__(FwdCfg<HS, kDropout>::kThreads, 1)
                 const bool diag = (j == qt);
                 const bool edge = j <= j_edge;
                 const int cut = (qt - j) * kTile + row - window;  // on an edge tile, columns <= cut are masked
-                // pass 1: row maximum
-                float mx = -INFINITY;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t sr[32];
-                    tmem_ld_x32(tS + 32 * ch, sr);
-                    if (diag) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
-                    }
-                    if (kBand && edge) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (32 * ch + c <= cut) sr[c] = __float_as_uint(-INFINITY);
-                    }
-                    float a = __uint_as_float(sr[0]), bb = __uint_as_float(sr[1]);
-#pragma unroll
-                    for (int c = 2; c < 32; c += 2) a = fmax3(a, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                    mx = fmax3(mx, a, bb);
-                }
-                // lazy max: keep the reference unless it grows by more than 8 (log2 units)
-                const float m_cand = mx * scale_log2;
-                const bool grow = m_cand > mrow + 8.f;
-                const float m_new = grow ? m_cand : mrow;
-                const float alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
-                // a row with no visible key yet (band edge) keeps weight 0, not NaN
-                const float m_use = (kBand && m_new == -INFINITY) ? 0.f : m_new;
-                const uint64_t negm2 = f32x2_pack(-m_use, -m_use);
-                // pass 2: weights, sums, P back into TMEM (bf16 pairs over columns already read)
                 uint64_t sum2 = f32x2_pack(0.f, 0.f), sumr2 = f32x2_pack(0.f, 0.f);
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t sr[32];
-                    tmem_ld_x32(tS + 32 * ch, sr);
+                float m_new, alpha;
+                if constexpr (!kDropout) {
+                    // one pass: the whole S row into registers (four loads in flight, one wait),
+                    // masked, its max, then the weights written back over its first 64 columns
+                    uint32_t sr[128];
+                    tmem_ld_x32_nowait(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld_x32_nowait(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                    tmem_ld_x32_nowait(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                    tmem_ld_x32_nowait(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+                    tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                    tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                    tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+                    tmem_ld_wait_32(*reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
                     if (diag) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 128; ++c)
+                            if (c > row) sr[c] = __float_as_uint(-INFINITY);
                     }
                     if (kBand && edge) {
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (32 * ch + c <= cut) sr[c] = __float_as_uint(-INFINITY);
+                        for (int c = 0; c < 128; ++c)
+                            if (c <= cut) sr[c] = __float_as_uint(-INFINITY);
                     }
-                    uint32_t pk[16];
+                    float mp[8];  // eight independent max chains of 16 columns
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
-                        float x0, x1;
-                        f32x2_unpack(x, x0, x1);
-                        const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-                        const uint32_t wv = pack_bf16x2(p0, p1);
-                        // with dropout the stored weights are masked, the sums are not
-                        if constexpr (kDropout)
-                            pk[c >> 1] = wv & keep_pair_mask(kb[ch] << (c >> 2), (c >> 1) & 1);
-                        else
+                    for (int q = 0; q < 8; ++q) mp[q] = __uint_as_float(sr[16 * q]);
+#pragma unroll
+                    for (int c = 1; c < 15; c += 2)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            mp[q] = fmax3(mp[q], __uint_as_float(sr[16 * q + c]), __uint_as_float(sr[16 * q + c + 1]));
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) mp[q] = fmaxf(mp[q], __uint_as_float(sr[16 * q + 15]));
+                    const float mx =
+                        fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+                    const float m_cand = mx * scale_log2;
+                    const bool grow = m_cand > mrow + 8.f;
+                    m_new = grow ? m_cand : mrow;
+                    alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
+                    // a row with no visible key yet (band edge) keeps weight 0, not NaN
+                    const float m_use = (kBand && m_new == -INFINITY) ? 0.f : m_new;
+                    const uint64_t negm2 = f32x2_pack(-m_use, -m_use);
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const uint64_t x = ffma2(
+                                f32x2_pack(__uint_as_float(sr[32 * ch + c]), __uint_as_float(sr[32 * ch + c + 1])), c2,
+                                negm2);
+                            float x0, x1;
+                            f32x2_unpack(x, x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const uint32_t wv = pack_bf16x2(p0, p1);
                             pk[c >> 1] = wv;
-                        sum2 = fadd2(sum2, f32x2_pack(p0, p1));
-                        sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                            sum2 = fadd2(sum2, f32x2_pack(p0, p1));
+                            sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                        }
+                        tmem_st_x16(tS + 16 * ch, pk);
                     }
-                    tmem_st_x16(tS + 16 * ch, pk);
+                } else {
+                    // pass 1: row maximum
+                    float mx = -INFINITY;
+    #pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t sr[32];
+                        tmem_ld_x32(tS + 32 * ch, sr);
+                        if (diag) {
+    #pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
+                        }
+                        if (kBand && edge) {
+    #pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (32 * ch + c <= cut) sr[c] = __float_as_uint(-INFINITY);
+                        }
+                        float a = __uint_as_float(sr[0]), bb = __uint_as_float(sr[1]);
+    #pragma unroll
+                        for (int c = 2; c < 32; c += 2) a = fmax3(a, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                        mx = fmax3(mx, a, bb);
+                    }
+                    // lazy max: keep the reference unless it grows by more than 8 (log2 units)
+                    const float m_cand = mx * scale_log2;
+                    const bool grow = m_cand > mrow + 8.f;
+                    m_new = grow ? m_cand : mrow;
+                    alpha = grow ? ex2_approx(mrow - m_new) : 1.f;
+                    // a row with no visible key yet (band edge) keeps weight 0, not NaN
+                    const float m_use = (kBand && m_new == -INFINITY) ? 0.f : m_new;
+                    const uint64_t negm2 = f32x2_pack(-m_use, -m_use);
+                    // pass 2: weights, sums, P back into TMEM (bf16 pairs over columns already read)
+    #pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t sr[32];
+                        tmem_ld_x32(tS + 32 * ch, sr);
+                        if (diag) {
+    #pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (32 * ch + c > row) sr[c] = __float_as_uint(-INFINITY);
+                        }
+                        if (kBand && edge) {
+    #pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                if (32 * ch + c <= cut) sr[c] = __float_as_uint(-INFINITY);
+                        }
+                        uint32_t pk[16];
+    #pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            const uint64_t x = ffma2(f32x2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), c2, negm2);
+                            float x0, x1;
+                            f32x2_unpack(x, x0, x1);
+                            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+                            const uint32_t wv = pack_bf16x2(p0, p1);
+                            // with dropout the stored weights are masked, the sums are not
+                            if constexpr (kDropout)
+                                pk[c >> 1] = wv & keep_pair_mask(kb[ch] << (c >> 2), (c >> 1) & 1);
+                            else
+                                pk[c >> 1] = wv;
+                            sum2 = fadd2(sum2, f32x2_pack(p0, p1));
+                            sumr2 = fadd2(sumr2, f32x2_pack(bf16lo_to_f32(wv), bf16hi_to_f32(wv)));
+                        }
+                        tmem_st_x16(tS + 16 * ch, pk);
+                    }
                 }
                 float s0, s1, r0, r1;
                 f32x2_unpack(sum2, s0, s1);
@@ -513,7 +576,7 @@ cudaError_t launch_fwd_variant(const CUtensorMap &map_qkv, const CUtensorMap &ma
     auto kern = fwd_bf16_kernel<HS, kBand, kDropout>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::kSmemBytes);
     if (e != cudaSuccess) return e;
-    if constexpr (kDropout) {
+    {
         // the warpgroups' register budgets add up to the launch allocation only at kLaunchRegs
         // per thread; otherwise a setmaxnreg.inc could never be satisfied, so refuse to launch
         cudaFuncAttributes fa{};
