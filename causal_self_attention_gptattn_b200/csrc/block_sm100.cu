@@ -293,32 +293,39 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16 *__r
     const int n8 = C / 8;
     const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)row * C);
     uint4 buf[kLnMaxPerLane];
-    float sum = 0.f;
+    // bf16 pair -> the two floats, packed for the paired fp32 instructions
+    auto pair = [](uint32_t u) { return f32x2_pack(bf16lo_to_f32(u), bf16hi_to_f32(u)); };
+    uint64_t sum2 = f32x2_pack(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane; ++k) {
         const int i = lane + 32 * k;
         buf[k] = i < n8 ? xr[i] : make_uint4(0u, 0u, 0u, 0u);
-        const uint32_t u[4] = {buf[k].x, buf[k].y, buf[k].z, buf[k].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sum += bf16lo_to_f32(u[e]) + bf16hi_to_f32(u[e]);
+        sum2 = fadd2(sum2, fadd2(fadd2(pair(buf[k].x), pair(buf[k].y)), fadd2(pair(buf[k].z), pair(buf[k].w))));
     }
+    float s0, s1;
+    f32x2_unpack(sum2, s0, s1);
+    float sum = s0 + s1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float mean = sum / (float)C;
-    float sq = 0.f;
+    const uint64_t negmean2 = f32x2_pack(-mean, -mean);
+    uint64_t sq2 = f32x2_pack(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < kLnMaxPerLane; ++k) {
         if (lane + 32 * k >= n8) continue;
         const uint32_t u[4] = {buf[k].x, buf[k].y, buf[k].z, buf[k].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float a = bf16lo_to_f32(u[e]) - mean, c = bf16hi_to_f32(u[e]) - mean;
-            sq += a * a + c * c;
+            const uint64_t d = fadd2(pair(u[e]), negmean2);
+            sq2 = ffma2(d, d, sq2);
         }
     }
+    f32x2_unpack(sq2, s0, s1);
+    float sq = s0 + s1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
     const float rstd = rsqrtf(sq / (float)C + 1e-5f);
+    const uint64_t rstd2 = f32x2_pack(rstd, rstd);
     const uint4 *wr = reinterpret_cast<const uint4 *>(w), *br = reinterpret_cast<const uint4 *>(b);
     uint4 *orow = reinterpret_cast<uint4 *>(out + (size_t)row * C);
 #pragma unroll
@@ -330,9 +337,14 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const __nv_bfloat16 *__r
         const uint32_t wu[4] = {wq.x, wq.y, wq.z, wq.w}, bu[4] = {bq.x, bq.y, bq.z, bq.w};
         uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[e] = pack_bf16x2((bf16lo_to_f32(u[e]) - mean) * rstd * bf16lo_to_f32(wu[e]) + bf16lo_to_f32(bu[e]),
-                               (bf16hi_to_f32(u[e]) - mean) * rstd * bf16hi_to_f32(wu[e]) + bf16hi_to_f32(bu[e]));
+        for (int e = 0; e < 4; ++e) {
+            // (x - mean) * rstd * w + b as x * a + c with a = rstd * w, c = b - mean * a
+            const uint64_t a = fmul2(rstd2, pair(wu[e]));
+            const uint64_t c = ffma2(negmean2, a, pair(bu[e]));
+            float lo, hi;
+            f32x2_unpack(ffma2(pair(u[e]), a, c), lo, hi);
+            o[e] = pack_bf16x2(lo, hi);
+        }
         orow[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
