@@ -299,14 +299,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int st1 = (gi + 1) % kQStages;
                         const bool more = it + 1 < niter;
                         const uint32_t ph = (uint32_t)gi & 1u;
+                        // The barriers this tile waits on have usually completed by the time this
+                        // thread reaches them (it is the one that falls behind: it shares its
+                        // sub-partition's issue slots with three busy warps, and every dependent
+                        // round trip costs it hundreds of cycles).  So all of them are tested at
+                        // once, and a blocking wait runs only for one that was still open.  A
+                        // completed phase stays completed until this thread's own later MMAs let
+                        // the next phase complete, so a set bit cannot go stale.
+                        const uint32_t r1 = mbar_test4(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u,
+                                                       bar(kBarSEmpty), ph, bar(kBarPFull), ph, bar(kBardPEmpty), ph);
                         if (more) {  // S^T of the next query tile
-                            if (!(ok = mbar_wait(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u, g))) break;
-                            if (!(ok = mbar_wait(bar(kBarSEmpty), ph, g))) break;
+                            if (!(r1 & 1u) &&
+                                !(ok = mbar_wait(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u, g)))
+                                break;
+                            if (!(r1 & 2u) && !(ok = mbar_wait(bar(kBarSEmpty), ph, g))) break;
                             tc_fence_after();
                             issue_S(kvs, st1);
                         }
                         // dV += P^T dO
-                        if (!(ok = mbar_wait(bar(kBarPFull), ph, g))) break;
+                        if (!(r1 & 4u) && !(ok = mbar_wait(bar(kBarPFull), ph, g))) break;
                         if (it == 0 && n > 0 && !(ok = mbar_wait(bar(kBarAccFree), (uint32_t)(n - 1) & 1u, g))) break;
                         tc_fence_after();
                         {
@@ -320,12 +331,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // dP^T of the next query tile, ahead of this tile's dK and dQ (which wait for
                         // this tile's dS), so the softmax warps find it ready when they reach it
                         if (more) {
-                            if (!(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
+                            if (!(r1 & 8u) && !(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
                             tc_fence_after();
                             issue_dP(kvs, st1);
                         }
-                        // dK += dS^T Q ; dQ = dS K
-                        if (!(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
+                        // dK += dS^T Q ; dQ = dS K  (gi = 0 tests the phase before the first, which
+                        // counts as complete)
+                        const uint32_t r2 = mbar_test4(bar(kBardSFull), ph, bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u,
+                                                       bar(kBardSFull), ph, bar(kBardSFull), ph);
+                        if (!(r2 & 1u) && !(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
                         tc_fence_after();
                         {
                             const uint64_t b = at(dQmn0, st * kTileBytes);
@@ -337,7 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         // dK was the last reader of Q_i and dO_i (dQ reads dS and K): release their stage
                         umma_commit(bar(kBarQEmpty + st));
-                        if (gi > 0 && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
+                        if (gi > 0 && !(r2 & 2u) && !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g)))
+                            break;
                         tc_fence_after();
                         {
                             const uint64_t b = at(dKmn0, kvs * kTileBytes);

@@ -70,6 +70,35 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking tests of four phases at once: bit k of the result is set when
+// barrier k's phase of the given parity has completed.  One instruction
+// sequence with no dependence between the tests, so a thread that polls
+// several barriers pays one shared-memory round trip instead of four.
+__device__ __forceinline__ uint32_t mbar_test4(uint32_t b0, uint32_t p0, uint32_t b1, uint32_t p1, uint32_t b2,
+                                               uint32_t p2, uint32_t b3, uint32_t p3) {
+    uint32_t m;
+    asm volatile(
+        "{\n"
+        ".reg .pred q0, q1, q2, q3;\n"
+        ".reg .b32 t1, t2, t3;\n"
+        "mbarrier.test_wait.parity.shared::cta.b64 q0, [%1], %2;\n"
+        "mbarrier.test_wait.parity.shared::cta.b64 q1, [%3], %4;\n"
+        "mbarrier.test_wait.parity.shared::cta.b64 q2, [%5], %6;\n"
+        "mbarrier.test_wait.parity.shared::cta.b64 q3, [%7], %8;\n"
+        "selp.u32 %0, 1, 0, q0;\n"
+        "selp.u32 t1, 2, 0, q1;\n"
+        "selp.u32 t2, 4, 0, q2;\n"
+        "selp.u32 t3, 8, 0, q3;\n"
+        "or.b32 %0, %0, t1;\n"
+        "or.b32 t2, t2, t3;\n"
+        "or.b32 %0, %0, t2;\n"
+        "}\n"
+        : "=r"(m)
+        : "r"(b0), "r"(p0), "r"(b1), "r"(p1), "r"(b2), "r"(p2), "r"(b3), "r"(p3)
+        : "memory");
+    return m;
+}
+
 // Every wait inside the kernels goes through this context: a CTA-wide abort
 // flag in shared memory, the device status word, and a time budget.
 struct WaitGuard {
