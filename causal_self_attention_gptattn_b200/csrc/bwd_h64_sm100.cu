@@ -95,8 +95,7 @@ constexpr int kBardPEmpty = kBardPFull + 1;
 constexpr int kBarPFull = kBardPEmpty + 1;
 constexpr int kBarPEmpty = kBarPFull + 1;
 constexpr int kBardSFull = kBarPEmpty + 1;
-constexpr int kBardSEmpty = kBardSFull + 1;
-constexpr int kBardQFull = kBardSEmpty + 1;
+constexpr int kBardQFull = kBardSFull + 1;  // dQ_i done; also frees the dS buffer (dK_i ran before it)
 constexpr int kBardQEmpty = kBardQFull + 1;
 constexpr int kBarKdV = kBardQEmpty + 1;
 constexpr int kBarAccFree = kBarKdV + 1;
@@ -181,7 +180,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(kBarPFull), kSoftmaxThreads);
         mbar_init(bar(kBarPEmpty), 1);
         mbar_init(bar(kBardSFull), kSoftmaxThreads);
-        mbar_init(bar(kBardSEmpty), 1);
         mbar_init(bar(kBardQFull), 1);
         mbar_init(bar(kBardQEmpty), kDrainThreads);
         mbar_init(bar(kBarKdV), 1);
@@ -264,6 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
                 bool ok = true, any = false;
                 int n = 0, gi = 0;
+                int qst = 0;        // gi % kQStages, kept incrementally (no divisions on this thread)
+                uint32_t qpar = 0;  // (gi / kQStages) & 1
                 auto issue_S = [&](int kvs, int st) {
                     const uint64_t a = at(dK0, kvs * kTileBytes), b = at(dQ0, st * kTileBytes);
     #pragma unroll
@@ -286,17 +286,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int kvs = n & 1;
                     if (!(ok = mbar_wait(bar(kBarKVFull + kvs), (uint32_t)(n >> 1) & 1u, g))) break;
                     // first S and dP of this item
-                    if (!(ok = mbar_wait(bar(kBarQFull + gi % kQStages), (uint32_t)(gi / kQStages) & 1u, g))) break;
+                    if (!(ok = mbar_wait(bar(kBarQFull + qst), qpar, g))) break;
                     if (gi > 0 && !(ok = mbar_wait(bar(kBarSEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
                     tc_fence_after();
-                    issue_S(kvs, gi % kQStages);
+                    issue_S(kvs, qst);
                     any = true;
                     if (gi > 0 && !(ok = mbar_wait(bar(kBardPEmpty), (uint32_t)(gi - 1) & 1u, g))) break;
                     tc_fence_after();
-                    issue_dP(kvs, gi % kQStages);
+                    issue_dP(kvs, qst);
                     for (int it = 0; it < niter; ++it, ++gi) {
-                        const int st = gi % kQStages;
-                        const int st1 = (gi + 1) % kQStages;
+                        const int st = qst;
+                        const int st1 = qst == kQStages - 1 ? 0 : qst + 1;
+                        const uint32_t qpar1 = qst == kQStages - 1 ? qpar ^ 1u : qpar;  // parity of tile gi + 1
                         const bool more = it + 1 < niter;
                         const uint32_t ph = (uint32_t)gi & 1u;
                         // The barriers this tile waits on have usually completed by the time this
@@ -306,12 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // once, and a blocking wait runs only for one that was still open.  A
                         // completed phase stays completed until this thread's own later MMAs let
                         // the next phase complete, so a set bit cannot go stale.
-                        const uint32_t r1 = mbar_test4(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u,
-                                                       bar(kBarSEmpty), ph, bar(kBarPFull), ph, bar(kBardPEmpty), ph);
+                        const uint32_t r1 = mbar_test4(bar(kBarQFull + st1), qpar1, bar(kBarSEmpty), ph, bar(kBarPFull),
+                                                       ph, bar(kBardPEmpty), ph);
                         if (more) {  // S^T of the next query tile
-                            if (!(r1 & 1u) &&
-                                !(ok = mbar_wait(bar(kBarQFull + st1), (uint32_t)((gi + 1) / kQStages) & 1u, g)))
-                                break;
+                            if (!(r1 & 1u) && !(ok = mbar_wait(bar(kBarQFull + st1), qpar1, g))) break;
                             if (!(r1 & 2u) && !(ok = mbar_wait(bar(kBarSEmpty), ph, g))) break;
                             tc_fence_after();
                             issue_S(kvs, st1);
@@ -360,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int kk = 0; kk < 8; ++kk)
                                 umma_ss(tmem + kColdQ, at(ddSmn, kk * 2048u), at(b, kk * 2048u), idQ, kk > 0 ? 1u : 0u);
                         }
-                        umma_commit(bar(kBardQFull));
-                        umma_commit(bar(kBardSEmpty));
+                        umma_commit(bar(kBardQFull));  // dQ_i retired, and dK_i before it: dS free
+                        qst = st1;
+                        qpar = qpar1;
                     }
                     if (!ok) break;
                     umma_commit(bar(kBarKdV));
@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (ok) ok = warp_wait(bar(kBardPFull), ph, g);
-                if (ok && gi > 0) ok = warp_wait(bar(kBardSEmpty), (uint32_t)(gi - 1) & 1u, g);
+                if (ok && gi > 0) ok = warp_wait(bar(kBardQFull), (uint32_t)(gi - 1) & 1u, g);  // dS buffer free
                 if (ok) {
                     tc_fence_after();
                     const float4 *D4 = reinterpret_cast<const float4 *>(sD + st * 128 + 64 * half);
