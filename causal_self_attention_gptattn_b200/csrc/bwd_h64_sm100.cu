@@ -100,11 +100,19 @@ constexpr int kBardQEmpty = kBardQFull + 1;
 constexpr int kBarKdV = kBardQEmpty + 1;
 constexpr int kBarAccFree = kBarKdV + 1;
 constexpr int kBarDone = kBarAccFree + 1;
-constexpr int kBarMFull = kBarDone + 1;          // kMStages
+constexpr int kBarDoneB = kBarDone + 1;          // second issuer's last MMAs retired
+constexpr int kBarMFull = kBarDoneB + 1;         // kMStages
 constexpr int kBarMEmpty = kBarMFull + kMStages;  // kMStages
 constexpr int kNumBars = kBarMEmpty + kMStages;
 static_assert(kNumBars * 8 + 16 <= kBarArea, "barrier area");
 constexpr int kMaskThreads = 64;
+// MMA issuers.  Without dropout a second thread (warp 2) issues the gradient products dK and dQ
+// while warp 1 issues S, dV and dP: a lone issuing thread shares its sub-partition's issue slots
+// with three busy warps and runs a few times slower than the tensor pipe it feeds.  With dropout
+// warps 2 and 3 draw the keep words and warp 1 issues everything.  Buffers that both issuers'
+// products read are released by a commit from each (barrier count = number of issuers).
+template <bool kDropout>
+constexpr uint32_t kIssuers = kDropout ? 1u : 2u;
 
 constexpr int kSoftmaxThreads = 256;
 constexpr int kDrainThreads = 128;
@@ -167,11 +175,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kKVStages; ++s) {
             mbar_init(bar(kBarKVFull + s), 1);
-            mbar_init(bar(kBarKVEmpty + s), 1);
+            mbar_init(bar(kBarKVEmpty + s), kIssuers<kDropout>);
         }
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(bar(kBarQFull + s), 1);
-            mbar_init(bar(kBarQEmpty + s), 1);
+            mbar_init(bar(kBarQEmpty + s), kIssuers<kDropout>);
         }
         mbar_init(bar(kBarSFull), 1);
         mbar_init(bar(kBarSEmpty), kSoftmaxThreads);
@@ -182,9 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(kBardSFull), kSoftmaxThreads);
         mbar_init(bar(kBardQFull), 1);
         mbar_init(bar(kBardQEmpty), kDrainThreads);
-        mbar_init(bar(kBarKdV), 1);
+        mbar_init(bar(kBarKdV), kIssuers<kDropout>);
         mbar_init(bar(kBarAccFree), kDrainThreads);
         mbar_init(bar(kBarDone), 1);
+        mbar_init(bar(kBarDoneB), 1);
         for (int s = 0; s < kMStages; ++s) {
             mbar_init(bar(kBarMFull + s), kMaskThreads);
             mbar_init(bar(kBarMEmpty + s), kSoftmaxThreads);
@@ -327,12 +336,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 umma_ts(tmem + kColdV, tmem + kColP + 8u * kk, at(b, kk * 2048u), idAcc, kk > 0 ? 1u : acc);
                         }
                         umma_commit(bar(kBarPEmpty));
+                        // this issuer's reads of Q_i and dO_i (S_i, dP_i, dV_i) are done
+                        if constexpr (!kDropout) umma_commit(bar(kBarQEmpty + st));
                         // dP^T of the next query tile, ahead of this tile's dK and dQ (which wait for
                         // this tile's dS), so the softmax warps find it ready when they reach it
                         if (more) {
                             if (!(r1 & 8u) && !(ok = mbar_wait(bar(kBardPEmpty), ph, g))) break;
                             tc_fence_after();
                             issue_dP(kvs, st1);
+                        }
+                        if constexpr (!kDropout) {
+                            qst = st1;
+                            qpar = qpar1;
+                            continue;  // dK and dQ come from the second issuer
                         }
                         // dK += dS^T Q ; dQ = dS K  (gi = 0 tests the phase before the first, which
                         // counts as complete)
@@ -373,6 +389,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         } else {
+            if constexpr (!kDropout) {
+                // ================================================================ second MMA issuer (warp 2)
+                if (warp == 2 && lane == 0) {
+                    constexpr uint32_t idAcc = idesc_bf16_f32(128, HS, false, true);
+                    constexpr uint32_t idQ = idesc_bf16_f32(128, HS, true, true);
+                    const uint64_t dQmn0 = sdesc_sw128(sQ(0), kSlabBytes, 1024);
+                    const uint64_t dKmn0 = sdesc_sw128(sK(0), kSlabBytes, 1024);
+                    const uint64_t ddS = sdesc_sw128(sdS, 16, 1024), ddSmn = sdesc_sw128(sdS, kSlabBytes, 1024);
+                    auto at = [](uint64_t d, uint32_t bytes) -> uint64_t { return d + (uint64_t)(bytes >> 4); };
+                    bool ok = true, any = false;
+                    int n = 0, gi = 0, qst = 0;
+                    uint32_t qpar = 0;
+                    for (int k = 0; ok; ++k, ++n) {
+                        const int w = item_index(k, blockIdx.x, gridDim.x);
+                        if (w >= n_items) break;
+                        const int kt = w / BH;
+                        const int niter = band_hi_tile(kt, window, n_t) - kt + 1;
+                        const int kvs = n & 1;
+                        if (!(ok = mbar_wait(bar(kBarKVFull + kvs), (uint32_t)(n >> 1) & 1u, g))) break;
+                        for (int it = 0; it < niter; ++it, ++gi) {
+                            const int st = qst;
+                            const uint32_t ph = (uint32_t)gi & 1u;
+                            // one batch of tests, a blocking wait only for a phase still open; none of
+                            // these phases can be overtaken before this thread's own later commits
+                            // (gi = 0 / n = 0 test the phase before the first, which counts as complete)
+                            const uint32_t r = mbar_test4(bar(kBardSFull), ph, bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u,
+                                                          bar(kBarQFull + st), qpar, bar(kBarAccFree),
+                                                          (uint32_t)(n - 1) & 1u);
+                            if (!(r & 4u) && !(ok = mbar_wait(bar(kBarQFull + st), qpar, g))) break;
+                            if (!(r & 1u) && !(ok = mbar_wait(bar(kBardSFull), ph, g))) break;
+                            if (it == 0 && n > 0 && !(r & 8u) &&
+                                !(ok = mbar_wait(bar(kBarAccFree), (uint32_t)(n - 1) & 1u, g)))
+                                break;
+                            tc_fence_after();
+                            any = true;
+                            {  // dK += dS^T Q
+                                const uint64_t b = at(dQmn0, st * kTileBytes);
+                                const uint32_t acc = it > 0 ? 1u : 0u;
+    #pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    umma_ss(tmem + kColdK, at(ddS, (kk >> 2) * kSlabBytes + (kk & 3) * 32u),
+                                            at(b, kk * 2048u), idAcc, kk > 0 ? 1u : acc);
+                            }
+                            umma_commit(bar(kBarQEmpty + st));  // this issuer's read of Q_i is done
+                            if (gi > 0 && !(r & 2u) &&
+                                !(ok = mbar_wait(bar(kBardQEmpty), (uint32_t)(gi - 1) & 1u, g)))
+                                break;
+                            tc_fence_after();
+                            {  // dQ = dS K
+                                const uint64_t b = at(dKmn0, kvs * kTileBytes);
+    #pragma unroll
+                                for (int kk = 0; kk < 8; ++kk)
+                                    umma_ss(tmem + kColdQ, at(ddSmn, kk * 2048u), at(b, kk * 2048u), idQ,
+                                            kk > 0 ? 1u : 0u);
+                            }
+                            umma_commit(bar(kBardQFull));  // dQ_i retired, and dK_i before it: dS free
+                            qst = qst == kQStages - 1 ? 0 : qst + 1;
+                            qpar = qst == 0 ? qpar ^ 1u : qpar;
+                        }
+                        if (!ok) break;
+                        umma_commit(bar(kBarKdV));
+                        umma_commit(bar(kBarKVEmpty + kvs));
+                    }
+                    if (any) {
+                        umma_commit(bar(kBarDoneB));
+                        drain_wait(bar(kBarDoneB), 0, budget_ns);
+                    }
+                }
+            }
             // ================================================================ dropout mask (warps 2, 3)
             if constexpr (kDropout) {
                 // thread -> key rows 4*kg .. 4*kg+3 and query columns 64*qh .. 64*qh+63 of every
