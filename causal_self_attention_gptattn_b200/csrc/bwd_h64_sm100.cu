@@ -28,14 +28,18 @@
 // first warpgroup to the last):
 //   warp 0        TMA producer: K_j, V_j (double-buffered across items), and
 //                 Q_i, dO_i, lse_i, D_i through a 3-stage ring
-//   warp 1        TMEM owner + MMA issuer (warps 2, 3 idle)
+//   warp 1        TMEM owner + MMA issuer of S, dP, dV (with dropout: of all five)
+//   warp 2        MMA issuer of dK, dQ (without dropout; with it, warps 2-3 draw
+//                 the dropout keep words)
 //   warps 4..11   softmax: TMEM sub-partition warp%4 (32 key rows), column
 //                 half warp/4 - 1 (64 query columns): P^T, dS^T
 //   warps 12..15  dQ drain: TMEM -> smem (fp32, swizzled) -> TMA reduce-add;
 //                 and per item the dK/dV epilogue (TMEM -> bf16 -> TMA store)
 // TMEM (512 columns): S^T [0,128)  dP^T [128,256)  P^T [256,320) (bf16 pairs)
 //                     dV [320,384)  dK [384,448)  dQ [448,512)
-// MMA order per item: S_0 dP_0 | S_1 dV_0 dP_1 dK_0 dQ_0 | S_2 dV_1 dP_2 ...
+// MMA order per item: S_0 dP_0 | S_1 dV_0 dP_1 | S_2 dV_1 dP_2 ... on warp 1, and
+// dK_i dQ_i on warp 2 as soon as dS_i is written (with dropout warp 1 issues them
+// after dP_{i+1}).
 // S^T and dP^T are released as soon as the softmax warps hold them in
 // registers, so the tensor pipe computes tile i+1 while tile i is in softmax.
 // Every wait is bounded; roles never leave their loops early, so all named
