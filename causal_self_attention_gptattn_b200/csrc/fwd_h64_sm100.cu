@@ -184,6 +184,11 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
                     mbar_arrive_expect_tx(qb, (hasB ? 2u : 1u) * kTileBytes);
                     for (int t = 0; t < (hasB ? 2 : 1); ++t)
                         tma_load_3d(sQ(qs, t), &map_qkv, qb, h * HS, (2 * m + t) * kTile, b);
+                    // Without a tile B the stage's release counts one arrival for it, made here: the
+                    // wait above has just seen the stage's previous phase complete, so the arrival
+                    // falls into this item's phase.  (Made by tile B's idle warpgroup instead, it could
+                    // run several such items ahead and arrive into a phase still open for tile A.)
+                    if (!hasB) mbar_arrive(bar(kBarQEmpty + qs));
                     ++nq;
                     for (int j = 0; j < nkv; ++j) {
                         const int st = gkv % kKVStages;
@@ -319,10 +324,7 @@ __global__ void __launch_bounds__(FwdCfg<kDropout>::kThreads, 1)
             const int b = bh / n_head, h = bh % n_head;
             const int qt = 2 * m + t;
             const int qs = n % kQStages;
-            if (qt >= n_qt) {
-                if (leader) mbar_arrive(bar(kBarQEmpty + qs));
-                continue;
-            }
+            if (qt >= n_qt) continue;  // no tile B in this item (the producer released its share of the stage)
             const int jlo_t = band_lo_tile(qt, window);
             // key tiles at or below this one need the band's lower edge masked
             const int j_edge = (qt * kTile + kTile - 1 - window) / kTile;

@@ -191,6 +191,11 @@ __global__ void __launch_bounds__(FwdCfg<HS, kDropout>::kThreads, 1)
                 for (int t = 0; t < (hasB ? 2 : 1); ++t)
                     for (int s = 0; s < K::kSlabs; ++s)
                         tma_load_3d(sQ(qs, t) + s * kSlabBytes, &map_qkv, qb, h * HS + 64 * s, (2 * m + t) * kTile, b);
+                // Without a tile B the stage's release counts one arrival for it, made here: the
+                // wait above has just seen the stage's previous phase complete, so the arrival falls
+                // into this item's phase.  (Made by tile B's idle warpgroup instead, it could run
+                // several such items ahead and arrive into a phase still open for tile A.)
+                if (!hasB) mbar_arrive(bar(K::kBarQEmpty + qs));
                 ++nq;
                 for (int j = 0; j < nkv; ++j) {
                     const int st = gkv % K::kKVStages;
@@ -333,11 +338,7 @@ __global__ void __launch_bounds__(FwdCfg<HS, kDropout>::kThreads, 1)
             const int b = bh / n_head, h = bh % n_head;
             const int qt = 2 * m + t;
             const int qs = n % K::kQStages;
-            if (qt >= n_qt) {
-                // this tile stream has no work in this item; release its share of the Q stage
-                if (leader) mbar_arrive(bar(K::kBarQEmpty + qs));
-                continue;
-            }
+            if (qt >= n_qt) continue;  // no work for this stream in this item (the producer released its share)
             const int jlo_t = kBand ? band_lo_tile(qt, window) : 0;
             // key tiles at or below j_edge need the band's lower edge masked (a band narrower
             // than T: query t sees keys t-window < s <= t)

@@ -131,6 +131,16 @@ def test_bf16_many_short_sequences():
 
 
 @pytest.mark.parametrize("hs", [64, 128])
+def test_bf16_odd_tile_count_many_items(hs):
+    """T = 300 (three query tiles, so every item of the last pair has no second tile) with
+    B * n_head = 200 pairs: on 148 SMs a CTA gets two such items in a row, the case in which
+    the warpgroup without a tile must not release a shared Q stage ahead of the other."""
+    qkv, dy = make_inputs(20, 300, 10, hs, dtype=torch.bfloat16, seed=300 + hs)
+    got = run_fwd_bwd(qkv, dy, 10)
+    compare(got, oracle_all(qkv, dy, 10), torch.bfloat16, f"200 x 300, hs={hs}")
+
+
+@pytest.mark.parametrize("hs", [64, 128])
 def test_bf16_max_length_closed_form(hs):
     """T = 16384 (128 query tiles per (b, h)) against closed forms instead of the oracle: with
     q = 0 every score is 0, so each weight is 1/(t+1) and
